@@ -1,0 +1,451 @@
+"""Benchmark of the trellis-coded MoE routed-expert path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload moe_decode_t16]
+
+A step is one pass of the whole hot path over one batch: route_topk -> route_permute ->
+hadamard128 -> moe_trellis_gemv (gate/up+SiLU, rotation of h, down) -> route_unpermute,
+for one 384-expert layer (D = 4096, F = 1024, mixed widths 368/15/1 experts at
+K = 2/3/4) and 16 tokens with top-8 routing.  Four such layers (independent synthetic
+weights and inputs) are cycled so that a weight byte is re-read only after ~1.4 GB of
+other weights: every step reads its ~0.35 GB of touched bit streams from HBM, not L2.
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank runs an independent
+replica (the path has no exchange step); value = all ranks' tokens / max-over-ranks time.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed-expert tok/s per MoE layer; GEMV HBM GB/s and GEMM tensor-pipe % of peak"
+N_LAYER_COPIES = 4
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="moe_decode_t16", choices=["moe_decode_t16"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def csrc_digest():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "trellis_quantized_moe_gemv_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(name):
+    """DRAM bytes per launch recorded by an ncu capture (profiles/<name>.txt), or None
+    when missing or taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", name + ".txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    with open(path) as f:
+        for line in f:
+            if "=" in line and not line.lstrip().startswith("#"):
+                k, v = line.split("=", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("csrc_digest") != csrc_digest() or "dram_bytes_per_unit" not in kv:
+        return None
+    return kv
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML every 10 ms."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.time(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return None
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if not inside:
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            window = "nearest to the timed region (region shorter than the sampling period)"
+        if not inside:
+            return None
+        reasons = set()
+        for _, _, rs in inside:
+            for bit, name in self.REASONS.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(inside), "window": window}
+
+
+# ----------------------------------------------------------------------------- workload
+
+def build_decode_workload(api, inputs, torch, device, rank):
+    """Layer copy 0 from the seeded numpy generators (the copy the parity tests check);
+    copies 1..3 with the same widths, their bit streams and scales drawn on the device
+    from a seeded torch generator; every copy has its own tokens and logits."""
+    w0 = inputs.moe_decode_t16(seed=1003 + 100 * rank)
+    host_layer = w0["layer"]
+    layers, xs, logits = [], [], []
+    layers.append(api.DeviceLayer.from_synthetic(host_layer, device))
+    gen = torch.Generator(device=device)
+    for c in range(1, N_LAYER_COPIES):
+        gen.manual_seed(7000 + 100 * rank + c)
+        groups = []
+        for g in host_layer.groups:
+            def rbits(shape):
+                return torch.randint(-2 ** 31, 2 ** 31 - 1, shape, dtype=torch.int32, device=device,
+                                     generator=gen)
+
+            def rscale(shape):
+                return (torch.rand(shape, device=device, generator=gen) + 0.5).to(torch.float16)
+            groups.append(dict(K=g.K, ids=g.ids, gate=rbits(g.gate.shape), up=rbits(g.up.shape),
+                               down=rbits(g.down.shape), s_gate=rscale(g.s_gate.shape),
+                               s_up=rscale(g.s_up.shape), s_down=rscale(g.s_down.shape)))
+        layers.append(api.DeviceLayer(host_layer.E, host_layer.D, host_layer.F, groups, device))
+    for c in range(N_LAYER_COPIES):
+        rng = np.random.default_rng(9000 + 100 * rank + c)
+        x = w0["x"] if c == 0 else inputs.random_activations(rng, (16, host_layer.D), "bf16")
+        lg = w0["logits"] if c == 0 else inputs.normal_logits(rng, 16, host_layer.E)
+        xs.append((x, lg))
+    return w0, layers, xs
+
+
+def gateup_algorithmic_bytes(layer, counts):
+    """Algorithmic bytes of one gate/up GEMV launch: the touched experts' gate and up bit
+    streams (K/8 B per weight) and scales, their tokens' rotated activations read once
+    per expert, and h written (fp32)."""
+    K_of = {}
+    for g in layer.groups:
+        for e in g["ids"].tolist():
+            K_of[e] = g["K"]
+    total = 0
+    for e, n in enumerate(counts):
+        if n == 0:
+            continue
+        total += 2 * layer.F * layer.D * K_of[e] // 8 + 2 * layer.F * 2
+        total += n * layer.D * 2 + n * layer.F * 4
+    return total
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from trellis_quantized_moe_gemv_b200 import api, inputs
+    from trellis_quantized_moe_gemv_b200 import build as tqbuild
+
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if rank == 0:
+        tqbuild.build()
+    if world > 1:
+        dist.barrier()
+    api.lib()
+
+    T, k = 16, 8
+    w0, layers, xs = build_decode_workload(api, inputs, torch, device, rank)
+    E, D, F = layers[0].E, layers[0].D, layers[0].F
+    bufs = [api.MoeBuffers(L, T, k) for L in layers]
+    x_dev = [torch.from_numpy(x).to(torch.bfloat16).to(device) for x, _ in xs]
+    l_dev = [torch.from_numpy(lg).to(device) for _, lg in xs]
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        c = i % N_LAYER_COPIES
+        api.moe_layer(layers[c], x_dev[c], l_dev[c], k, bufs=bufs[c], path="gemv")
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    api.device_status(clear=True)
+
+    # ---- device-timed region
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    api.profile_enable(16 * (args.steps + 1))
+    api.profile_collect()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = api.launch_count()
+    t_wall0 = time.time()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    launches = api.launch_count() - launches0
+    stages = api.profile_collect()
+    api.profile_disable()
+    sampler.stop()
+    ms_total = ev0.elapsed_time(ev1)
+    flags = api.device_status()
+    if flags:
+        raise RuntimeError("device anomaly flags %d during the timed region" % flags)
+
+    ms_max = ms_total
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+
+    # ---- algorithmic bytes of the dominant kernel (gate/up GEMV) per launch
+    counts = [b.routing.counts.cpu().numpy() for b in bufs]
+    per_copy_bytes = [gateup_algorithmic_bytes(L, c) for L, c in zip(layers, counts)]
+    gu_bytes = sum(per_copy_bytes[i % N_LAYER_COPIES] for i in range(args.steps)) / max(args.steps, 1)
+    gu_ms, gu_n = stages["gemv_gateup"]
+    gu_avg_ms = gu_ms / max(gu_n, 1)
+    peaks, peak_src = load_peaks()
+    achieved = gu_bytes / (gu_avg_ms * 1e-3) / 1e9
+    prof = profile_traffic("moe_gemv_gateup_decode_t16")
+    traffic = None
+    if prof is not None:
+        unit_bytes = float(prof["dram_bytes_per_unit"])
+        units = sum(int((c > 0).sum()) for c in counts) / N_LAYER_COPIES
+        traffic = unit_bytes * units
+
+    # ---- end to end through the public API with host buffers
+    pin_x = [torch.from_numpy(x).to(torch.bfloat16).pin_memory() for x, _ in xs]
+    pin_l = [torch.from_numpy(lg).pin_memory() for _, lg in xs]
+    pin_out = torch.empty((T, D), dtype=torch.float32).pin_memory()
+
+    def e2e_step(i):
+        c = i % N_LAYER_COPIES
+        x_dev[c].copy_(pin_x[c], non_blocking=True)
+        l_dev[c].copy_(pin_l[c], non_blocking=True)
+        out = api.moe_layer(layers[c], x_dev[c], l_dev[c], k, bufs=bufs[c], path="gemv")
+        pin_out.copy_(out, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = T * D * 2 + T * E * 4
+    d2h = T * D * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w0, routes=16)
+
+    tokens = T * args.steps * world
+    line = {
+        "metric": METRIC,
+        "value": tokens / (ms_max * 1e-3),
+        "unit": "tok/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic",
+        "config": {
+            "workload": "moe_decode_t16", "experts": E, "hidden": D, "intermediate": F,
+            "tokens": T, "top_k": k, "widths": "368/15/1 experts at K=2/3/4",
+            "layer_copies_cycled": N_LAYER_COPIES,
+            "l2": "inputs larger than L2: each step reads ~0.35 GB of bit streams; 4 layers "
+                  "(4.9 GB) cycled",
+            "path": "gemv", "parallelism": "replicas" if world > 1 else "single-gpu",
+        },
+        "roofline": {
+            "kernel": "moe_gateup_kernel (gate/up GEMV + SiLU)",
+            "bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]),
+            "unit": "GB/s", "frac": achieved / float(peaks["hbm_gbs"]),
+            "peak_source": peak_src, "bytes_per_launch": gu_bytes,
+            "avg_launch_ms": gu_avg_ms, "traffic": traffic,
+        },
+        "stages_ms_per_step": {k_: v[0] / max(args.steps, 1) for k_, v in stages.items() if v[1]},
+        "gpu_launches": launches,
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": sampler.summary(t_wall0, t_wall1),
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def cpu_baseline(w0, routes):
+    """The fp64 CPU oracle, as it stands, on `routes` (token, expert) routes of layer
+    copy 0 (single-threaded BLAS); reported in tok/s (k routes = one token)."""
+    from oracle import layer as OL
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=1)
+    except Exception:
+        limiter = None
+    layer, x, logits, k = w0["layer"], w0["x"], w0["logits"], w0["k"]
+    ids, wts = OL.route_topk(logits, k)
+    weights = OL.ExpertWeights(layer)
+    t0 = time.time()
+    done = 0
+    for t in range(x.shape[0]):
+        xr = OL.rotate(x[t:t + 1].astype(np.float64))
+        for s in range(k):
+            OL.expert_forward(weights, int(ids[t, s]), xr)
+            done += 1
+            if done >= routes:
+                break
+        if done >= routes:
+            break
+    dt = time.time() - t0
+    if limiter is not None:
+        limiter.unregister()
+    return {"value": (done / k) / dt, "unit": "tok/s", "cores": 1, "kind": "oracle",
+            "sample": "%d routes (= %d tokens x top-%d) of the 384-expert decode layer, fp64 "
+                      "scalar-C decode + numpy, %.1f s" % (done, done // k, k, dt)}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step is one (token, expert) route of the
+    decode layer, decoded and computed in fp64 on the host; value in tok/s."""
+    if rank != 0:
+        return
+    from oracle import layer as OL
+    from trellis_quantized_moe_gemv_b200 import inputs
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(limits=1)
+    except Exception:
+        pass
+    w0 = inputs.moe_decode_t16()
+    layer, x, logits, k = w0["layer"], w0["x"], w0["logits"], w0["k"]
+    ids, _ = OL.route_topk(logits, k)
+    routes = [(t, s) for t in range(x.shape[0]) for s in range(k)]
+
+    def step(i):
+        t, s = routes[i % len(routes)]
+        weights = OL.ExpertWeights(layer)   # no decode reuse across steps
+        OL.expert_forward(weights, int(ids[t, s]), OL.rotate(x[t:t + 1].astype(np.float64)))
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.time()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.time() - t0
+    value = (args.steps / k) / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "moe_decode_t16", "experts": 384, "hidden": 4096,
+                   "intermediate": 1024, "tokens": 16, "top_k": k,
+                   "widths": "368/15/1 experts at K=2/3/4"},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": 1, "kind": "oracle",
+                         "sample": "one (token, expert) route per step = 1/%d token" % k},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank, world, local_rank = dist_env()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

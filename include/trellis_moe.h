@@ -1,0 +1,240 @@
+/*
+ * trellis_moe.h -- C ABI of the B200 (sm_100a) library for the routed-expert matrix
+ * multiply of a trellis-coded quantised mixture-of-experts layer.
+ *
+ * The method (web pages on T16 / TrellisMX / exlr8 trellis-coded DeepSeek experts):
+ *   "DeepSeek-V4.1-Flash-1017 · dsx T16", section "How T16 works":
+ *     - experts quantised with a QTIP-style bitshift trellis and 128-wide Hadamard
+ *       rotations (section intro);
+ *     - item 1, the T16 codebook: a weight's value comes from its 16-bit window of the
+ *       bit stream, multiplied by 0x3A2F (16 bits), plus the product's two bytes;
+ *     - item 2: column-major positions inside each 16 x 16 tile;
+ *     - item 4: each output channel's stored scale.
+ *   same card, "October 25 runtime checkpoint": warp Hadamard transforms, fixed-bit
+ *     weight expansion, fused gate/up post-processing of the routed experts;
+ *   "DeepSeek-V4.1-Flash-1017 TrellisMX K2 Mix", "What is stored": one tensor group per
+ *     width present in a layer, each with its ascending global expert ids; "Status":
+ *     each width's routes bit-identical to the single-width kernels, full CUDA-graph
+ *     replay with changing routes.
+ *
+ * Stored format (readings where the pages are silent):
+ *   - A matrix of R x C weights (R = output channels, C = inputs; both multiples of 16)
+ *     is (R/16) x (C/16) tiles in row-major tile order; tile (i, j) holds rows
+ *     16i..16i+15 and columns 16j..16j+15 and is 8*K little-endian uint32 words
+ *     (exactly 256*K bits, K = 2, 3 or 4 bits per weight).
+ *   - Stream bit b of a tile is bit (b mod 32) of its word b/32.  The weight at tile
+ *     position p (row p mod 16, column p div 16) takes the 16-bit window whose bit i is
+ *     stream bit (p*K + i) mod 256K (tail-biting inside the tile).
+ *   - t = lo + hi, the two unsigned bytes of (window * 0x3A2F) mod 2^16; code c = t - 255.
+ *   - W[r][col] = s[r] * 2^-12 * c[r][col], s the fp16 per-output-channel scale.
+ *   - A projection's input is rotated first: x' = (1/sqrt(128)) * H_128 x on every
+ *     contiguous 128-chunk, H_128 the natural-order Sylvester matrix.
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers to memory the caller owns (e.g. PyTorch
+ *     tensors), unless stated otherwise.  The library allocates nothing, keeps no
+ *     pointer after the call returns, and never synchronises the host: work is enqueued
+ *     on `stream` (a cudaStream_t; NULL means the legacy default stream).
+ *   - fp16 / bf16 buffers are passed as uint16_t bit patterns.
+ *   - Return value: TQ_OK, or a tq_status error.  Argument errors are detected on the
+ *     host before anything is enqueued; TQ_ERR_CUDA reports a launch error.  Device-side
+ *     anomalies (an out-of-range id met by a kernel, a bounded wait that gave up) never
+ *     trap: the kernel skips the work and raises a flag readable by tq_device_status().
+ *   - No C++ exception crosses this ABI.  Every entry point is usable inside CUDA-graph
+ *     capture: none reads device data on the host or synchronises.
+ *   - Sizes of zero (T = 0, rows = 0) are valid no-ops returning TQ_OK.
+ */
+#ifndef TRELLIS_MOE_H
+#define TRELLIS_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TQ_ABI_VERSION 1
+
+typedef enum {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1,     /* a size, width, count or pointer is invalid        */
+    TQ_ERR_UNSUPPORTED = 2,     /* valid but outside what this build implements      */
+    TQ_ERR_ALIGNMENT = 3,       /* a pointer is not aligned as documented            */
+    TQ_ERR_WORKSPACE = 4,       /* workspace missing or smaller than required         */
+    TQ_ERR_CUDA = 5,            /* a CUDA launch or runtime call failed               */
+    TQ_ERR_DEVICE_TIMEOUT = 6   /* a kernel's bounded wait gave up (device flag)      */
+} tq_status;
+
+typedef enum { TQ_DTYPE_F16 = 0, TQ_DTYPE_BF16 = 1, TQ_DTYPE_F32 = 2 } tq_dtype;
+
+typedef void *tq_stream; /* cudaStream_t */
+
+/* Human-readable name of a status code (static string; never NULL). */
+const char *tq_status_string(int status);
+
+/* TQ_ABI_VERSION of the loaded library. */
+int tq_abi_version(void);
+
+/*
+ * Device-side anomaly flags of the current device, OR-ed since the last clear:
+ *   bit 0: a kernel met an expert id outside [0, E) or a route index outside [0, T*k)
+ *          and skipped that work;
+ *   bit 1: a bounded wait inside a kernel gave up (the kernel returned early).
+ * Reads the flag word with a synchronous copy (not for use inside graph capture);
+ * `clear` != 0 resets it.  Writes the flags to *flags_out (host pointer).
+ */
+int tq_device_status(int32_t *flags_out, int clear);
+
+/*
+ * Launch accounting and per-stage timing of the library's own kernels (tracing; no
+ * counterpart on the pages).  Every kernel launch increments a host counter.  While
+ * profiling is enabled, each launch is bracketed by two CUDA events recorded on its
+ * stream and tagged with its stage:
+ *   0 route_topk, 1 route_permute, 2 hadamard128 of the input, 3 GEMV gate/up+SiLU,
+ *   4 rotation of h, 5 GEMV down, 6 route_unpermute, 7 trellis_decode, 8 trellis_gemv,
+ *   9 GEMM gate/up+SiLU, 10 GEMM down.
+ * tq_profile_enable creates 2*max_launches events (host-side CUDA resources; call it
+ * outside graph capture, and do not capture while it is enabled); launches beyond
+ * max_launches are not recorded.  tq_profile_collect waits for the recorded events,
+ * writes per-stage summed milliseconds and launch counts into the host arrays
+ * stage_ms[n_stages] / stage_launches[n_stages], and clears the record.
+ */
+unsigned long long tq_launch_count(void);
+int tq_profile_enable(int max_launches);
+int tq_profile_disable(void);
+int tq_profile_collect(double *stage_ms, int32_t *stage_launches, int n_stages);
+
+/*
+ * trellis_decode -- standalone T16 decode to dense codes ("fixed-bit weight
+ * expansion", dsx T16 card, "October 25 runtime checkpoint"; codebook and tile order
+ * from "How T16 works", items 1 and 2).
+ *   bits : [rows/16][cols/16][8K] uint32, 16-byte aligned.
+ *   out  : [rows][cols] fp16, row-major, 16-byte aligned; out[r][c] = c_rc = t - 255
+ *          (an integer in [-255, 255], exact in fp16).  Scales are not applied.
+ *   rows, cols: multiples of 16.  K in {2, 3, 4}.
+ */
+int trellis_decode(const uint32_t *bits, int K, int rows, int cols, uint16_t *out,
+                   tq_stream stream);
+
+/*
+ * hadamard128 -- x' = (1/sqrt(128)) * H_128 x on every contiguous 128-chunk of each
+ * row ("128-wide Hadamard rotations", dsx T16 card "How T16 works"; "warp Hadamard
+ * transforms", its "October 25 runtime checkpoint").  Computed in fp32, rounded to fp16.
+ *   x    : [rows][cols] of x_dtype (F16, BF16 or F32), row-major, 16-byte aligned.
+ *   out  : [rows][cols] fp16, row-major, 16-byte aligned.  May not alias x.
+ *   cols : a multiple of 128.
+ */
+int hadamard128(const void *x, int x_dtype, int64_t rows, int64_t cols, uint16_t *out,
+                tq_stream stream);
+
+/*
+ * trellis_gemv -- one trellis-coded matrix times a small batch of rotated activations:
+ *   y[b][r] = s[r] * 2^-12 * sum_c code[r][c] * x_rot[b][c]
+ * (the projection of "How T16 works", items 1, 2 and 4, on decode-sized batches).
+ *   bits   : [rows/16][cols/16][8K] uint32, 16-byte aligned.
+ *   scales : [rows] fp16.
+ *   x_rot  : [batch][cols] fp16 (already rotated, e.g. by hadamard128), 16-byte aligned.
+ *   y      : [batch][rows] fp32.
+ *   rows % 16 == 0, cols % 128 == 0, 0 <= batch <= 256, K in {2, 3, 4}.
+ */
+int trellis_gemv(const uint32_t *bits, const uint16_t *scales, int K, int rows, int cols,
+                 const uint16_t *x_rot, int batch, float *y, tq_stream stream);
+
+/*
+ * route_topk -- top-k experts of every token and their route weights ("top-8 softmax
+ * routing"): ids sorted by decreasing logit, ties to the lower expert id; weights are
+ * the softmax of the k kept logits (fp32, expf).  NaN logits are not supported.
+ *   logits   : [T][E] fp32.   topk_ids : [T][k] int32.   topk_w : [T][k] fp32.
+ *   1 <= k <= 32, k <= E <= 1024.
+ */
+int route_topk(const float *logits, int T, int E, int k, int32_t *topk_ids, float *topk_w,
+               tq_stream stream);
+
+/*
+ * route_permute -- group the T*k (token, slot) routes by expert ("per-width tensor
+ * groups, each with its ascending global expert_ids", TrellisMX K2 Mix card, "What is
+ * stored"; grouping is stable in route order).  Route index i = t*k + s.
+ *   topk_ids  : [T*k] int32, each in [0, E) (out-of-range ids: flag bit 0, route dropped).
+ *   counts    : [E] int32     routes per expert.
+ *   offsets   : [E+1] int32   exclusive prefix sum of counts.
+ *   perm      : [T*k] int32   route indices sorted by (expert, route index).
+ *   inv       : [T*k] int32   inv[perm[j]] = j.
+ *   active_ids: [E] int32     experts with counts > 0, ascending (rest untouched).
+ *   n_active  : [1] int32     number of such experts.
+ *   1 <= E <= 1024.  Deterministic; one CTA.
+ */
+int route_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *counts,
+                  int32_t *offsets, int32_t *perm, int32_t *inv, int32_t *active_ids,
+                  int32_t *n_active, tq_stream stream);
+
+/*
+ * route_unpermute -- combine: out[t][d] = sum_{s=0..k-1} topk_w[t][s] * y_perm[inv[t*k+s]][d],
+ * summed in slot order in fp32 (deterministic, no atomics).
+ *   y_perm : [T*k][D] fp32 in expert-grouped order.  inv, topk_w : [T*k].
+ *   out    : [T][D] fp32.  D % 4 == 0; y_perm and out 16-byte aligned.
+ */
+int route_unpermute(const float *y_perm, const int32_t *inv, const float *topk_w, int T, int k,
+                    int D, float *out, tq_stream stream);
+
+/* One width group of a layer: experts of one K, concatenated in ascending global id. */
+typedef struct {
+    int K;                       /* 2, 3 or 4 bits per weight                          */
+    int n_experts;               /* experts in the group                               */
+    const int32_t *expert_ids;   /* device [n_experts], ascending global ids           */
+    const uint32_t *gate;        /* device [n_experts][F/16][D/16][8K] words           */
+    const uint32_t *up;          /* device [n_experts][F/16][D/16][8K] words           */
+    const uint32_t *down;        /* device [n_experts][D/16][F/16][8K] words           */
+    const uint16_t *s_gate;      /* device fp16 [n_experts][F]                         */
+    const uint16_t *s_up;        /* device fp16 [n_experts][F]                         */
+    const uint16_t *s_down;      /* device fp16 [n_experts][D]                         */
+} tq_width_group;
+
+/* A trellis-coded MoE layer: E experts of hidden size D and intermediate size F. */
+typedef struct {
+    int E, D, F;                 /* D % 128 == 0, F % 128 == 0                         */
+    int n_groups;                /* 1..3 width groups                                  */
+    tq_width_group groups[3];
+    const int32_t *expert_slot;  /* device [E]: (group << 16) | index in group, or -1  */
+} tq_moe_layer;
+
+/*
+ * Workspace bytes moe_trellis_gemv / moe_trellis_gemm need for T tokens and k routes:
+ * the SwiGLU activations h of every route ([T*k][F] fp32) and their rotation h'
+ * ([T*k][F] fp16), 256-byte aligned.  Returns 0 on invalid arguments.
+ */
+size_t moe_trellis_workspace_size(const tq_moe_layer *layer, int T, int k);
+
+/*
+ * moe_trellis_gemv -- the routed experts of one MoE layer for decode-sized batches
+ * (the SwiGLU expert with fused gate/up post-processing, "October 25 runtime
+ * checkpoint" of the dsx T16 card, on T16 weights, "How T16 works"):
+ *   for every route i (expert e = expert of route i, token t = perm[i] / k):
+ *     g = W_gate[e] x'_t,  u = W_up[e] x'_t,  h = silu(g) * u,
+ *     h' = rotate128(h),   y_perm[i] = W_down[e] h'
+ *   x_rot    : [T][D] fp16 rotated tokens (hadamard128 of the layer input).
+ *   offsets, perm, active_ids, n_active : from route_permute (device).
+ *   y_perm   : [T*k][D] fp32, expert-grouped route order.
+ *   ws       : device workspace of at least moe_trellis_workspace_size() bytes.
+ *   Mixed widths run in one launch per stage; routes of an expert are processed
+ *   together, each weight decoded once per 16 of its routes.
+ */
+int moe_trellis_gemv(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
+                     const int32_t *perm, const int32_t *active_ids, const int32_t *n_active,
+                     int T, int k, float *y_perm, void *ws, size_t ws_bytes, tq_stream stream);
+
+/*
+ * moe_trellis_gemm -- same result as moe_trellis_gemv for prefill-sized batches: the
+ * bit streams are decoded to fp16 operands of tcgen05 tensor-core MMAs (accumulating
+ * in tensor memory), each weight decoded once per 128 routes of its expert.
+ * Same arguments and workspace as moe_trellis_gemv.
+ */
+int moe_trellis_gemm(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
+                     const int32_t *perm, const int32_t *active_ids, const int32_t *n_active,
+                     int T, int k, float *y_perm, void *ws, size_t ws_bytes, tq_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRELLIS_MOE_H */

@@ -126,6 +126,18 @@ def route_permute(topk_ids, E: int):
     return counts, offsets, perm, inv
 
 
+def combine(y_perm, inv, topk_w):
+    """out[t] = sum_s w[t, s] * y_perm[inv[t*k + s]], summed in slot order (fp64)."""
+    y = np.asarray(y_perm, dtype=np.float64)
+    w = np.asarray(topk_w, dtype=np.float64)
+    T, k = w.shape
+    inv = np.asarray(inv).reshape(T, k)
+    out = np.zeros((T, y.shape[1]))
+    for s in range(k):
+        out += w[:, s:s + 1] * y[inv[:, s]]
+    return out
+
+
 # ----------------------------------------------------------------------------- experts
 
 def silu(z):

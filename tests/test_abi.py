@@ -1,0 +1,124 @@
+"""The C-ABI library loads, exports every entry point include/*.h declares, and rejects
+invalid arguments on the host before anything is enqueued (no GPU needed)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+import trellis_quantized_moe_gemv_b200.build as tqbuild
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tqbuild.build()
+    from trellis_quantized_moe_gemv_b200 import api
+    return api.lib()
+
+
+def declared_functions():
+    names = set()
+    for path in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(path).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w]*\s*\**\s*\**\s*([A-Za-z_]\w*)\s*\(",
+                             text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("trellis_decode", "hadamard128", "trellis_gemv", "route_topk", "route_permute",
+                     "route_unpermute", "moe_trellis_gemv", "moe_trellis_gemm",
+                     "moe_trellis_workspace_size", "tq_status_string", "tq_abi_version",
+                     "tq_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_abi_version_and_status_strings(lib):
+    from trellis_quantized_moe_gemv_b200 import api
+    assert api.abi_version() == 1
+    for code in range(7):
+        assert lib.tq_status_string(code)
+    assert b"ALIGNMENT" in lib.tq_status_string(3)
+    assert lib.tq_status_string(99) == b"unknown tq_status"
+
+
+FAKE = ctypes.c_void_p(0x10000)        # 16-byte aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p(0x10004)
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    # widths, shapes
+    assert lib.trellis_decode(FAKE, 5, 16, 16, FAKE, None) == 1
+    assert lib.trellis_decode(FAKE, 2, 15, 16, FAKE, None) == 1
+    assert lib.trellis_decode(None, 2, 16, 16, FAKE, None) == 1
+    assert lib.trellis_decode(MISALIGNED, 2, 16, 16, FAKE, None) == 3
+    assert lib.trellis_decode(FAKE, 2, 0, 16, FAKE, None) == 0          # empty: no-op
+    assert lib.hadamard128(FAKE, 0, 4, 100, FAKE, None) == 1            # cols % 128
+    assert lib.hadamard128(FAKE, 7, 4, 128, FAKE, None) == 1            # dtype
+    assert lib.hadamard128(MISALIGNED, 0, 4, 128, FAKE, None) == 3
+    assert lib.hadamard128(FAKE, 0, 0, 128, FAKE, None) == 0
+    assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 64, FAKE, 1, FAKE, None) == 1   # cols % 128
+    assert lib.trellis_gemv(FAKE, FAKE, 1, 16, 128, FAKE, 1, FAKE, None) == 1  # K
+    assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 128, FAKE, 257, FAKE, None) == 1
+    assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 128, FAKE, 0, FAKE, None) == 0
+    assert lib.route_topk(FAKE, 4, 384, 0, FAKE, FAKE, None) == 1
+    assert lib.route_topk(FAKE, 4, 4, 8, FAKE, FAKE, None) == 1         # k > E
+    assert lib.route_topk(FAKE, 0, 384, 8, FAKE, FAKE, None) == 0
+    assert lib.route_permute(FAKE, 4, 8, 2000, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert lib.route_unpermute(FAKE, FAKE, FAKE, 4, 8, 6, FAKE, None) == 1
+    assert lib.route_unpermute(MISALIGNED, FAKE, FAKE, 4, 8, 8, FAKE, None) == 3
+
+
+def _layer_struct(K=2, E=16, D=256, F=128, n_groups=1):
+    from trellis_quantized_moe_gemv_b200 import api
+    st = api.TqMoeLayer()
+    st.E, st.D, st.F, st.n_groups = E, D, F, n_groups
+    for g in range(n_groups):
+        w = st.groups[g]
+        w.K, w.n_experts = K, E
+        for key in ("expert_ids", "gate", "up", "down", "s_gate", "s_up", "s_down"):
+            setattr(w, key, 0x10000)
+    st.expert_slot = 0x10000
+    return st
+
+
+def test_moe_workspace_and_layer_validation(lib):
+    st = _layer_struct()
+    need = lib.moe_trellis_workspace_size(ctypes.byref(st), 16, 8)
+    assert need == 128 * 128 * 4 + 128 * 128 * 2
+    bad = _layer_struct(K=5)
+    assert lib.moe_trellis_workspace_size(ctypes.byref(bad), 16, 8) == 0
+    bad = _layer_struct(D=200)
+    assert lib.moe_trellis_workspace_size(ctypes.byref(bad), 16, 8) == 0
+    args = [FAKE] * 5
+    # workspace too small
+    assert lib.moe_trellis_gemv(ctypes.byref(st), *args, 16, 8, FAKE, FAKE, need - 1, None) == 4
+    assert lib.moe_trellis_gemv(ctypes.byref(st), *args, 16, 8, FAKE, None, need, None) == 4
+    # misaligned activations
+    assert lib.moe_trellis_gemv(ctypes.byref(st), MISALIGNED, *args[1:], 16, 8, FAKE, FAKE, need,
+                                None) == 3
+    # T = 0 is a no-op
+    assert lib.moe_trellis_gemv(ctypes.byref(st), *args, 0, 8, FAKE, FAKE, 0, None) == 0
+    # misaligned bit streams
+    mis = _layer_struct()
+    mis.groups[0].gate = 0x10004
+    assert lib.moe_trellis_gemv(ctypes.byref(mis), *args, 16, 8, FAKE, FAKE, need, None) == 3
+
+
+def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
+    from trellis_quantized_moe_gemv_b200 import api
+    monkeypatch.setattr(api, "_lib", None)
+    monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(api.TQError):
+        api.lib()

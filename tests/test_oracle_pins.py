@@ -255,6 +255,16 @@ def test_permute_invariants():
         assert np.all(flat[seg] == e) and np.all(np.diff(seg) > 0)
 
 
+def test_combine_closed_forms():
+    # k = 1 with unit weights is a pure gather; equal weights 1/k give the mean.
+    rng = np.random.default_rng(4)
+    y = rng.standard_normal((6, 5))
+    inv = np.array([3, 0, 5, 1, 4, 2])
+    np.testing.assert_array_equal(L.combine(y, inv, np.ones((6, 1))), y[inv])
+    out = L.combine(y, np.arange(6), np.full((3, 2), 0.5))
+    np.testing.assert_allclose(out, 0.5 * (y[0::2] + y[1::2]), rtol=1e-15)
+
+
 # ----------------------------------------------------------------------------- expert
 
 def test_silu_identities():

@@ -1,0 +1,111 @@
+// Status codes, version and the device anomaly flag word of the C ABI.
+#include "tq_common.cuh"
+
+TQ_API const char *tq_status_string(int status) {
+    switch (status) {
+        case TQ_OK: return "TQ_OK";
+        case TQ_ERR_INVALID_ARG: return "TQ_ERR_INVALID_ARG: invalid size, width, count or pointer";
+        case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED: outside what this build implements";
+        case TQ_ERR_ALIGNMENT: return "TQ_ERR_ALIGNMENT: pointer not aligned as documented";
+        case TQ_ERR_WORKSPACE: return "TQ_ERR_WORKSPACE: workspace missing or too small";
+        case TQ_ERR_CUDA: return "TQ_ERR_CUDA: CUDA launch or runtime error";
+        case TQ_ERR_DEVICE_TIMEOUT: return "TQ_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
+        default: return "unknown tq_status";
+    }
+}
+
+TQ_API int tq_abi_version(void) { return TQ_ABI_VERSION; }
+
+TQ_API int tq_device_status(int32_t *flags_out, int clear) {
+    if (!flags_out) return TQ_ERR_INVALID_ARG;
+    if (cudaMemcpyFromSymbol(flags_out, tq::g_device_flags, sizeof(int32_t)) != cudaSuccess)
+        return TQ_ERR_CUDA;
+    if (clear) {
+        const int32_t zero = 0;
+        if (cudaMemcpyToSymbol(tq::g_device_flags, &zero, sizeof(int32_t)) != cudaSuccess)
+            return TQ_ERR_CUDA;
+    }
+    return TQ_OK;
+}
+
+// ---------------------------------------------------------------------------- profiling
+namespace tq {
+
+struct Profiler {
+    bool on = false;
+    int capacity = 0;
+    int used = 0;
+    cudaEvent_t *events = nullptr;   // 2 per recorded launch
+    int *stage = nullptr;
+};
+static Profiler g_prof;
+static unsigned long long g_launches = 0;
+
+LaunchScope::LaunchScope(cudaStream_t s, int st) : stream(s), slot(-1) {
+    ++g_launches;
+    if (g_prof.on && g_prof.used < g_prof.capacity) {
+        slot = g_prof.used++;
+        g_prof.stage[slot] = st;
+        cudaEventRecord(g_prof.events[2 * slot], s);
+    }
+}
+
+LaunchScope::~LaunchScope() {
+    if (slot >= 0) cudaEventRecord(g_prof.events[2 * slot + 1], stream);
+}
+
+static void profile_release() {
+    for (int i = 0; i < 2 * g_prof.capacity; ++i) cudaEventDestroy(g_prof.events[i]);
+    delete[] g_prof.events;
+    delete[] g_prof.stage;
+    g_prof = Profiler();
+}
+
+}  // namespace tq
+
+TQ_API unsigned long long tq_launch_count(void) { return tq::g_launches; }
+
+TQ_API int tq_profile_enable(int max_launches) {
+    if (max_launches < 1 || max_launches > (1 << 20)) return TQ_ERR_INVALID_ARG;
+    tq::profile_release();
+    tq::g_prof.events = new cudaEvent_t[2 * (size_t)max_launches];
+    tq::g_prof.stage = new int[max_launches];
+    for (int i = 0; i < 2 * max_launches; ++i) {
+        if (cudaEventCreate(&tq::g_prof.events[i]) != cudaSuccess) {
+            tq::g_prof.capacity = i / 2;
+            tq::profile_release();
+            return TQ_ERR_CUDA;
+        }
+    }
+    tq::g_prof.capacity = max_launches;
+    tq::g_prof.on = true;
+    return TQ_OK;
+}
+
+TQ_API int tq_profile_disable(void) {
+    tq::profile_release();
+    return TQ_OK;
+}
+
+TQ_API int tq_profile_collect(double *stage_ms, int32_t *stage_launches, int n_stages) {
+    if (!stage_ms || !stage_launches || n_stages < 1) return TQ_ERR_INVALID_ARG;
+    for (int i = 0; i < n_stages; ++i) {
+        stage_ms[i] = 0.0;
+        stage_launches[i] = 0;
+    }
+    if (!tq::g_prof.on) return TQ_OK;
+    for (int l = 0; l < tq::g_prof.used; ++l) {
+        if (cudaEventSynchronize(tq::g_prof.events[2 * l + 1]) != cudaSuccess) return TQ_ERR_CUDA;
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, tq::g_prof.events[2 * l], tq::g_prof.events[2 * l + 1]) !=
+            cudaSuccess)
+            return TQ_ERR_CUDA;
+        const int st = tq::g_prof.stage[l];
+        if (st >= 0 && st < n_stages) {
+            stage_ms[st] += ms;
+            stage_launches[st] += 1;
+        }
+    }
+    tq::g_prof.used = 0;
+    return TQ_OK;
+}

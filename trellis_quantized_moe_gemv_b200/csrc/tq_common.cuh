@@ -1,0 +1,90 @@
+// Shared device/host helpers of the sm_100a trellis-MoE library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "trellis_moe.h"
+
+#define TQ_API extern "C" __attribute__((visibility("default")))
+
+namespace tq {
+
+// T16 codebook multiplier ("How T16 works", item 1 of the dsx T16 card).
+constexpr uint32_t kT16Mult = 0x3A2Fu;
+// Decoded codes are t - 255 with t = byte0 + byte1 of the product.
+constexpr int kCentre = 255;
+// Fixed normaliser of every code: W = s * 2^-12 * c.
+constexpr float kKappa = 1.0f / 4096.0f;
+constexpr float kInvSqrt128 = 0.08838834764831845f;
+
+// Device flag word (bit 0: bad id skipped, bit 1: bounded wait gave up).  The library
+// is one translation unit (tq_library.cu), so this is its only definition.
+__device__ int32_t g_device_flags = 0;
+
+__device__ __forceinline__ void raise_flag(int32_t bit) { atomicOr(&g_device_flags, bit); }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned8(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+// ---------------------------------------------------------------------------- profiling
+// Stage tags of the library's kernel launches (tq_profile_* in the C ABI).
+enum Stage {
+    kStageTopk = 0, kStagePermute = 1, kStageRotateX = 2, kStageGemvGateUp = 3,
+    kStageRotateH = 4, kStageGemvDown = 5, kStageUnpermute = 6, kStageDecode = 7,
+    kStageGemv = 8, kStageGemmGateUp = 9, kStageGemmDown = 10, kNumStages = 11
+};
+
+// Brackets one kernel launch: counts it and, while profiling is on, records a start
+// and a stop event on the launching stream under the given stage tag.
+struct LaunchScope {
+    LaunchScope(cudaStream_t s, int stage);
+    ~LaunchScope();
+    cudaStream_t stream;
+    int slot;
+};
+
+inline int launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+inline int num_sms() {
+    static int cached = 0;
+    if (cached == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&cached, cudaDevAttrMultiProcessorCount, dev);
+        if (cached <= 0) cached = 148;
+    }
+    return cached;
+}
+
+// ---------------------------------------------------------------------------- PTX wrappers
+
+// Low 32 bits of the 64-bit value (hi:lo) >> sh, sh in [0, 31].
+__device__ __forceinline__ uint32_t funnel_r(uint32_t lo, uint32_t hi, uint32_t sh) {
+    return __funnelshift_r(lo, hi, sh);
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// D = A * B + D,  m16n8k16, fp16 operands, fp32 accumulators (mma.sync register operands).
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
+
+}  // namespace tq

@@ -1,0 +1,278 @@
+// Routing: top-k + softmax, stable expert grouping, and the weighted combine.
+//
+// "top-8 softmax routing" of the routed experts; per-width groups with ascending
+// global expert ids ("DeepSeek-V4.1-Flash-1017 TrellisMX K2 Mix", "What is stored").
+#include "tq_common.cuh"
+
+namespace tq {
+
+constexpr int kTopkMaxPerLane = 32;   // E <= 32 * 32
+
+// One warp per token.  Each lane owns logits e = lane + 32*j.  k rounds of a warp-wide
+// arg-max (larger logit first, ties to the lower id) select the experts in order.
+template <int PER_LANE>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T,
+                                                         int E, int k, int32_t *__restrict__ ids,
+                                                         float *__restrict__ w) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= T) return;
+    const float *row = logits + (size_t)warp * E;
+    float v[PER_LANE];
+#pragma unroll
+    for (int j = 0; j < PER_LANE; ++j) {
+        int e = lane + 32 * j;
+        v[j] = e < E ? row[e] : -INFINITY;
+    }
+    uint32_t taken = 0;  // bit j: v[j] already selected (or absent)
+#pragma unroll
+    for (int j = 0; j < PER_LANE; ++j)
+        if (lane + 32 * j >= E) taken |= 1u << j;
+    float sel_v = 0.f, vmax = 0.f;
+    int sel_e = 0;
+    for (int r = 0; r < k; ++r) {
+        // lane-local best (lowest id among equals: j ascending => id ascending)
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < PER_LANE; ++j) {
+            bool free_slot = !((taken >> j) & 1u);
+            if (free_slot && (v[j] > bv || be == 0x7fffffff)) {
+                bv = v[j];
+                be = lane + 32 * j;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (ov > bv || (ov == bv && oe < be)) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if (r == 0) vmax = bv;
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (lane == r) {
+            sel_v = bv;
+            sel_e = be;
+        }
+    }
+    // softmax over the k kept logits; lane r < k holds the r-th choice
+    float ex = lane < k ? expf(sel_v - vmax) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < k) {
+        ids[(size_t)warp * k + lane] = sel_e;
+        w[(size_t)warp * k + lane] = ex / sum;
+    }
+}
+
+// Stable grouping of routes by expert in one CTA of 1024 threads.  Routes are taken
+// in chunks of 1024 in index order; inside a chunk, a route's rank among equal
+// experts is its rank inside its warp (match.any) plus the counts of the same expert
+// in the chunk's earlier warps, plus the routes of that expert in earlier chunks.
+constexpr int kPermThreads = 1024;
+constexpr int kPermWarps = kPermThreads / 32;
+constexpr int kPermMaxE = 1024;
+
+inline size_t permute_smem_bytes(int E) {
+    return sizeof(int32_t) * ((size_t)(3 + kPermWarps) * E);
+}
+
+__global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
+    const int32_t *__restrict__ topk_ids, int n_routes, int E, int32_t *__restrict__ counts,
+    int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv,
+    int32_t *__restrict__ active_ids, int32_t *__restrict__ n_active) {
+    extern __shared__ int32_t smem[];
+    int32_t *cursor = smem;                 // [E] histogram, then routes placed so far
+    int32_t *base = cursor + E;             // [E] exclusive offsets
+    int32_t *total = base + E;              // [E] routes of the current chunk
+    int32_t *wcnt = total + E;              // [kPermWarps][E] per-warp counts of a chunk
+    __shared__ int32_t warp_sum[kPermWarps], warp_sum_a[kPermWarps];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    for (int e = tid; e < E; e += kPermThreads) cursor[e] = 0;
+    for (int x = tid; x < kPermWarps * E; x += kPermThreads) wcnt[x] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int i = tid; i < n_routes; i += kPermThreads) {
+        int e = topk_ids[i];
+        if (e >= 0 && e < E) atomicAdd(&cursor[e], 1);
+        else bad = true;
+    }
+    if (bad) raise_flag(1);
+    __syncthreads();
+
+    // Exclusive scan of the histogram (one expert per thread) and of "expert active".
+    const int c = tid < E ? cursor[tid] : 0;
+    const int a = c > 0 ? 1 : 0;
+    int incl = c, incl_a = a;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        int t1 = __shfl_up_sync(0xffffffffu, incl, off);
+        int t2 = __shfl_up_sync(0xffffffffu, incl_a, off);
+        if (lane >= off) {
+            incl += t1;
+            incl_a += t2;
+        }
+    }
+    if (lane == 31) {
+        warp_sum[warp] = incl;
+        warp_sum_a[warp] = incl_a;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int s = warp_sum[lane], sa = warp_sum_a[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            int t1 = __shfl_up_sync(0xffffffffu, s, off);
+            int t2 = __shfl_up_sync(0xffffffffu, sa, off);
+            if (lane >= off) {
+                s += t1;
+                sa += t2;
+            }
+        }
+        warp_sum[lane] = s;
+        warp_sum_a[lane] = sa;
+    }
+    __syncthreads();
+    const int prior = warp > 0 ? warp_sum[warp - 1] : 0;
+    const int prior_a = warp > 0 ? warp_sum_a[warp - 1] : 0;
+    if (tid < E) {
+        const int ex = prior + incl - c;
+        base[tid] = ex;
+        offsets[tid] = ex;
+        counts[tid] = c;
+        if (c > 0) active_ids[prior_a + incl_a - 1] = tid;
+        if (tid == E - 1) {
+            offsets[E] = ex + c;
+            *n_active = prior_a + incl_a;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kPermThreads) cursor[e] = 0;
+    __syncthreads();
+
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int chunk = 0; chunk < n_routes; chunk += kPermThreads) {
+        const int i = chunk + tid;
+        const int e = i < n_routes ? topk_ids[i] : -1;
+        const bool valid = e >= 0 && e < E;
+        const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+        const int rank = __popc(peers & lt_mask);
+        const bool leader = lane == 31 - __clz(peers);
+        if (valid && leader) wcnt[warp * E + e] = __popc(peers);
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += kPermThreads) {
+            int run = 0;
+            for (int w = 0; w < kPermWarps; ++w) {
+                const int v = wcnt[w * E + ee];
+                wcnt[w * E + ee] = run;
+                run += v;
+            }
+            total[ee] = run;
+        }
+        __syncthreads();
+        if (valid) {
+            const int dst = base[e] + cursor[e] + wcnt[warp * E + e] + rank;
+            perm[dst] = i;
+            inv[i] = dst;
+        } else if (i < n_routes) {
+            inv[i] = -1;
+        }
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += kPermThreads) cursor[ee] += total[ee];
+        for (int x = tid; x < kPermWarps * E; x += kPermThreads) wcnt[x] = 0;
+        __syncthreads();
+    }
+}
+
+// out[t][d] = sum_s w[t][s] * y_perm[inv[t*k+s]][d], slot order, float4 per thread.
+__global__ void __launch_bounds__(256) route_unpermute_kernel(const float *__restrict__ y_perm,
+                                                              const int32_t *__restrict__ inv,
+                                                              const float *__restrict__ w, int T,
+                                                              int k, int D, int n_routes,
+                                                              float *__restrict__ out) {
+    const int d4 = D >> 2;
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (long long)T * d4) return;
+    const int t = (int)(idx / d4);
+    const int c = (int)(idx % d4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < k; ++s) {
+        int r = inv[t * k + s];
+        float ws = w[t * k + s];
+        if (r < 0 || r >= n_routes) {
+            raise_flag(1);
+            continue;
+        }
+        float4 y = reinterpret_cast<const float4 *>(y_perm + (size_t)r * D)[c];
+        acc.x = fmaf(ws, y.x, acc.x);
+        acc.y = fmaf(ws, y.y, acc.y);
+        acc.z = fmaf(ws, y.z, acc.z);
+        acc.w = fmaf(ws, y.w, acc.w);
+    }
+    reinterpret_cast<float4 *>(out + (size_t)t * D)[c] = acc;
+}
+
+}  // namespace tq
+
+using namespace tq;
+
+TQ_API int route_topk(const float *logits, int T, int E, int k, int32_t *topk_ids, float *topk_w,
+                      tq_stream stream) {
+    if (T < 0 || k < 1 || k > 32 || E < k || E > 32 * kTopkMaxPerLane) return TQ_ERR_INVALID_ARG;
+    if (T == 0) return TQ_OK;
+    if (!logits || !topk_ids || !topk_w) return TQ_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int threads = 256;
+    const int blocks = (int)(((long long)T * 32 + threads - 1) / threads);
+    const int per = (E + 31) / 32;
+    LaunchScope ls(s, kStageTopk);
+    if (per <= 4)
+        route_topk_kernel<4><<<blocks, threads, 0, s>>>(logits, T, E, k, topk_ids, topk_w);
+    else if (per <= 12)
+        route_topk_kernel<12><<<blocks, threads, 0, s>>>(logits, T, E, k, topk_ids, topk_w);
+    else
+        route_topk_kernel<32><<<blocks, threads, 0, s>>>(logits, T, E, k, topk_ids, topk_w);
+    return launch_status();
+}
+
+TQ_API int route_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *counts,
+                         int32_t *offsets, int32_t *perm, int32_t *inv, int32_t *active_ids,
+                         int32_t *n_active, tq_stream stream) {
+    if (T < 0 || k < 1 || E < 1 || E > kPermMaxE) return TQ_ERR_INVALID_ARG;
+    if ((long long)T * k > (1ll << 30)) return TQ_ERR_UNSUPPORTED;
+    if (!counts || !offsets || !active_ids || !n_active) return TQ_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_ids || !perm || !inv)) return TQ_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t smem = permute_smem_bytes(E);
+    static bool configured = false;
+    if (!configured) {
+        if (cudaFuncSetAttribute(route_permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)permute_smem_bytes(kPermMaxE)) != cudaSuccess)
+            return TQ_ERR_CUDA;
+        configured = true;
+    }
+    LaunchScope ls(s, kStagePermute);
+    route_permute_kernel<<<1, kPermThreads, smem, s>>>(topk_ids, T * k, E, counts, offsets, perm,
+                                                       inv, active_ids, n_active);
+    return launch_status();
+}
+
+TQ_API int route_unpermute(const float *y_perm, const int32_t *inv, const float *topk_w, int T,
+                           int k, int D, float *out, tq_stream stream) {
+    if (T < 0 || k < 1 || D < 4 || D % 4) return TQ_ERR_INVALID_ARG;
+    if (T == 0) return TQ_OK;
+    if (!y_perm || !inv || !topk_w || !out) return TQ_ERR_INVALID_ARG;
+    if (!aligned16(y_perm) || !aligned16(out)) return TQ_ERR_ALIGNMENT;
+    cudaStream_t s = (cudaStream_t)stream;
+    const long long n = (long long)T * (D / 4);
+    const int threads = 256;
+    LaunchScope ls(s, kStageUnpermute);
+    route_unpermute_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, s>>>(
+        y_perm, inv, topk_w, T, k, D, T * k, out);
+    return launch_status();
+}
