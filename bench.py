@@ -192,6 +192,7 @@ def gateup_algorithmic_bytes(layer, counts):
             K_of[e] = g["K"]
     total = 0
     for e, n in enumerate(counts):
+        n = int(n)
         if n == 0:
             continue
         total += 2 * layer.F * layer.D * K_of[e] // 8 + 2 * layer.F * 2

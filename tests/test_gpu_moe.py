@@ -68,6 +68,19 @@ def test_wider_layer_more_tokens_per_expert(api):
     check_against_oracle(got, OL.moe_layer(layer, x, logits, 2))
 
 
+def test_multi_pass_experts_with_stage_reuse(api):
+    # D = 1024, F = 512: every warp streams several shared-memory stages per pass (stage
+    # buffers and their barriers are reused), and with 64 tokens, top-2 of 4 experts
+    # each expert has ~32 routes, i.e. several 8-route passes per work item.
+    layer = inputs.small_layer(61, E=4, D=1024, F=512, split={2: 2, 3: 1, 4: 1})
+    rng = np.random.default_rng(62)
+    x = inputs.random_activations(rng, (64, 1024), "bf16")
+    logits = inputs.normal_logits(rng, 64, 4)
+    got, _, _ = run_layer(api, layer, x, logits, 2)
+    check_against_oracle(got, OL.moe_layer(layer, x, logits, 2))
+    assert api.device_status() == 0
+
+
 def test_mixed_width_routes_bit_identical_to_single_width(api):
     # After the TrellisMX K2 Mix card's layer test: every width's routes computed in the
     # mixed-width launch equal, bit for bit, the same routes in a launch whose layer holds
@@ -143,6 +156,7 @@ def test_full_size_decode_layer_sampled_tokens(api):
     # the launch configuration the benchmark times; the oracle computes 2 tokens.
     w = inputs.moe_decode_t16()
     got, bufs, _ = run_layer(api, w["layer"], w["x"], w["logits"], 8)
+    assert np.isfinite(got).all()
     res = OL.moe_tokens(w["layer"], w["x"], w["logits"], 8, token_ids=[0, 11])
     np.testing.assert_array_equal(bufs.ids.cpu().numpy(), res["topk_ids"])
     check_against_oracle(got, res, tokens=[0, 11])

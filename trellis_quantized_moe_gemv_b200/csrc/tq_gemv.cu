@@ -202,6 +202,11 @@ __device__ __forceinline__ float finish(float d, float sx, float scale) {
     return scale * kKappa * (d - kOffset * sx);
 }
 
+// Subnormal planes: D = 2^-24 * sum_j t_j x_j, so sum_j c_j x_j = 2^24 D - 255 sum_j x_j.
+__device__ __forceinline__ float finish_sub(float d, float sx, float scale) {
+    return scale * kKappa * fmaf(16777216.0f, d, -255.0f * sx);
+}
+
 __device__ __forceinline__ void split_range(int n, int part, int parts, int &b, int &e) {
     const int per = (n + parts - 1) / parts;
     b = min(n, part * per);
@@ -216,7 +221,7 @@ template <int K, int NG>
 __global__ void __launch_bounds__(kGemvThreads, 2)
     trellis_gemv_kernel(const uint32_t *__restrict__ bits, const __half *__restrict__ scales, int rows,
                         int cols, const __half *__restrict__ x, int batch, float *__restrict__ y) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(128) unsigned char smem_raw[];
     RedSmem<NG> &red = *reinterpret_cast<RedSmem<NG> *>(smem_raw);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2;
     const int n_strips = rows / 16, tiles = cols / 16;
@@ -273,117 +278,270 @@ __device__ __forceinline__ bool expert_ref(const tq_moe_layer &L, int e, ExpertR
     return true;
 }
 
-template <int NG>
-__device__ __forceinline__ void accumulate_any_k(int K, const uint32_t *strip0, int jb, int je,
-                                                 const __half *const (&xr)[NG], Acc<NG> &acc) {
-    if (K == 2) accumulate<2, NG>(strip0, jb, je, xr, acc);
-    else if (K == 3) accumulate<3, NG>(strip0, jb, je, xr, acc);
-    else accumulate<4, NG>(strip0, jb, je, xr, acc);
+// ----------------------------------------------------------------------------- MoE items
+//
+// MoE GEMV work item = one CTA of kItemWarps warps: (active expert, 8 strips of 16
+// rows, 8 of the expert's routes).  The warps split the column tiles into contiguous
+// ranges; each streams its range of the 8 strips through its own ring of shared-memory
+// stages filled by bulk copies (lanes 0..7 copy one strip each, completing on one
+// mbarrier per stage; consumers poll with a bound), and the warps' MMA partial sums
+// are added in shared memory in a fixed order at the end of the item.
+//
+// Per weight: one funnel shift brings the window to bit 0 (none for windows that start
+// a word), one integer multiply by 0x3A2F0000 leaves the T16 product's bytes lo, hi in
+// bytes 2 and 3 with zeros below, and one PRMT pairs the lo (or hi) bytes of two
+// weights with zero bytes: fp16 subnormals lo * 2^-24 and hi * 2^-24, exact operands.
+// The MMA accumulates D = 2^-24 * sum_j t_j x_j in fp32 (no offset to cancel).
+
+constexpr int kItemWarps = 4;
+constexpr int kItemThreads = kItemWarps * 32;
+constexpr int kStages = 2;
+constexpr int kSlotBytes = 576;               // per strip per stage: >= 8*64, 5*96, 4*128 B,
+                                              // 64 B pad so 2 strips share no bank in a phase
+constexpr int kStageBytes = 8 * kSlotBytes;
+
+template <int K>
+constexpr int tiles_per_stage() { return K == 2 ? 8 : (K == 3 ? 5 : 4); }
+
+// A warp's ring: its stage buffers and one mbarrier per stage.  The barriers live in a
+// region of their own (ItemSmem::bar) that nothing else ever writes: an mbarrier's
+// memory must not be reused by ordinary stores while the barrier is initialised.
+struct WarpRing {
+    unsigned char (*buf)[kStageBytes];
+    uint64_t *bar;
+};
+
+struct __align__(128) ItemSmem {
+    unsigned char buf[kItemWarps][kStages][kStageBytes];
+    uint64_t bar[kItemWarps][kStages];
+};
+
+// T16 product of the window at compile-time bit offset O of the lane's span, in the
+// high half of the result (low half zero): bytes [0, 0, lo, hi].
+template <int O, int NS>
+__device__ __forceinline__ uint32_t t16_product_hi(const uint32_t (&v)[NS]) {
+    constexpr int wi = O >> 5, sh = O & 31;
+    uint32_t bottom;
+    if constexpr (sh == 0) bottom = v[wi];
+    else bottom = funnel_r(v[wi], v[wi + 1], sh);
+    return bottom * (kT16Mult << 16);
 }
 
-// Gate/up + SiLU: item = (active expert, 64 intermediate rows).  Lane groups 0..3 walk
-// gate strips, 4..7 the up strips of the same rows.  h[route][f] = silu(g) * u (fp32).
-template <int NG>
-__global__ void __launch_bounds__(kGemvThreads, 2)
-    moe_gateup_kernel(const tq_moe_layer L, const __half *__restrict__ x_rot,
-                      const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm,
-                      const int32_t *__restrict__ active_ids, const int32_t *__restrict__ n_active_p,
-                      int k, int n_routes, float *__restrict__ h) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    RedSmem<NG> &red = *reinterpret_cast<RedSmem<NG> *>(smem_raw);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2;
-    const int D = L.D, F = L.F, tiles = D / 16;
-    const int items_per_expert = F / 64;
-    const int n_items = *n_active_p * items_per_expert;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int a = item / items_per_expert, fi = item % items_per_expert;
-        const int e = active_ids[a];
-        ExpertRef ex;
-        if (!expert_ref(L, e, ex)) {
-            if (threadIdx.x == 0) raise_flag(1);
-            continue;
-        }
-        const int r0 = offsets[e], ne = offsets[e + 1] - r0;
-        const int f_strip = fi * 4 + (gq & 3);
-        const uint32_t *proj = gq < 4 ? ex.gate : ex.up;
-        const uint32_t *strip0 = proj + (size_t)f_strip * tiles * (8 * ex.K);
-        for (int tb = 0; tb < ne; tb += 8 * NG) {
-            const __half *xr[NG];
-#pragma unroll
-            for (int g = 0; g < NG; ++g) {
-                const int tt = tb + 8 * g + gq;
-                const int ri = r0 + tt;
-                const int pr = tt < ne ? perm[ri] : -1;
-                xr[g] = (pr >= 0 && pr < n_routes) ? x_rot + (size_t)(pr / k) * D : nullptr;
-            }
-            Acc<NG> acc;
-            zero(acc);
-            int jb, je;
-            split_range(tiles, warp, kGemvWarps, jb, je);
-            accumulate_any_k<NG>(ex.K, strip0, jb, je, xr, acc);
-            __syncthreads();   // previous pass / item finished reading red
-            store_partials(acc, red);
-            __syncthreads();
-            for (int i = threadIdx.x; i < NG * 4 * 16 * 8; i += kGemvThreads) {
-                const int tok = i & 7, row = (i >> 3) & 15, st = (i >> 7) & 3, g = i >> 9;
-                const int tt = tb + 8 * g + tok;
-                if (tt >= ne) continue;
-                const int f = (fi * 4 + st) * 16 + row;
-                const float sx = red_s(red, g, tok);
-                const float gv = finish(red_d(red, g, st, row, tok), sx, __half2float(ex.s_gate[f]));
-                const float uv = finish(red_d(red, g, st + 4, row, tok), sx, __half2float(ex.s_up[f]));
-                h[(size_t)(r0 + tt) * F + f] = silu_f32(gv) * uv;
-            }
-        }
+template <int K, int P>
+__device__ __forceinline__ void tile_pairs_sub(const uint32_t (&v)[2 * K + 1], uint2 xb, Acc<1> &acc) {
+    if constexpr (P < 8) {
+        constexpr int r0 = P, r1 = P + 8;
+        const uint32_t R00 = t16_product_hi<0 * 16 * K + K * r0>(v);
+        const uint32_t R01 = t16_product_hi<1 * 16 * K + K * r0>(v);
+        const uint32_t R02 = t16_product_hi<2 * 16 * K + K * r0>(v);
+        const uint32_t R03 = t16_product_hi<3 * 16 * K + K * r0>(v);
+        const uint32_t R10 = t16_product_hi<0 * 16 * K + K * r1>(v);
+        const uint32_t R11 = t16_product_hi<1 * 16 * K + K * r1>(v);
+        const uint32_t R12 = t16_product_hi<2 * 16 * K + K * r1>(v);
+        const uint32_t R13 = t16_product_hi<3 * 16 * K + K * r1>(v);
+        mma_f16_16816(acc.d[P][0], prmt(R00, R01, kSelLo), prmt(R10, R11, kSelLo), prmt(R02, R03, kSelLo),
+                      prmt(R12, R13, kSelLo), xb.x, xb.y);
+        mma_f16_16816(acc.d[P][0], prmt(R00, R01, kSelHi), prmt(R10, R11, kSelHi), prmt(R02, R03, kSelHi),
+                      prmt(R12, R13, kSelHi), xb.x, xb.y);
+        tile_pairs_sub<K, P + 1>(v, xb, acc);
     }
 }
 
-// Down projection: item = (active expert, 128 output rows).  y[route][d] = W_down h'.
-template <int NG>
-__global__ void __launch_bounds__(kGemvThreads, 2)
-    moe_down_kernel(const tq_moe_layer L, const __half *__restrict__ h_rot,
-                    const int32_t *__restrict__ offsets, const int32_t *__restrict__ active_ids,
-                    const int32_t *__restrict__ n_active_p, float *__restrict__ y) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    RedSmem<NG> &red = *reinterpret_cast<RedSmem<NG> *>(smem_raw);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2;
-    const int D = L.D, F = L.F, tiles = F / 16;
-    const int items_per_expert = D / 128;
-    const int n_items = *n_active_p * items_per_expert;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int a = item / items_per_expert, di = item % items_per_expert;
-        const int e = active_ids[a];
-        ExpertRef ex;
-        if (!expert_ref(L, e, ex)) {
-            if (threadIdx.x == 0) raise_flag(1);
-            continue;
+__device__ __forceinline__ void ring_init(const WarpRing &ring) {
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&ring.bar[s], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+}
+
+// Issue chunk c (tiles [j0 + c*S, ...), at most `je` exclusive) of the 8 strips into
+// stage st.  strip_lane: base of the strip this lane copies (lanes 0..7).
+template <int K>
+__device__ __forceinline__ void ring_issue(const WarpRing &ring, int st, int c, int j0, int je,
+                                           const uint32_t *strip_lane) {
+    constexpr int S = tiles_per_stage<K>();
+    constexpr int TB = 32 * K;  // bytes per tile
+    const int lane = threadIdx.x & 31;
+    const int jb = j0 + c * S;
+    const int nt = min(S, je - jb);
+    if (lane == 0) {
+        fence_proxy_async();
+        mbar_arrive_expect_tx(&ring.bar[st], 8u * nt * TB);
+    }
+    __syncwarp();
+    if (lane < 8) bulk_g2s(ring.buf[st] + lane * kSlotBytes, strip_lane + (size_t)jb * (8 * K), nt * TB, &ring.bar[st]);
+}
+
+// Stream tiles [j0, je) of the 8 strips against the lane's token row xr (fp16 or null).
+// Returns false, after draining its copies, if a bounded wait gave up.
+template <int K>
+__device__ __forceinline__ bool stream_range(const WarpRing &ring, uint32_t &parity, int j0, int je,
+                                          const uint32_t *strip_lane, const __half *xr, Acc<1> &acc) {
+    constexpr int S = tiles_per_stage<K>();
+    constexpr int TB = 32 * K;
+    const int lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
+    const int n_chunks = (je - j0 + S - 1) / S;
+    for (int c = 0; c < min(kStages, n_chunks); ++c) ring_issue<K>(ring, c, c, j0, je, strip_lane);
+    uint2 xn = (xr && j0 < je) ? __ldg(reinterpret_cast<const uint2 *>(xr + 16 * j0 + 4 * t4)) : make_uint2(0u, 0u);
+    for (int c = 0; c < n_chunks; ++c) {
+        const int st = c % kStages;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&ring.bar[st], (parity >> st) & 1u));
+        parity ^= 1u << st;
+        if (!ok) {
+            for (int d = c + 1; d < min(c + kStages, n_chunks); ++d) {
+                const int sd = d % kStages;
+                mbar_wait_bounded(&ring.bar[sd], (parity >> sd) & 1u);
+                parity ^= 1u << sd;
+            }
+            return false;
         }
-        const int r0 = offsets[e], ne = offsets[e + 1] - r0;
-        const uint32_t *strip0 = ex.down + (size_t)(di * 8 + gq) * tiles * (8 * ex.K);
-        for (int tb = 0; tb < ne; tb += 8 * NG) {
-            const __half *xr[NG];
+        const int jb = j0 + c * S;
+        const int nt = min(S, je - jb);
+        const unsigned char *slot = ring.buf[st] + gq * kSlotBytes;
+#pragma unroll 1
+        for (int t = 0; t < nt; ++t) {
+            const unsigned char *tile = slot + t * TB;
+            uint32_t v[2 * K + 1];
+            if constexpr (K == 2) {
+                uint4 a = *reinterpret_cast<const uint4 *>(tile + 16 * t4);
+                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            } else if constexpr (K == 3) {
+                const uint2 *q = reinterpret_cast<const uint2 *>(tile + 24 * t4);
+                uint2 a = q[0], b = q[1], d = q[2];
+                v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y; v[4] = d.x; v[5] = d.y;
+            } else {
+                const uint4 *q = reinterpret_cast<const uint4 *>(tile + 32 * t4);
+                uint4 a = q[0], b = q[1];
+                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+                v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+            }
+            v[2 * K] = *reinterpret_cast<const uint32_t *>(tile + 8 * K * ((t4 + 1) & 3));
+            const uint2 x = xn;
+            const int jn = jb + t + 1;
+            if (xr && jn < je) xn = __ldg(reinterpret_cast<const uint2 *>(xr + 16 * jn + 4 * t4));
+            tile_pairs_sub<K, 0>(v, x, acc);
+            mma_f16_16816(acc.s[0], kOneH2, kOneH2, kOneH2, kOneH2, x.x, x.y);
+        }
+        __syncwarp();
+        if (c + kStages < n_chunks) ring_issue<K>(ring, st, c + kStages, j0, je, strip_lane);
+    }
+    return true;
+}
+
+// Shared-memory partials of the CTA's warps; aliases the stage buffers (never the
+// barriers) once every warp has consumed its last stage.
+struct ItemRed {
+    float d[kItemWarps][8][16][8];   // [warp][strip][row][token]
+    float s[kItemWarps][8];          // [warp][token]
+};
+static_assert(sizeof(ItemRed) <= sizeof(ItemSmem::buf), "reduction buffer must fit in the stage buffers");
+
+// GATEUP: item = (active expert, 64 intermediate rows: strips 0..3 of gate, 0..3 of up),
+//         out = h [routes][F] fp32, h = silu(gate x') * (up x').
+// !GATEUP: item = (active expert, 128 output rows), xsrc = h' [routes][F] fp16,
+//          out = y [routes][D] fp32.
+template <bool GATEUP>
+__global__ void __launch_bounds__(kItemThreads, 5)
+    moe_gemv_items_kernel(const tq_moe_layer L, const __half *__restrict__ xsrc,
+                          const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm,
+                          const int32_t *__restrict__ active_ids, const int32_t *__restrict__ n_active_p,
+                          int k, int n_routes, float *__restrict__ out) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    ItemSmem &sm_items = *reinterpret_cast<ItemSmem *>(smem_raw);
+    ItemRed &red = *reinterpret_cast<ItemRed *>(smem_raw);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2, t4 = lane & 3;
+    const int per_expert = GATEUP ? L.F / 64 : L.D / 128;
+    const int item = blockIdx.x;
+    if (item >= *n_active_p * per_expert) return;
+    const int a = item / per_expert, sub = item % per_expert;
+    const int e = active_ids[a];
+    ExpertRef ex;
+    if (!expert_ref(L, e, ex)) {
+        if (threadIdx.x == 0) raise_flag(1);
+        return;
+    }
+    const WarpRing ring{sm_items.buf[warp], sm_items.bar[warp]};
+    ring_init(ring);
+    uint32_t parity = 0;
+
+    const int r0 = offsets[e], ne = offsets[e + 1] - r0;
+    const int tiles = GATEUP ? L.D / 16 : L.F / 16;
+    int jb, je;
+    split_range(tiles, warp, kItemWarps, jb, je);
+    const int cs = lane & 7;
+    const uint32_t *strip_lane;
+    if (GATEUP)
+        strip_lane = (cs < 4 ? ex.gate : ex.up) + (size_t)(sub * 4 + (cs & 3)) * tiles * (8 * ex.K);
+    else
+        strip_lane = ex.down + (size_t)(sub * 8 + cs) * tiles * (8 * ex.K);
+
+    for (int tb = 0; tb < ne; tb += 8) {
+        const int tt = tb + gq;
+        const __half *xr = nullptr;
+        if (tt < ne) {
+            if (GATEUP) {
+                const int pr = perm[r0 + tt];
+                if (pr >= 0 && pr < n_routes) xr = xsrc + (size_t)(pr / k) * L.D;
+            } else {
+                xr = xsrc + (size_t)(r0 + tt) * L.F;
+            }
+        }
+        Acc<1> acc;
+        zero(acc);
+        bool ok;
+        if (ex.K == 2) ok = stream_range<2>(ring, parity, jb, je, strip_lane, xr, acc);
+        else if (ex.K == 3) ok = stream_range<3>(ring, parity, jb, je, strip_lane, xr, acc);
+        else ok = stream_range<4>(ring, parity, jb, je, strip_lane, xr, acc);
+        ok = __syncthreads_and(ok);
+        if (!ok) return;   // every warp drained its copies; the item is left unwritten
+        // partials -> shared memory (the rings are idle now)
 #pragma unroll
-            for (int g = 0; g < NG; ++g) {
-                const int tt = tb + 8 * g + gq;
-                xr[g] = tt < ne ? h_rot + (size_t)(r0 + tt) * F : nullptr;
+        for (int p = 0; p < 8; ++p) {
+            red.d[warp][gq][p][2 * t4] = acc.d[p][0][0];
+            red.d[warp][gq][p][2 * t4 + 1] = acc.d[p][0][1];
+            red.d[warp][gq][p + 8][2 * t4] = acc.d[p][0][2];
+            red.d[warp][gq][p + 8][2 * t4 + 1] = acc.d[p][0][3];
+        }
+        if (gq == 0) {
+            red.s[warp][2 * t4] = acc.s[0][0];
+            red.s[warp][2 * t4 + 1] = acc.s[0][1];
+        }
+        __syncthreads();
+        if (GATEUP) {
+            for (int i = threadIdx.x; i < 4 * 16 * 8; i += kItemThreads) {
+                const int tok = i & 7, row = (i >> 3) & 15, st = i >> 7;
+                const int t2 = tb + tok;
+                if (t2 >= ne) continue;
+                float dg = 0.f, du = 0.f, sx = 0.f;
+#pragma unroll
+                for (int w = 0; w < kItemWarps; ++w) {
+                    dg += red.d[w][st][row][tok];
+                    du += red.d[w][st + 4][row][tok];
+                    sx += red.s[w][tok];
+                }
+                const int f = (sub * 4 + st) * 16 + row;
+                const float gv = finish_sub(dg, sx, __half2float(ex.s_gate[f]));
+                const float uv = finish_sub(du, sx, __half2float(ex.s_up[f]));
+                out[(size_t)(r0 + t2) * L.F + f] = silu_f32(gv) * uv;
             }
-            Acc<NG> acc;
-            zero(acc);
-            int jb, je;
-            split_range(tiles, warp, kGemvWarps, jb, je);
-            accumulate_any_k<NG>(ex.K, strip0, jb, je, xr, acc);
-            __syncthreads();
-            store_partials(acc, red);
-            __syncthreads();
-            for (int i = threadIdx.x; i < NG * 8 * 16 * 8; i += kGemvThreads) {
-                const int tok = i & 7, row = (i >> 3) & 15, st = (i >> 7) & 7, g = i >> 10;
-                const int tt = tb + 8 * g + tok;
-                if (tt >= ne) continue;
-                const int d = (di * 8 + st) * 16 + row;
-                y[(size_t)(r0 + tt) * D + d] =
-                    finish(red_d(red, g, st, row, tok), red_s(red, g, tok), __half2float(ex.s_down[d]));
+        } else {
+            for (int i = threadIdx.x; i < 8 * 16 * 8; i += kItemThreads) {
+                const int tok = i & 7, row = (i >> 3) & 15, st = i >> 7;
+                const int t2 = tb + tok;
+                if (t2 >= ne) continue;
+                float dd = 0.f, sx = 0.f;
+#pragma unroll
+                for (int w = 0; w < kItemWarps; ++w) {
+                    dd += red.d[w][st][row][tok];
+                    sx += red.s[w][tok];
+                }
+                const int d = (sub * 8 + st) * 16 + row;
+                out[(size_t)(r0 + t2) * L.D + d] = finish_sub(dd, sx, __half2float(ex.s_down[d]));
             }
         }
+        __syncthreads();   // the rings are reused by the next pass
     }
 }
 
@@ -420,14 +578,14 @@ size_t workspace_bytes(const tq_moe_layer *L, int T, int k) {
 int launch_hadamard128(const void *x, int x_dtype, long long rows, long long cols, __half *out,
                        cudaStream_t s, int stage);
 
-template <int NG>
 int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offsets, const int32_t *perm,
                  const int32_t *active_ids, const int32_t *n_active, int T, int k, float *y_perm,
                  void *ws, cudaStream_t s) {
-    const size_t smem = sizeof(RedSmem<NG>);
+    const size_t smem = sizeof(ItemSmem);
     static bool configured = false;
     if (!configured) {
-        if (set_smem(moe_gateup_kernel<NG>, smem) || set_smem(moe_down_kernel<NG>, smem)) return TQ_ERR_CUDA;
+        if (set_smem(moe_gemv_items_kernel<true>, smem) || set_smem(moe_gemv_items_kernel<false>, smem))
+            return TQ_ERR_CUDA;
         configured = true;
     }
     const int routes = T * k;
@@ -435,21 +593,20 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     __half *h_rot = reinterpret_cast<__half *>(reinterpret_cast<char *>(ws) +
                                                align256((size_t)routes * L->F * sizeof(float)));
     const int max_active = min(L->E, routes);
-    const int grid_cap = 2 * num_sms();
     const int gu_items = max_active * (L->F / 64);
     const int dn_items = max_active * (L->D / 128);
     {
-    LaunchScope ls(s, kStageGemvGateUp);
-    moe_gateup_kernel<NG><<<min(gu_items, grid_cap), kGemvThreads, smem, s>>>(
-        *L, x_rot, offsets, perm, active_ids, n_active, k, routes, h);
+        LaunchScope ls(s, kStageGemvGateUp);
+        moe_gemv_items_kernel<true><<<gu_items, kItemThreads, smem, s>>>(*L, x_rot, offsets, perm, active_ids,
+                                                                          n_active, k, routes, h);
     }
     int st = launch_status();
     if (st) return st;
     st = launch_hadamard128(h, TQ_DTYPE_F32, routes, L->F, h_rot, s, kStageRotateH);
     if (st) return st;
     LaunchScope ls(s, kStageGemvDown);
-    moe_down_kernel<NG><<<min(dn_items, grid_cap), kGemvThreads, smem, s>>>(*L, h_rot, offsets,
-                                                                             active_ids, n_active, y_perm);
+    moe_gemv_items_kernel<false><<<dn_items, kItemThreads, smem, s>>>(*L, h_rot, offsets, perm, active_ids,
+                                                                       n_active, k, routes, y_perm);
     return launch_status();
 }
 
@@ -524,6 +681,5 @@ TQ_API int moe_trellis_gemv(const tq_moe_layer *layer, const uint16_t *x_rot, co
     if (st || T == 0) return st;
     const __half *x = reinterpret_cast<const __half *>(x_rot);
     cudaStream_t s = (cudaStream_t)stream;
-    if (T <= 8) return run_moe_gemv<1>(layer, x, offsets, perm, active_ids, n_active, T, k, y_perm, ws, s);
-    return run_moe_gemv<2>(layer, x, offsets, perm, active_ids, n_active, T, k, y_perm, ws, s);
+    return run_moe_gemv(layer, x, offsets, perm, active_ids, n_active, T, k, y_perm, ws, s);
 }
