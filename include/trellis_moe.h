@@ -224,6 +224,29 @@ int moe_trellis_gemv(const tq_moe_layer *layer, const uint16_t *x_rot, const int
                      int T, int k, float *y_perm, void *ws, size_t ws_bytes, tq_stream stream);
 
 /*
+ * moe_trellis_gemv_noalloc -- moe_trellis_gemv without a caller-provided workspace, for
+ * callers that cannot allocate device memory when they run the layer (a serving
+ * runtime whose memory is one pool carved up at start-up, a plugin or sandboxed engine
+ * that only receives the call's own tensors, a latency-critical path where an
+ * allocation and the synchronisation it may imply are not allowed).  The pages have no
+ * counterpart: this is a packaging of the same computation.
+ *   Same arguments and result as moe_trellis_gemv, minus ws / ws_bytes.  The workspace
+ *   is a 4 MiB array compiled into the library (a __device__ array every GPU that loads
+ *   the library holds until exit), so T * k * F may be at most 699,050 (T * k <= 682 for
+ *   F = 1024); larger calls return TQ_ERR_WORKSPACE without doing anything.
+ *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *   once per device, with that device current); make that first call before any stream
+ *   capture.  Every call on a device shares the one array and it keeps the last call's
+ *   contents; each call writes every workspace byte it reads before reading it, so
+ *   nothing needs clearing, but calls that overlap on the GPU (other streams, other
+ *   threads) race on the array and must be serialised by the caller.
+ */
+int moe_trellis_gemv_noalloc(const tq_moe_layer *layer, const uint16_t *x_rot,
+                             const int32_t *offsets, const int32_t *perm, const int32_t *active_ids,
+                             const int32_t *n_active, int T, int k, float *y_perm, tq_stream stream);
+
+/*
  * moe_trellis_gemm -- same result as moe_trellis_gemv for prefill-sized batches: the
  * bit streams are decoded to fp16 operands of tcgen05 tensor-core MMAs (accumulating
  * in tensor memory), each weight decoded once per 128 routes of its expert.

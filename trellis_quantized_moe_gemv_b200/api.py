@@ -63,6 +63,8 @@ SIGNATURES = {
                           _SZ, _VP], _I),
     "moe_trellis_gemm": ([ctypes.POINTER(TqMoeLayer), _VP, _VP, _VP, _VP, _VP, _I, _I, _VP, _VP,
                           _SZ, _VP], _I),
+    "moe_trellis_gemv_noalloc": ([ctypes.POINTER(TqMoeLayer), _VP, _VP, _VP, _VP, _VP, _I, _I, _VP,
+                                  _VP], _I),
 }
 
 
@@ -326,6 +328,20 @@ def _moe_call(name, layer: DeviceLayer, x_rot, routing: Routing, T, k, y_perm=No
 
 def moe_trellis_gemv(layer, x_rot, routing, T, k, y_perm=None, ws=None, stream=None):
     return _moe_call("moe_trellis_gemv", layer, x_rot, routing, T, k, y_perm, ws, stream)
+
+
+def moe_trellis_gemv_noalloc(layer: DeviceLayer, x_rot: torch.Tensor, routing: Routing, T: int, k: int,
+                             y_perm: torch.Tensor, stream=None) -> torch.Tensor:
+    """moe_trellis_gemv with the library's own fixed scratch array instead of a workspace,
+    for callers that cannot allocate device memory at call time.  y_perm ([T*k, D] fp32)
+    must be provided; the call itself allocates nothing.  At most T*k*F = 699,050."""
+    _require(x_rot, torch.float16, "x_rot")
+    _require(y_perm, torch.float32, "y_perm")
+    _check(_fn("moe_trellis_gemv_noalloc")(ctypes.byref(layer.struct), _p(x_rot), _p(routing.offsets),
+                                           _p(routing.perm), _p(routing.active_ids),
+                                           _p(routing.n_active), T, k, _p(y_perm), _stream(stream)),
+           "moe_trellis_gemv_noalloc")
+    return y_perm
 
 
 def moe_trellis_gemm(layer, x_rot, routing, T, k, y_perm=None, ws=None, stream=None):

@@ -6,3 +6,4 @@
 #include "tq_decode.cu"
 #include "tq_gemv.cu"
 #include "tq_gemm.cu"
+#include "tq_noalloc.cu"

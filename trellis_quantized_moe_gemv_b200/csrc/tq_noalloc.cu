@@ -1,0 +1,65 @@
+// moe_trellis_gemv for callers that cannot allocate device memory.
+//
+// Some callers of this library cannot call cudaMalloc (or any allocator) when they run
+// the layer: a serving runtime whose device memory is one pool carved up at start-up,
+// an engine that runs inside a sandbox or plugin host which hands it only the tensors
+// of the call, or a latency-critical path where an allocation (and the device
+// synchronisation it can imply) is not allowed.  moe_trellis_gemv needs a workspace
+// for the SwiGLU activations h and their rotation h'; this entry point takes that
+// workspace from a fixed array compiled into the library instead.
+#include "tq_common.cuh"
+
+namespace tq {
+
+// Scratch for h (fp32) and h' (fp16) of every route: at most 4 MiB, i.e. T * k * F up
+// to 699,050 (T * k <= 682 routes for F = 1024).  Every GPU that loads the library
+// holds this array until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+static void *g_noalloc_ptr[kNoAllocMaxDevices];
+
+// Device address of the scratch array on the current device; looked up once per
+// device (the array's name is only a host-side stand-in in host code).
+static int noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return TQ_ERR_UNSUPPORTED;
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return TQ_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return TQ_OK;
+}
+
+int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offsets, const int32_t *perm,
+                 const int32_t *active_ids, const int32_t *n_active, int T, int k, float *y_perm,
+                 void *ws, cudaStream_t s);
+
+}  // namespace tq
+
+int moe_validate_call(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
+                      const int32_t *perm, const int32_t *active_ids, const int32_t *n_active, int T,
+                      int k, float *y_perm, void *ws, size_t ws_bytes);
+
+TQ_API int moe_trellis_gemv_noalloc(const tq_moe_layer *layer, const uint16_t *x_rot,
+                                    const int32_t *offsets, const int32_t *perm,
+                                    const int32_t *active_ids, const int32_t *n_active, int T, int k,
+                                    float *y_perm, tq_stream stream) {
+    const int valid = tq::validate_layer(layer);
+    if (valid != TQ_OK) return valid;
+    if (T < 0 || k < 1) return TQ_ERR_INVALID_ARG;
+    if (T == 0) return TQ_OK;
+    if (tq::workspace_bytes(layer, T, k) > tq::kNoAllocScratchBytes) return TQ_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    int st = tq::noalloc_scratch(&scratch);
+    if (st) return st;
+    st = moe_validate_call(layer, x_rot, offsets, perm, active_ids, n_active, T, k, y_perm, scratch,
+                           tq::kNoAllocScratchBytes);
+    if (st) return st;
+    return tq::run_moe_gemv(layer, reinterpret_cast<const __half *>(x_rot), offsets, perm, active_ids,
+                            n_active, T, k, y_perm, scratch, (cudaStream_t)stream);
+}
