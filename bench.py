@@ -28,7 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "routed-expert tok/s per MoE layer; GEMV HBM GB/s and GEMM tensor-pipe % of peak"
-N_LAYER_COPIES = 4
+N_LAYER_COPIES = 4   # default of --layers
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
@@ -40,6 +40,9 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="moe_decode_t16", choices=["moe_decode_t16"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--layers", type=int, default=4,
+                   help="synthetic layer copies cycled through (4 keep every step's weights out of L2)")
+    p.add_argument("--eager", action="store_true", help="launch every step from the host instead of a CUDA graph")
     return p.parse_args()
 
 
@@ -151,7 +154,7 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workload
 
-def build_decode_workload(api, inputs, torch, device, rank):
+def build_decode_workload(api, inputs, torch, device, rank, n_copies):
     """Layer copy 0 from the seeded numpy generators (the copy the parity tests check);
     copies 1..3 with the same widths, their bit streams and scales drawn on the device
     from a seeded torch generator; every copy has its own tokens and logits."""
@@ -160,7 +163,7 @@ def build_decode_workload(api, inputs, torch, device, rank):
     layers, xs, logits = [], [], []
     layers.append(api.DeviceLayer.from_synthetic(host_layer, device))
     gen = torch.Generator(device=device)
-    for c in range(1, N_LAYER_COPIES):
+    for c in range(1, n_copies):
         gen.manual_seed(7000 + 100 * rank + c)
         groups = []
         for g in host_layer.groups:
@@ -174,7 +177,7 @@ def build_decode_workload(api, inputs, torch, device, rank):
                                down=rbits(g.down.shape), s_gate=rscale(g.s_gate.shape),
                                s_up=rscale(g.s_up.shape), s_down=rscale(g.s_down.shape)))
         layers.append(api.DeviceLayer(host_layer.E, host_layer.D, host_layer.F, groups, device))
-    for c in range(N_LAYER_COPIES):
+    for c in range(n_copies):
         rng = np.random.default_rng(9000 + 100 * rank + c)
         x = w0["x"] if c == 0 else inputs.random_activations(rng, (16, host_layer.D), "bf16")
         lg = w0["logits"] if c == 0 else inputs.normal_logits(rng, 16, host_layer.E)
@@ -217,27 +220,54 @@ def run_ours(args, rank, world, local_rank):
     api.lib()
 
     T, k = 16, 8
-    w0, layers, xs = build_decode_workload(api, inputs, torch, device, rank)
+    NL = args.layers
+    w0, layers, xs = build_decode_workload(api, inputs, torch, device, rank, NL)
     E, D, F = layers[0].E, layers[0].D, layers[0].F
     bufs = [api.MoeBuffers(L, T, k) for L in layers]
     x_dev = [torch.from_numpy(x).to(torch.bfloat16).to(device) for x, _ in xs]
     l_dev = [torch.from_numpy(lg).to(device) for _, lg in xs]
     stream = torch.cuda.current_stream()
 
-    def step(i):
-        c = i % N_LAYER_COPIES
+    def eager_step(i):
+        c = i % NL
         api.moe_layer(layers[c], x_dev[c], l_dev[c], k, bufs=bufs[c], path="gemv")
 
     for i in range(args.warmup):
-        step(i)
+        eager_step(i)
     torch.cuda.synchronize()
     api.device_status(clear=True)
+
+    # One CUDA graph per layer copy; the library's per-launch profiling events are
+    # captured with the kernels, so every replay re-records them.
+    api.profile_enable(64 * NL)
+    api.profile_collect()
+    launches0 = api.launch_count()
+    graphs = []
+    if not args.eager:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for c in range(NL):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    eager_step(c)
+                graphs.append(g)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        launches_per_step = (api.launch_count() - launches0) // NL
+        for i in range(args.warmup):
+            graphs[i % NL].replay()
+        torch.cuda.synchronize()
+
+    def step(i):
+        if args.eager:
+            eager_step(i)
+        else:
+            graphs[i % NL].replay()
 
     # ---- device-timed region
     sampler = ClockSampler(local_rank)
     sampler.start()
-    api.profile_enable(16 * (args.steps + 1))
-    api.profile_collect()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -253,7 +283,7 @@ def run_ours(args, rank, world, local_rank):
     t_wall1 = time.time()
     if world > 1:
         dist.barrier()
-    launches = api.launch_count() - launches0
+    launches = (api.launch_count() - launches0) if args.eager else launches_per_step * args.steps
     stages = api.profile_collect()
     api.profile_disable()
     sampler.stop()
@@ -268,19 +298,24 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_max = float(t.item())
 
-    # ---- algorithmic bytes of the dominant kernel (gate/up GEMV) per launch
+    # ---- algorithmic bytes of the dominant kernel (gate/up GEMV) per launch: the stage
+    # totals cover the last replay of each layer copy's graph (eager: every step)
     counts = [b.routing.counts.cpu().numpy() for b in bufs]
     per_copy_bytes = [gateup_algorithmic_bytes(L, c) for L, c in zip(layers, counts)]
-    gu_bytes = sum(per_copy_bytes[i % N_LAYER_COPIES] for i in range(args.steps)) / max(args.steps, 1)
     gu_ms, gu_n = stages["gemv_gateup"]
+    if args.eager:
+        gu_bytes = sum(per_copy_bytes[i % NL] for i in range(args.steps)) / max(args.steps, 1)
+    else:
+        gu_bytes = sum(per_copy_bytes) / NL
     gu_avg_ms = gu_ms / max(gu_n, 1)
+    stage_avg = {k_: v[0] / v[1] for k_, v in stages.items() if v[1]}
     peaks, peak_src = load_peaks()
     achieved = gu_bytes / (gu_avg_ms * 1e-3) / 1e9
     prof = profile_traffic("moe_gemv_gateup_decode_t16")
     traffic = None
     if prof is not None:
         unit_bytes = float(prof["dram_bytes_per_unit"])
-        units = sum(int((c > 0).sum()) for c in counts) / N_LAYER_COPIES
+        units = sum(int((c > 0).sum()) for c in counts) / NL
         traffic = unit_bytes * units
 
     # ---- end to end through the public API with host buffers
@@ -289,7 +324,7 @@ def run_ours(args, rank, world, local_rank):
     pin_out = torch.empty((T, D), dtype=torch.float32).pin_memory()
 
     def e2e_step(i):
-        c = i % N_LAYER_COPIES
+        c = i % NL
         x_dev[c].copy_(pin_x[c], non_blocking=True)
         l_dev[c].copy_(pin_l[c], non_blocking=True)
         out = api.moe_layer(layers[c], x_dev[c], l_dev[c], k, bufs=bufs[c], path="gemv")
@@ -336,10 +371,11 @@ def run_ours(args, rank, world, local_rank):
         "config": {
             "workload": "moe_decode_t16", "experts": E, "hidden": D, "intermediate": F,
             "tokens": T, "top_k": k, "widths": "368/15/1 experts at K=2/3/4",
-            "layer_copies_cycled": N_LAYER_COPIES,
-            "l2": "inputs larger than L2: each step reads ~0.35 GB of bit streams; 4 layers "
-                  "(4.9 GB) cycled",
-            "path": "gemv", "parallelism": "replicas" if world > 1 else "single-gpu",
+            "layer_copies_cycled": NL,
+            "l2": "inputs larger than L2: each step reads ~0.35 GB of bit streams; %d layers "
+                  "(%.1f GB) cycled" % (NL, 1.23 * NL),
+            "path": "gemv", "launch": "eager" if args.eager else "cuda-graph replay per step",
+            "parallelism": "replicas" if world > 1 else "single-gpu",
         },
         "roofline": {
             "kernel": "moe_gateup_kernel (gate/up GEMV + SiLU)",
@@ -348,7 +384,7 @@ def run_ours(args, rank, world, local_rank):
             "peak_source": peak_src, "bytes_per_launch": gu_bytes,
             "avg_launch_ms": gu_avg_ms, "traffic": traffic,
         },
-        "stages_ms_per_step": {k_: v[0] / max(args.steps, 1) for k_, v in stages.items() if v[1]},
+        "stage_avg_launch_ms": stage_avg,
         "gpu_launches": launches,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

@@ -95,10 +95,12 @@ int tq_device_status(int32_t *flags_out, int clear);
  *   4 rotation of h, 5 GEMV down, 6 route_unpermute, 7 trellis_decode, 8 trellis_gemv,
  *   9 GEMM gate/up+SiLU, 10 GEMM down.
  * tq_profile_enable creates 2*max_launches events (host-side CUDA resources; call it
- * outside graph capture, and do not capture while it is enabled); launches beyond
- * max_launches are not recorded.  tq_profile_collect waits for the recorded events,
- * writes per-stage summed milliseconds and launch counts into the host arrays
- * stage_ms[n_stages] / stage_launches[n_stages], and clears the record.
+ * outside graph capture); launches beyond max_launches are not recorded.  A launch made
+ * during stream capture records its events as external event-record nodes of the graph,
+ * re-recorded at every replay, so a collect after replays reads the last replay.
+ * tq_profile_collect waits for the recorded events, writes per-stage summed
+ * milliseconds and launch counts into the host arrays stage_ms[n_stages] /
+ * stage_launches[n_stages] (skipping events never recorded), and clears the record.
  */
 unsigned long long tq_launch_count(void);
 int tq_profile_enable(int max_launches);

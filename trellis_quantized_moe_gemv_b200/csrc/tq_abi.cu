@@ -41,17 +41,27 @@ struct Profiler {
 static Profiler g_prof;
 static unsigned long long g_launches = 0;
 
+// Inside stream capture an event record becomes an external event-record node of the
+// graph (re-recorded at every replay); otherwise it is an ordinary record.
+static void record_event(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, s);
+}
+
 LaunchScope::LaunchScope(cudaStream_t s, int st) : stream(s), slot(-1) {
     ++g_launches;
     if (g_prof.on && g_prof.used < g_prof.capacity) {
         slot = g_prof.used++;
         g_prof.stage[slot] = st;
-        cudaEventRecord(g_prof.events[2 * slot], s);
+        record_event(g_prof.events[2 * slot], s);
     }
 }
 
 LaunchScope::~LaunchScope() {
-    if (slot >= 0) cudaEventRecord(g_prof.events[2 * slot + 1], stream);
+    if (slot >= 0) record_event(g_prof.events[2 * slot + 1], stream);
 }
 
 static void profile_release() {
@@ -98,8 +108,10 @@ TQ_API int tq_profile_collect(double *stage_ms, int32_t *stage_launches, int n_s
         if (cudaEventSynchronize(tq::g_prof.events[2 * l + 1]) != cudaSuccess) return TQ_ERR_CUDA;
         float ms = 0.f;
         if (cudaEventElapsedTime(&ms, tq::g_prof.events[2 * l], tq::g_prof.events[2 * l + 1]) !=
-            cudaSuccess)
-            return TQ_ERR_CUDA;
+            cudaSuccess) {
+            cudaGetLastError();   // a captured launch whose graph was never replayed
+            continue;
+        }
         const int st = tq::g_prof.stage[l];
         if (st >= 0 && st < n_stages) {
             stage_ms[st] += ms;
