@@ -76,6 +76,10 @@ const char *tq_status_string(int status);
 /* TQ_ABI_VERSION of the loaded library. */
 int tq_abi_version(void);
 
+/* Text of the most recent CUDA failure behind a TQ_ERR_CUDA return (static buffer,
+ * overwritten by the next failure; "" if none).  Host-only, not thread-safe. */
+const char *tq_last_error_string(void);
+
 /*
  * Device-side anomaly flags of the current device, OR-ed since the last clear:
  *   bit 0: a kernel met an expert id outside [0, E) or a route index outside [0, T*k)

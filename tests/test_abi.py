@@ -96,14 +96,19 @@ def _layer_struct(K=2, E=16, D=256, F=128, n_groups=1):
 def test_moe_workspace_and_layer_validation(lib):
     st = _layer_struct()
     need = lib.moe_trellis_workspace_size(ctypes.byref(st), 16, 8)
-    assert need == 128 * 128 * 4 + 128 * 128 * 2
+    gemv_need = 128 * 128 * 4 + 128 * 128 * 2
+    # the GEMM path also holds route-ordered activations (fp16), their row sums, h, h'
+    # and its tile list
+    gemm_need = 128 * 256 * 2 + 512 + 128 * 128 * 4 + 128 * 128 * 2 + 512 + 256
+    assert need == max(gemv_need, gemm_need)
     bad = _layer_struct(K=5)
     assert lib.moe_trellis_workspace_size(ctypes.byref(bad), 16, 8) == 0
     bad = _layer_struct(D=200)
     assert lib.moe_trellis_workspace_size(ctypes.byref(bad), 16, 8) == 0
     args = [FAKE] * 5
     # workspace too small
-    assert lib.moe_trellis_gemv(ctypes.byref(st), *args, 16, 8, FAKE, FAKE, need - 1, None) == 4
+    assert lib.moe_trellis_gemv(ctypes.byref(st), *args, 16, 8, FAKE, FAKE, gemv_need - 1, None) == 4
+    assert lib.moe_trellis_gemm(ctypes.byref(st), *args, 16, 8, FAKE, FAKE, gemm_need - 1, None) == 4
     assert lib.moe_trellis_gemv(ctypes.byref(st), *args, 16, 8, FAKE, None, need, None) == 4
     # misaligned activations
     assert lib.moe_trellis_gemv(ctypes.byref(st), MISALIGNED, *args[1:], 16, 8, FAKE, FAKE, need,

@@ -47,6 +47,7 @@ _VP, _I, _I64, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_siz
 SIGNATURES = {
     "tq_status_string": ([_I], ctypes.c_char_p),
     "tq_abi_version": ([], _I),
+    "tq_last_error_string": ([], ctypes.c_char_p),
     "tq_device_status": ([_VP, _I], _I),
     "tq_launch_count": ([], ctypes.c_ulonglong),
     "tq_profile_enable": ([_I], _I),
@@ -96,6 +97,8 @@ def _fn(name):
 def _check(status, name):
     if status != 0:
         msg = _fn("tq_status_string")(status).decode()
+        if status == 5:
+            msg += " (%s)" % _fn("tq_last_error_string")().decode()
         raise TQError("%s failed: %s" % (name, msg))
 
 

@@ -1,6 +1,8 @@
 // Status codes, version and the device anomaly flag word of the C ABI.
 #include "tq_common.cuh"
 
+#include <stdio.h>
+
 TQ_API const char *tq_status_string(int status) {
     switch (status) {
         case TQ_OK: return "TQ_OK";
@@ -15,6 +17,23 @@ TQ_API const char *tq_status_string(int status) {
 }
 
 TQ_API int tq_abi_version(void) { return TQ_ABI_VERSION; }
+
+namespace tq {
+static char g_last_error[256] = "";
+
+int record_error(const char *what) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s", what ? what : "");
+    return TQ_ERR_CUDA;
+}
+
+int record_cuda_error(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(e));
+    return TQ_ERR_CUDA;
+}
+}  // namespace tq
+
+TQ_API const char *tq_last_error_string(void) { return tq::g_last_error; }
 
 TQ_API int tq_device_status(int32_t *flags_out, int clear) {
     if (!flags_out) return TQ_ERR_INVALID_ARG;

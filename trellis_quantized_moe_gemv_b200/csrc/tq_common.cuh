@@ -46,9 +46,14 @@ struct LaunchScope {
     int slot;
 };
 
+// Text of the most recent CUDA failure seen by the library (tq_last_error_string).
+int record_error(const char *what);
+int record_cuda_error(const char *what);
+
 inline int launch_status() {
     cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+    if (e == cudaSuccess) return TQ_OK;
+    return record_error(cudaGetErrorString(e));
 }
 
 inline int num_sms() {

@@ -1,9 +1,595 @@
-// Prefill-sized routed-expert GEMM on tcgen05 tensor cores.
+// Prefill-sized routed-expert GEMM on the 5th-generation tensor cores (tcgen05).
 //
-// Not implemented yet in this build: the entry point validates its arguments and
-// returns TQ_ERR_UNSUPPORTED, so callers fail loudly instead of getting a result from
-// another path.
+// Same computation as moe_trellis_gemv (T16 codebook and 16x16 column-major tiles,
+// "How T16 works" items 1, 2 and 4 of the dsx T16 card; SwiGLU experts with fused
+// gate/up post-processing, its "October 25 runtime checkpoint"), for hundreds to
+// thousands of routes per expert, where each decoded weight feeds a 256-route MMA.
+//
+// Data flow of one launch (gate/up or down):
+//   * The routes' activations are a route-ordered fp16 matrix B_all [T*k][Kdim]
+//     (gate/up: the rotated tokens gathered to their route rows by route_rows_kernel;
+//     down: the rotated h'), with per-route row sums.
+//   * A CTA owns one tile: (expert, block of <= 256 of its routes, 128 weight rows).
+//     Per K-block of 64 columns (4 stages in flight):
+//       - producer warp: bulk-copies the 8 strips' 4 trellis tiles (the bit stream)
+//         and TMA-loads the routes' 64-column slab (128-byte swizzle) into the stage;
+//       - two decode groups of 4 warps (alternating K-blocks) decode the 8192 weights
+//         of the stage into the K-major 128-byte-swizzled A buffer as fp16 subnormals
+//         t * 2^-24 (exact; t = lo + hi of the T16 product);
+//       - one thread issues 4 tcgen05.mma (M=128, N<=256, K=16, fp32 accumulator in
+//         tensor memory) and commits them to the stage's "empty" barrier.
+//   * Epilogue (4 warps, one per tensor-memory lane quarter): tcgen05.ld of the
+//     accumulator, D -> s * 2^-12 * (2^24 D - 255 * rowsum), then
+//       gate/up: strips are interleaved gate/up per 16 rows, so lane l and l^16 hold g
+//                and u of the same intermediate row: h = silu(g) * u (fp32);
+//       down:    y_perm (fp32).
+// Every wait on an mbarrier is bounded; a wait that gives up raises device flag bit 1,
+// the CTA stops issuing work, drains what it issued and releases its tensor memory.
 #include "tq_common.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+namespace tq {
+
+constexpr int kGBM = 128;          // weight rows per tile
+constexpr int kGBN = 256;          // max routes per tile
+constexpr int kGBK = 64;           // K columns per stage
+constexpr int kGStages = 4;
+constexpr int kGDecodeWarps = 8;   // two groups of 4
+constexpr int kGThreads = (2 + kGDecodeWarps) * 32;
+constexpr int kGBitsSlot = 512;    // per strip per stage: 4 tiles x up to 128 B
+constexpr int kGBoxes = 4;         // TMA boxes of 32, 64, 128, 256 rows
+
+struct __align__(1024) GemmSmem {
+    __half a[kGStages][kGBM * kGBK];      // 16 KB per stage, 1024-byte aligned
+    __half b[kGStages][kGBN * kGBK];      // 32 KB per stage
+    unsigned char bits[kGStages][8 * kGBitsSlot];
+    uint64_t full[kGStages];              // producer -> decoders (bits + B landed)
+    uint64_t decoded[kGStages];           // decoders -> MMA (A written)
+    uint64_t empty[kGStages];             // MMA -> producer (stage consumed)
+    uint64_t acc_full;                    // MMA -> epilogue
+    uint64_t mma_done;                    // MMA drain on early exit
+    uint32_t tmem_base;
+    int32_t abort;                        // a role gave up
+};
+
+struct GemmMaps {
+    CUtensorMap b[kGBoxes];               // route-ordered activations, box rows 32..256
+};
+
+// ------------------------------------------------------------------------------ PTX
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t base, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base), "r"(cols) : "memory");
+}
+
+// K-major operand in shared memory with the 128-byte swizzle: rows of 128 B, 8-row
+// atoms 1024 B apart (SBO), start address advanced by 32 B per K=16 step.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;                 // leading byte offset (unused for this layout)
+    d |= (uint64_t)(1024u >> 4) << 32;       // stride byte offset: 8-row atoms
+    d |= (uint64_t)1u << 46;                 // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                 // SWIZZLE_128B
+    return d;
+}
+
+// kind::f16 instruction descriptor: fp16 A and B (K-major), fp32 D, M = 128, N.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kGBM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns; thread i of the warp gets lane base+i.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------ decode
+
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Product of the window at compile-time bit offset O, bytes [0, 0, lo, hi].
+template <int O, int NS>
+__device__ __forceinline__ uint32_t prod_hi(const uint32_t (&v)[NS]) {
+    constexpr int wi = O >> 5, sh = O & 31;
+    uint32_t bottom;
+    if constexpr (sh == 0) bottom = v[wi];
+    else bottom = funnel_r(v[wi], v[wi + 1], sh);
+    return bottom * (kT16Mult << 16);
+}
+
+// Rows R of the lane's 4 columns -> 4 fp16 subnormals t * 2^-24, stored (8 bytes) into
+// the swizzled A stage at row m = row0 + R, chunk c.
+template <int K, int R>
+__device__ __forceinline__ void decode_rows(const uint32_t (&v)[2 * K + 1], unsigned char *a_stage, int row0,
+                                            int chunk, int half_off) {
+    if constexpr (R < 16) {
+        const uint32_t p0 = prod_hi<0 * 16 * K + K * R>(v), p1 = prod_hi<1 * 16 * K + K * R>(v);
+        const uint32_t p2 = prod_hi<2 * 16 * K + K * R>(v), p3 = prod_hi<3 * 16 * K + K * R>(v);
+        const uint32_t ab = hadd2_u32(prmt(p0, p1, 0x4602u), prmt(p0, p1, 0x5713u));
+        const uint32_t cd = hadd2_u32(prmt(p2, p3, 0x4602u), prmt(p2, p3, 0x5713u));
+        const int m = row0 + R;
+        *reinterpret_cast<uint2 *>(a_stage + m * 128 + ((chunk ^ (m & 7)) << 4) + half_off) = make_uint2(ab, cd);
+        decode_rows<K, R + 1>(v, a_stage, row0, chunk, half_off);
+    }
+}
+
+// Decode one stage: thread (wl, lane) of a 4-warp group handles strip slot sig,
+// column tile j of the K-block, columns 4*t4..4*t4+3, all 16 rows.
+template <int K>
+__device__ __forceinline__ void decode_stage(const unsigned char *bits_stage, unsigned char *a_stage, int wl,
+                                             int lane) {
+    constexpr int TB = 32 * K;
+    const int pair = wl * 8 + (lane >> 2);
+    const int sig = pair >> 2, j = pair & 3, t4 = lane & 3;
+    const unsigned char *tile = bits_stage + sig * kGBitsSlot + j * TB;
+    uint32_t v[2 * K + 1];
+    if constexpr (K == 2) {
+        uint4 a = *reinterpret_cast<const uint4 *>(tile + 16 * t4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else if constexpr (K == 3) {
+        const uint2 *q = reinterpret_cast<const uint2 *>(tile + 24 * t4);
+        uint2 a = q[0], b = q[1], c = q[2];
+        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y; v[4] = c.x; v[5] = c.y;
+    } else {
+        const uint4 *q = reinterpret_cast<const uint4 *>(tile + 32 * t4);
+        uint4 a = q[0], b = q[1];
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+    v[2 * K] = *reinterpret_cast<const uint32_t *>(tile + 8 * K * ((t4 + 1) & 3));
+    const int kc = 16 * j + 4 * t4;   // first K column of the lane within the stage
+    decode_rows<K, 0>(v, a_stage, 16 * sig, kc >> 3, (kc & 7) * 2);
+}
+
+// ------------------------------------------------------------------------------ kernel
+
+struct GemmArgs {
+    tq_moe_layer L;
+    const int32_t *offsets;
+    const int32_t *tiles;        // [0] = count, then (expert, first route) pairs
+    const float *rowsum;         // [T*k] sum of each route's activation row
+    float *out;                  // gate/up: h [T*k][F]; down: y [T*k][D]
+    int kdim;                    // D (gate/up) or F (down)
+};
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kGThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs args) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    // the stage buffers need 1024-byte alignment (128-byte swizzle atoms)
+    GemmSmem &sm = *reinterpret_cast<GemmSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const tq_moe_layer &L = args.L;
+
+    const int t = blockIdx.y, mt = blockIdx.x;
+    if (t >= args.tiles[0]) return;
+    const int e = args.tiles[1 + 2 * t], n0 = args.tiles[2 + 2 * t];
+    ExpertRef ex;
+    if (!expert_ref(L, e, ex)) {
+        if (threadIdx.x == 0) raise_flag(1);
+        return;
+    }
+    const int r0 = args.offsets[e], ne = args.offsets[e + 1] - r0;
+    const int n = min(kGBN, ne - n0);
+    if (n <= 0) return;
+    int box = 0;
+    while ((32 << box) < n) ++box;          // box rows 32 << box >= n
+    const int nmma = max(16, (n + 15) & ~15);
+    const int num_kb = args.kdim / kGBK;
+    const int tiles_per_strip = args.kdim / 16;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.decoded[s], 4);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.mma_done, 1);
+        sm.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(&sm.tmem_base, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = sm.tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        const int K = ex.K;
+        const int strip_bytes = 4 * 32 * K;
+        const uint32_t *strip_base = nullptr;
+        if (lane < 8) {
+            if (GATEUP) strip_base = ((lane & 1) ? ex.up : ex.gate) + (size_t)(mt * 4 + (lane >> 1)) * tiles_per_strip * (8 * K);
+            else strip_base = ex.down + (size_t)(mt * 8 + lane) * tiles_per_strip * (8 * K);
+        }
+        uint32_t parity = 0;
+        bool ok = true;
+        int issued = 0;
+        for (int kb = 0; kb < num_kb && ok; ++kb) {
+            const int s = kb % kGStages;
+            if (kb >= kGStages) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.empty[s], (parity >> s) & 1u));
+                parity ^= 1u << s;
+                if (!ok || *(volatile int32_t *)&sm.abort) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.full[s], 8u * strip_bytes + (32u << box) * 128u);
+                tma_load_2d(sm.b[s], &maps.b[box], kb * kGBK, r0 + n0, &sm.full[s]);
+            }
+            __syncwarp();
+            if (lane < 8)
+                bulk_g2s(sm.bits[s] + lane * kGBitsSlot, strip_base + (size_t)kb * 4 * (8 * K), strip_bytes,
+                         &sm.full[s]);
+            ++issued;
+        }
+        if (!ok) {
+            sm.abort = 1;
+            // drain: wait (bounded) for every stage this warp filled last
+            for (int kb = max(0, issued - kGStages); kb < issued; ++kb) {
+                const int s = kb % kGStages;
+                const uint32_t ph = ((kb / kGStages) & 1u);
+                mbar_wait_bounded(&sm.full[s], ph);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint32_t idesc = umma_idesc_f16(nmma);
+        uint32_t parity = 0;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+            const int s = kb % kGStages;
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.decoded[s], (parity >> s) & 1u));
+            parity ^= 1u << s;
+            if (!ok || *(volatile int32_t *)&sm.abort) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+#pragma unroll
+                for (int k = 0; k < kGBK / 16; ++k)
+                    umma_f16(tmem_d, umma_desc_sw128(a0 + 32 * k), umma_desc_sw128(b0 + 32 * k), idesc,
+                             (kb | k) != 0);
+                umma_commit(&sm.empty[s]);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) umma_commit(ok ? &sm.acc_full : &sm.mma_done);
+        __syncwarp();
+        if (!ok) {
+            sm.abort = 1;
+            mbar_wait_bounded(&sm.mma_done, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ decoders
+        const int dw = warp - 2;
+        const int group = dw >> 2, wl = dw & 3;
+        uint32_t parity = 0;
+        bool ok = true;
+        for (int kb = group; kb < num_kb; kb += 2) {
+            const int s = kb % kGStages;
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[s], (parity >> s) & 1u));
+            parity ^= 1u << s;
+            if (!ok || *(volatile int32_t *)&sm.abort) {
+                ok = false;
+                break;
+            }
+            unsigned char *a_stage = reinterpret_cast<unsigned char *>(sm.a[s]);
+            if (ex.K == 2) decode_stage<2>(sm.bits[s], a_stage, wl, lane);
+            else if (ex.K == 3) decode_stage<3>(sm.bits[s], a_stage, wl, lane);
+            else decode_stage<4>(sm.bits[s], a_stage, wl, lane);
+            fence_proxy_async();      // make the generic-proxy writes visible to the MMA
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.decoded[s]);
+        }
+        if (!ok) sm.abort = 1;
+        // ------------------------------------------------------------ epilogue
+        if (group == 1) {
+            const int q = warp & 3;             // tensor-memory lane quarter of this warp
+            const bool acc_ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.acc_full, 0));
+            if (acc_ok && !*(volatile int32_t *)&sm.abort) {
+                tc_fence_after();
+                const int row = 32 * q + lane;  // weight row of the tile = tensor-memory lane
+                for (int c0 = 0; c0 < nmma; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem_d + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+                    if (GATEUP) {
+                        const int f = (mt * 4 + q) * 16 + (lane & 15);
+                        const float sg = __half2float(ex.s_gate[f]), su = __half2float(ex.s_up[f]);
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const float dv = __uint_as_float(v[c]);
+                            const float du = __shfl_xor_sync(0xffffffffu, dv, 16);
+                            const int col = c0 + c;
+                            if (lane < 16 && col < n) {
+                                const int route = r0 + n0 + col;
+                                const float sx = args.rowsum[route];
+                                const float g = sg * kKappa * fmaf(16777216.0f, dv, -255.0f * sx);
+                                const float u = su * kKappa * fmaf(16777216.0f, du, -255.0f * sx);
+                                args.out[(size_t)route * L.F + f] = silu_f32(g) * u;
+                            }
+                        }
+                    } else {
+                        const int d = mt * kGBM + row;
+                        const float sd = __half2float(ex.s_down[d]);
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const int col = c0 + c;
+                            if (col < n) {
+                                const int route = r0 + n0 + col;
+                                const float sx = args.rowsum[route];
+                                args.out[(size_t)route * L.D + d] =
+                                    sd * kKappa * fmaf(16777216.0f, __uint_as_float(v[c]), -255.0f * sx);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_d, 256);
+    }
+}
+
+// ------------------------------------------------------------------------------ helpers
+
+// Route-ordered fp16 activation rows, one warp per destination row j: the source row is
+// perm[j] / k (the token of grouped route j) or j itself when perm is null; ROTATE
+// applies the 128-wide rotation on the way.  rowsum[j] = fp32 sum of the stored fp16
+// values.  An out-of-range source raises device flag bit 0 and stores zeros.
+template <typename T, bool ROTATE>
+__global__ void __launch_bounds__(256) route_rows_kernel(const T *__restrict__ x, int dst_rows, int cols,
+                                                         const int32_t *__restrict__ perm, int k, int src_rows,
+                                                         __half *__restrict__ dst, float *__restrict__ rowsum) {
+    const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (j >= dst_rows) return;
+    const int src = perm ? perm[j] / k : j;
+    const bool valid = src >= 0 && src < src_rows && (!perm || perm[j] >= 0);
+    if (!valid && lane == 0) raise_flag(1);
+    float sum = 0.f;
+    for (int c = 0; c < cols; c += 128) {
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        if (valid) {
+            float4 f = load4<T>(x + (size_t)src * cols + c + 4 * lane);
+            v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+            if (ROTATE) fwht128_warp(v, lane);
+        }
+        __half2 lo = __floats2half2_rn(v[0], v[1]);
+        __half2 hi = __floats2half2_rn(v[2], v[3]);
+        const float2 lf = __half22float2(lo), hf = __half22float2(hi);
+        sum += (lf.x + lf.y) + (hf.x + hf.y);
+        uint2 u;
+        u.x = *reinterpret_cast<uint32_t *>(&lo);
+        u.y = *reinterpret_cast<uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(dst + (size_t)j * cols + c + 4 * lane) = u;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) rowsum[j] = sum;
+}
+
+// Tiles of <= 256 routes per active expert: out[0] = count, then (expert, first route).
+__global__ void __launch_bounds__(1024) gemm_tile_list_kernel(const int32_t *__restrict__ offsets,
+                                                              const int32_t *__restrict__ active_ids,
+                                                              const int32_t *__restrict__ n_active_p, int max_tiles,
+                                                              int32_t *__restrict__ out) {
+    __shared__ int32_t warp_sum[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n_active = *n_active_p;
+    int running = 0;
+    for (int base = 0; base < n_active; base += 1024) {
+        const int a = base + tid;
+        int e = -1, cnt = 0;
+        if (a < n_active) {
+            e = active_ids[a];
+            cnt = (offsets[e + 1] - offsets[e] + kGBN - 1) / kGBN;
+        }
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) warp_sum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int s = warp_sum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int v = __shfl_up_sync(0xffffffffu, s, o);
+                if (lane >= o) s += v;
+            }
+            warp_sum[lane] = s;
+        }
+        __syncthreads();
+        const int excl = running + (warp ? warp_sum[warp - 1] : 0) + incl - cnt;
+        for (int i = 0; i < cnt; ++i) {
+            const int ti = excl + i;
+            if (ti < max_tiles) {
+                out[1 + 2 * ti] = e;
+                out[2 + 2 * ti] = i * kGBN;
+            }
+        }
+        running += warp_sum[31];
+        __syncthreads();
+    }
+    if (tid == 0) out[0] = min(running, max_tiles);
+}
+
+// ------------------------------------------------------------------------------ host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// Route-ordered fp16 activations [rows][cols] -> 4 maps with boxes of 64 columns x
+// {32, 64, 128, 256} rows and the 128-byte swizzle.
+static int make_maps(const __half *base, int rows, int cols, GemmMaps &maps) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return record_error("cuTensorMapEncodeTiled entry point not found");
+    for (int b = 0; b < kGBoxes; ++b) {
+        cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+        cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(__half)};
+        cuuint32_t box[2] = {(cuuint32_t)kGBK, (cuuint32_t)(32 << b)};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&maps.b[b], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void *)base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return record_error("cuTensorMapEncodeTiled failed");
+    }
+    return TQ_OK;
+}
+
+static size_t align256_g(size_t b) { return (b + 255) & ~(size_t)255; }
+
+static int gemm_max_tiles(int T, int k, int E) {
+    const long long routes = (long long)T * k;
+    return (int)(routes / kGBN + min((long long)E, routes) + 1);
+}
+
+size_t gemm_workspace_bytes(const tq_moe_layer *L, int T, int k) {
+    const size_t R = (size_t)T * k;
+    return align256_g(R * L->D * sizeof(__half)) + align256_g(R * sizeof(float)) +
+           align256_g(R * L->F * sizeof(float)) + align256_g(R * L->F * sizeof(__half)) +
+           align256_g(R * sizeof(float)) + align256_g((1 + 2 * (size_t)gemm_max_tiles(T, k, L->E)) * sizeof(int32_t));
+}
+
+int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offsets, const int32_t *perm,
+                 const int32_t *active_ids, const int32_t *n_active, int T, int k, float *y_perm, void *ws,
+                 cudaStream_t s) {
+    static bool configured = false;
+    if (!configured) {
+        const int bytes = (int)(sizeof(GemmSmem) + 1024);
+        if (cudaFuncSetAttribute(moe_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+                cudaSuccess)
+            return record_cuda_error("cudaFuncSetAttribute(moe_gemm_kernel)");
+        configured = true;
+    }
+    const int R = T * k;
+    char *w = reinterpret_cast<char *>(ws);
+    __half *xp = reinterpret_cast<__half *>(w);
+    w += align256_g((size_t)R * L->D * sizeof(__half));
+    float *sxp = reinterpret_cast<float *>(w);
+    w += align256_g((size_t)R * sizeof(float));
+    float *h = reinterpret_cast<float *>(w);
+    w += align256_g((size_t)R * L->F * sizeof(float));
+    __half *hr = reinterpret_cast<__half *>(w);
+    w += align256_g((size_t)R * L->F * sizeof(__half));
+    float *shr = reinterpret_cast<float *>(w);
+    w += align256_g((size_t)R * sizeof(float));
+    int32_t *tiles = reinterpret_cast<int32_t *>(w);
+    const int max_tiles = gemm_max_tiles(T, k, L->E);
+
+    GemmMaps maps_x, maps_h;
+    int st = make_maps(xp, R, L->D, maps_x);
+    if (st) return st;
+    st = make_maps(hr, R, L->F, maps_h);
+    if (st) return st;
+
+    const size_t smem = sizeof(GemmSmem) + 1024;
+    {
+        LaunchScope ls(s, kStageGemmGateUp);
+        gemm_tile_list_kernel<<<1, 1024, 0, s>>>(offsets, active_ids, n_active, max_tiles, tiles);
+    }
+    st = launch_status();
+    if (st) return st;
+    {
+        // x_rot is already rotated: copy its rows to their route rows (+ row sums)
+        LaunchScope ls(s, kStageGemmGateUp);
+        route_rows_kernel<__half, false><<<(R * 32 + 255) / 256, 256, 0, s>>>(x_rot, R, L->D, perm, k, T, xp, sxp);
+    }
+    st = launch_status();
+    if (st) return st;
+    {
+        GemmArgs a{*L, offsets, tiles, sxp, h, L->D};
+        LaunchScope ls(s, kStageGemmGateUp);
+        moe_gemm_kernel<true><<<dim3(L->F / 64, max_tiles), kGThreads, smem, s>>>(maps_x, a);
+    }
+    st = launch_status();
+    if (st) return st;
+    {
+        LaunchScope ls(s, kStageRotateH);
+        route_rows_kernel<float, true><<<(R * 32 + 255) / 256, 256, 0, s>>>(h, R, L->F, nullptr, 1, R, hr, shr);
+    }
+    st = launch_status();
+    if (st) return st;
+    {
+        GemmArgs a{*L, offsets, tiles, shr, y_perm, L->F};
+        LaunchScope ls(s, kStageGemmDown);
+        moe_gemm_kernel<false><<<dim3(L->D / kGBM, max_tiles), kGThreads, smem, s>>>(maps_h, a);
+    }
+    return launch_status();
+}
+
+}  // namespace tq
 
 int moe_validate_call(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
                       const int32_t *perm, const int32_t *active_ids, const int32_t *n_active, int T,
@@ -12,8 +598,10 @@ int moe_validate_call(const tq_moe_layer *layer, const uint16_t *x_rot, const in
 TQ_API int moe_trellis_gemm(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
                             const int32_t *perm, const int32_t *active_ids, const int32_t *n_active, int T,
                             int k, float *y_perm, void *ws, size_t ws_bytes, tq_stream stream) {
-    (void)stream;
     int st = moe_validate_call(layer, x_rot, offsets, perm, active_ids, n_active, T, k, y_perm, ws, ws_bytes);
     if (st || T == 0) return st;
-    return TQ_ERR_UNSUPPORTED;
+    if (ws_bytes < tq::gemm_workspace_bytes(layer, T, k)) return TQ_ERR_WORKSPACE;
+    if ((long long)T * k / tq::kGBN + layer->E + 1 > 65535) return TQ_ERR_UNSUPPORTED;
+    return tq::run_moe_gemm(layer, reinterpret_cast<const __half *>(x_rot), offsets, perm, active_ids, n_active,
+                            T, k, y_perm, ws, (cudaStream_t)stream);
 }

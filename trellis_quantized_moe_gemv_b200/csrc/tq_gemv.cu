@@ -654,9 +654,14 @@ TQ_API int trellis_gemv(const uint32_t *bits, const uint16_t *scales, int K, int
     }
 }
 
+namespace tq {
+size_t gemm_workspace_bytes(const tq_moe_layer *L, int T, int k);
+}
+
 TQ_API size_t moe_trellis_workspace_size(const tq_moe_layer *layer, int T, int k) {
     if (validate_layer(layer) != TQ_OK || T < 0 || k < 1) return 0;
-    return workspace_bytes(layer, T, k);
+    const size_t gemv = workspace_bytes(layer, T, k), gemm = tq::gemm_workspace_bytes(layer, T, k);
+    return gemv > gemm ? gemv : gemm;
 }
 
 int moe_validate_call(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
