@@ -38,11 +38,13 @@ def parse_args():
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="moe_decode_t16", choices=["moe_decode_t16"])
+    p.add_argument("--workload", default="moe_decode_t16", choices=["moe_decode_t16", "moe_prefill_t8192"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--layers", type=int, default=4,
                    help="synthetic layer copies cycled through (4 keep every step's weights out of L2)")
     p.add_argument("--eager", action="store_true", help="launch every step from the host instead of a CUDA graph")
+    p.add_argument("--tokens", type=int, default=None, help="override the workload's token count (profiling runs)")
+    p.add_argument("--experts", type=int, default=None, help="override the workload's expert count (profiling runs)")
     return p.parse_args()
 
 
@@ -203,6 +205,31 @@ def gateup_algorithmic_bytes(layer, counts):
     return total
 
 
+def build_prefill_workload(api, inputs, device, rank, T=8192, E=384):
+    """The all-K=3 384-expert layer with 8192 Zipf(1.1)-routed tokens: one step touches
+    every expert (1.8 GB of bit streams), far beyond L2, so one layer copy suffices."""
+    w0 = inputs.moe_prefill_t8192(seed=1004 + 100 * rank, T=T, E=E)
+    layers = [api.DeviceLayer.from_synthetic(w0["layer"], device)]
+    return w0, layers, [(w0["x"], w0["logits"])]
+
+
+def gateup_flops(layer, T, k):
+    """Algorithmic FLOPs of one gate/up launch: 2 per weight per routed token, for the
+    gate and up projections of every route."""
+    return 2.0 * T * k * 2 * layer.F * layer.D
+
+
+WORKLOADS = {
+    "moe_decode_t16": dict(T=16, path="gemv", stage="gemv_gateup",
+                           kernel="moe_gemv_items_kernel<1> (gate/up GEMV + SiLU)",
+                           widths="368/15/1 experts at K=2/3/4", routing="top-8 of N(0,1) logits"),
+    "moe_prefill_t8192": dict(T=8192, path="gemm", stage="gemm_gateup",
+                              kernel="moe_gemm_kernel<1> (gate/up tcgen05 GEMM + SiLU)",
+                              widths="all 384 experts at K=3",
+                              routing="top-8 of log p + Gumbel, p ~ rank^-1.1 (Zipf)"),
+}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -219,9 +246,16 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     api.lib()
 
-    T, k = 16, 8
-    NL = args.layers
-    w0, layers, xs = build_decode_workload(api, inputs, torch, device, rank, NL)
+    wl = WORKLOADS[args.workload]
+    T, k = (args.tokens or wl["T"]), 8
+    if args.workload == "moe_decode_t16":
+        if args.tokens or args.experts:
+            raise SystemExit("--tokens/--experts apply to the prefill workload")
+        NL = args.layers
+        w0, layers, xs = build_decode_workload(api, inputs, torch, device, rank, NL)
+    else:
+        NL = 1
+        w0, layers, xs = build_prefill_workload(api, inputs, device, rank, T=T, E=args.experts or 384)
     E, D, F = layers[0].E, layers[0].D, layers[0].F
     bufs = [api.MoeBuffers(L, T, k) for L in layers]
     x_dev = [torch.from_numpy(x).to(torch.bfloat16).to(device) for x, _ in xs]
@@ -230,7 +264,7 @@ def run_ours(args, rank, world, local_rank):
 
     def eager_step(i):
         c = i % NL
-        api.moe_layer(layers[c], x_dev[c], l_dev[c], k, bufs=bufs[c], path="gemv")
+        api.moe_layer(layers[c], x_dev[c], l_dev[c], k, bufs=bufs[c], path=wl["path"])
 
     for i in range(args.warmup):
         eager_step(i)
@@ -298,25 +332,43 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_max = float(t.item())
 
-    # ---- algorithmic bytes of the dominant kernel (gate/up GEMV) per launch: the stage
-    # totals cover the last replay of each layer copy's graph (eager: every step)
+    # ---- the dominant kernel (gate/up) per launch: algorithmic bytes (decode GEMV,
+    # HBM-bound) or FLOPs (prefill GEMM, tensor-bound) over its average duration; the
+    # stage totals cover the last replay of each layer copy's graph (eager: every step)
     counts = [b.routing.counts.cpu().numpy() for b in bufs]
-    per_copy_bytes = [gateup_algorithmic_bytes(L, c) for L, c in zip(layers, counts)]
-    gu_ms, gu_n = stages["gemv_gateup"]
-    if args.eager:
-        gu_bytes = sum(per_copy_bytes[i % NL] for i in range(args.steps)) / max(args.steps, 1)
-    else:
-        gu_bytes = sum(per_copy_bytes) / NL
-    gu_avg_ms = gu_ms / max(gu_n, 1)
+    g_ms, g_n = stages[wl["stage"]]
+    g_avg_ms = g_ms / max(g_n, 1)
     stage_avg = {k_: v[0] / v[1] for k_, v in stages.items() if v[1]}
     peaks, peak_src = load_peaks()
-    achieved = gu_bytes / (gu_avg_ms * 1e-3) / 1e9
-    prof = profile_traffic("moe_gemv_gateup_decode_t16")
-    traffic = None
-    if prof is not None:
-        unit_bytes = float(prof["dram_bytes_per_unit"])
-        units = sum(int((c > 0).sum()) for c in counts) / NL
-        traffic = unit_bytes * units
+    if wl["path"] == "gemv":
+        per_copy_bytes = [gateup_algorithmic_bytes(L, c) for L, c in zip(layers, counts)]
+        if args.eager:
+            unit_work = sum(per_copy_bytes[i % NL] for i in range(args.steps)) / max(args.steps, 1)
+        else:
+            unit_work = sum(per_copy_bytes) / NL
+        achieved = unit_work / (g_avg_ms * 1e-3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        prof = profile_traffic("moe_gemv_gateup_decode_t16")
+        traffic = None
+        if prof is not None:
+            units = sum(int((c > 0).sum()) for c in counts) / NL
+            traffic = float(prof["dram_bytes_per_unit"]) * units
+        roofline = {"kernel": wl["kernel"], "bound": "hbm", "achieved": achieved, "peak": peak,
+                    "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_src + " (copy bandwidth)",
+                    "bytes_per_launch": unit_work, "avg_launch_ms": g_avg_ms, "traffic": traffic}
+    else:
+        unit_work = gateup_flops(layers[0], T, k)
+        E = layers[0].E
+        achieved = unit_work / (g_avg_ms * 1e-3) / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        prof = profile_traffic("moe_gemm_gateup_prefill_t8192")
+        traffic = None
+        if prof is not None:
+            traffic = float(prof["dram_bytes_per_unit"]) * float(prof.get("units", 1))
+        roofline = {"kernel": wl["kernel"], "bound": "tensor", "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak,
+                    "peak_source": peak_src + " (dense bf16 GEMM, sustained; fp16 dense rate is the same)",
+                    "flops_per_launch": unit_work, "avg_launch_ms": g_avg_ms, "traffic": traffic}
 
     # ---- end to end through the public API with host buffers
     pin_x = [torch.from_numpy(x).to(torch.bfloat16).pin_memory() for x, _ in xs]
@@ -327,7 +379,7 @@ def run_ours(args, rank, world, local_rank):
         c = i % NL
         x_dev[c].copy_(pin_x[c], non_blocking=True)
         l_dev[c].copy_(pin_l[c], non_blocking=True)
-        out = api.moe_layer(layers[c], x_dev[c], l_dev[c], k, bufs=bufs[c], path="gemv")
+        out = api.moe_layer(layers[c], x_dev[c], l_dev[c], k, bufs=bufs[c], path=wl["path"])
         pin_out.copy_(out, non_blocking=True)
 
     for i in range(args.warmup):
@@ -352,7 +404,7 @@ def run_ours(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w0, routes=16)
+        cpu = cpu_baseline(w0, routes=16, name=args.workload)
 
     tokens = T * args.steps * world
     line = {
@@ -369,21 +421,16 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "f16",
         "data": "synthetic",
         "config": {
-            "workload": "moe_decode_t16", "experts": E, "hidden": D, "intermediate": F,
-            "tokens": T, "top_k": k, "widths": "368/15/1 experts at K=2/3/4",
+            "workload": args.workload, "experts": E, "hidden": D, "intermediate": F,
+            "tokens": T, "top_k": k, "widths": wl["widths"], "routing": wl["routing"],
             "layer_copies_cycled": NL,
-            "l2": "inputs larger than L2: each step reads ~0.35 GB of bit streams; %d layers "
-                  "(%.1f GB) cycled" % (NL, 1.23 * NL),
-            "path": "gemv", "launch": "eager" if args.eager else "cuda-graph replay per step",
+            "l2": ("inputs larger than L2: each step reads ~0.35 GB of bit streams; %d layers "
+                   "(%.1f GB) cycled" % (NL, 1.23 * NL)) if wl["path"] == "gemv" else
+                  "inputs larger than L2: each step reads all 1.8 GB of bit streams",
+            "path": wl["path"], "launch": "eager" if args.eager else "cuda-graph replay per step",
             "parallelism": "replicas" if world > 1 else "single-gpu",
         },
-        "roofline": {
-            "kernel": "moe_gateup_kernel (gate/up GEMV + SiLU)",
-            "bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]),
-            "unit": "GB/s", "frac": achieved / float(peaks["hbm_gbs"]),
-            "peak_source": peak_src, "bytes_per_launch": gu_bytes,
-            "avg_launch_ms": gu_avg_ms, "traffic": traffic,
-        },
+        "roofline": roofline,
         "stage_avg_launch_ms": stage_avg,
         "gpu_launches": launches,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": h2d,
@@ -398,7 +445,7 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
-def cpu_baseline(w0, routes):
+def cpu_baseline(w0, routes, name="moe_decode_t16"):
     """The fp64 CPU oracle, as it stands, on `routes` (token, expert) routes of layer
     copy 0 (single-threaded BLAS); reported in tok/s (k routes = one token)."""
     from oracle import layer as OL
@@ -425,8 +472,8 @@ def cpu_baseline(w0, routes):
     if limiter is not None:
         limiter.unregister()
     return {"value": (done / k) / dt, "unit": "tok/s", "cores": 1, "kind": "oracle",
-            "sample": "%d routes (= %d tokens x top-%d) of the 384-expert decode layer, fp64 "
-                      "scalar-C decode + numpy, %.1f s" % (done, done // k, k, dt)}
+            "sample": "%d routes (= %d tokens x top-%d) of the %s layer, fp64 "
+                      "scalar-C decode + numpy, %.1f s" % (done, done // k, k, name, dt)}
 
 
 def run_reference(args, rank, world):
@@ -441,10 +488,11 @@ def run_reference(args, rank, world):
         threadpool_limits(limits=1)
     except Exception:
         pass
-    w0 = inputs.moe_decode_t16()
+    w0 = inputs.moe_decode_t16() if args.workload == "moe_decode_t16" else inputs.moe_prefill_t8192()
     layer, x, logits, k = w0["layer"], w0["x"], w0["logits"], w0["k"]
-    ids, _ = OL.route_topk(logits, k)
-    routes = [(t, s) for t in range(x.shape[0]) for s in range(k)]
+    n_tok = min(x.shape[0], 64)
+    ids, _ = OL.route_topk(logits[:n_tok], k)
+    routes = [(t, s) for t in range(n_tok) for s in range(k)]
 
     def step(i):
         t, s = routes[i % len(routes)]
@@ -463,9 +511,10 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "moe_decode_t16", "experts": 384, "hidden": 4096,
-                   "intermediate": 1024, "tokens": 16, "top_k": k,
-                   "widths": "368/15/1 experts at K=2/3/4"},
+        "config": {"workload": args.workload, "experts": 384, "hidden": 4096,
+                   "intermediate": 1024, "tokens": x.shape[0], "top_k": k,
+                   "widths": WORKLOADS[args.workload]["widths"],
+                   "routing": WORKLOADS[args.workload]["routing"]},
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": 1, "kind": "oracle",
                          "sample": "one (token, expert) route per step = 1/%d token" % k},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

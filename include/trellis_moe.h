@@ -97,7 +97,8 @@ int tq_device_status(int32_t *flags_out, int clear);
  * stream and tagged with its stage:
  *   0 route_topk, 1 route_permute, 2 hadamard128 of the input, 3 GEMV gate/up+SiLU,
  *   4 rotation of h, 5 GEMV down, 6 route_unpermute, 7 trellis_decode, 8 trellis_gemv,
- *   9 GEMM gate/up+SiLU, 10 GEMM down.
+ *   9 GEMM gate/up+SiLU, 10 GEMM down, 11 GEMM preparation (tile list, route-ordered
+ *   activation rows).
  * tq_profile_enable creates 2*max_launches events (host-side CUDA resources; call it
  * outside graph capture); launches beyond max_launches are not recorded.  A launch made
  * during stream capture records its events as external event-record nodes of the graph,
@@ -255,8 +256,10 @@ int moe_trellis_gemv_noalloc(const tq_moe_layer *layer, const uint16_t *x_rot,
 /*
  * moe_trellis_gemm -- same result as moe_trellis_gemv for prefill-sized batches: the
  * bit streams are decoded to fp16 operands of tcgen05 tensor-core MMAs (accumulating
- * in tensor memory), each weight decoded once per 128 routes of its expert.
- * Same arguments and workspace as moe_trellis_gemv.
+ * in tensor memory), each weight decoded once per block of up to 256 routes of its
+ * expert.  Same arguments as moe_trellis_gemv; the workspace must hold
+ * moe_trellis_workspace_size() bytes; D must be a multiple of 256 (TQ_ERR_UNSUPPORTED
+ * otherwise).
  */
 int moe_trellis_gemm(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
                      const int32_t *perm, const int32_t *active_ids, const int32_t *n_active,

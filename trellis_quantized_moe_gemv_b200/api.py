@@ -136,7 +136,7 @@ def device_status(clear: bool = False) -> int:
 
 
 STAGES = ("route_topk", "route_permute", "rotate_x", "gemv_gateup", "rotate_h", "gemv_down",
-          "route_unpermute", "trellis_decode", "trellis_gemv", "gemm_gateup", "gemm_down")
+          "route_unpermute", "trellis_decode", "trellis_gemv", "gemm_gateup", "gemm_down", "gemm_prep")
 
 
 def launch_count() -> int:

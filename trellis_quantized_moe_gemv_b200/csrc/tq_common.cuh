@@ -34,7 +34,7 @@ inline bool aligned8(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 7
 enum Stage {
     kStageTopk = 0, kStagePermute = 1, kStageRotateX = 2, kStageGemvGateUp = 3,
     kStageRotateH = 4, kStageGemvDown = 5, kStageUnpermute = 6, kStageDecode = 7,
-    kStageGemv = 8, kStageGemmGateUp = 9, kStageGemmDown = 10, kNumStages = 11
+    kStageGemv = 8, kStageGemmGateUp = 9, kStageGemmDown = 10, kStageGemmPrep = 11, kNumStages = 12
 };
 
 // Brackets one kernel launch: counts it and, while profiling is on, records a start
@@ -145,6 +145,38 @@ constexpr uint32_t kWaitPolls = 1u << 22;
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
     for (uint32_t i = 0; i < kWaitPolls; ++i)
         if (mbar_try_wait(bar, parity)) return true;
+    raise_flag(2);
+    return false;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity, letting the hardware suspend the thread
+// between polls (no spinning that would take issue slots from working warps), and give
+// up after kWaitSeconds of wall time (device flag bit 1).
+constexpr uint64_t kWaitNs = 4000000000ull;
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+        if (global_timer_ns() - t0 > kWaitNs) break;
+    }
     raise_flag(2);
     return false;
 }

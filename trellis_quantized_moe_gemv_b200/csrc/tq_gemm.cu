@@ -32,26 +32,35 @@
 
 namespace tq {
 
-constexpr int kGBM = 128;          // weight rows per tile
-constexpr int kGBN = 256;          // max routes per tile
-constexpr int kGBK = 64;           // K columns per stage
-constexpr int kGStages = 4;
-constexpr int kGDecodeWarps = 8;   // two groups of 4
-constexpr int kGThreads = (2 + kGDecodeWarps) * 32;
-constexpr int kGBitsSlot = 512;    // per strip per stage: 4 tiles x up to 128 B
+constexpr int kGBM = 128;          // weight rows per MMA tile (one accumulator)
+constexpr int kGTiles = 2;         // weight tiles per CTA: both share every activation slab
+constexpr int kGBN = 256;          // max routes per CTA
+constexpr int kGBK = 64;           // K columns per K-block
+constexpr int kGGroups = 2;        // decode groups of 4 warps; K-block kb -> group kb % 2
+constexpr int kGBitsStages = 6;    // bit-stream ring (multiple of kGGroups)
+constexpr int kGBStages = 3;       // activation (B) ring
+constexpr int kGDecodeWarps = 4 * kGGroups;
+constexpr int kGFirstDecodeWarp = 3;   // warp 0: bit-stream producer, 1: MMA, 2: B producer
+constexpr int kGThreads = (kGFirstDecodeWarp + kGDecodeWarps) * 32;
+constexpr int kGStrips = 8 * kGTiles;  // 16-row strips per CTA
+constexpr int kGBitsSlot = 512;    // per strip per K-block: 4 tiles x up to 128 B
 constexpr int kGBoxes = 4;         // TMA boxes of 32, 64, 128, 256 rows
+constexpr uint32_t kGTmemCols = 512;   // two 256-column fp32 accumulators
 
 struct __align__(1024) GemmSmem {
-    __half a[kGStages][kGBM * kGBK];      // 16 KB per stage, 1024-byte aligned
-    __half b[kGStages][kGBN * kGBK];      // 32 KB per stage
-    unsigned char bits[kGStages][8 * kGBitsSlot];
-    uint64_t full[kGStages];              // producer -> decoders (bits + B landed)
-    uint64_t decoded[kGStages];           // decoders -> MMA (A written)
-    uint64_t empty[kGStages];             // MMA -> producer (stage consumed)
-    uint64_t acc_full;                    // MMA -> epilogue
-    uint64_t mma_done;                    // MMA drain on early exit
+    __half a[kGGroups][kGTiles][kGBM * kGBK];  // 2 x 16 KB per decode group, 1024-aligned
+    __half b[kGBStages][kGBN * kGBK];          // 32 KB per stage
+    unsigned char bits[kGBitsStages][kGStrips * kGBitsSlot];
+    uint64_t bits_full[kGBitsStages];          // producer -> decoders (count 1 + bytes)
+    uint64_t bits_empty[kGBitsStages];         // decoders -> producer (count 4)
+    uint64_t b_full[kGBStages];                // B producer -> MMA (count 1 + bytes)
+    uint64_t b_empty[kGBStages];               // MMA -> B producer (commit)
+    uint64_t a_full[kGGroups];                 // decoders -> MMA (count 4)
+    uint64_t a_empty[kGGroups];                // MMA -> decoders (commit)
+    uint64_t acc_full;                         // MMA -> epilogue
+    uint64_t mma_done;                         // MMA drain on early exit
     uint32_t tmem_base;
-    int32_t abort;                        // a role gave up
+    int32_t abort;                             // a role gave up
 };
 
 struct GemmMaps {
@@ -146,29 +155,27 @@ __device__ __forceinline__ uint32_t prod_hi(const uint32_t (&v)[NS]) {
 }
 
 // Rows R of the lane's 4 columns -> 4 fp16 subnormals t * 2^-24, stored (8 bytes) into
-// the swizzled A stage at row m = row0 + R, chunk c.
+// the swizzled A stage: row m = row0 + R (row0 a multiple of 16), so the swizzle
+// depends on R only and addr[R & 7] + (R >> 3) * 1024 is the store address.
 template <int K, int R>
-__device__ __forceinline__ void decode_rows(const uint32_t (&v)[2 * K + 1], unsigned char *a_stage, int row0,
-                                            int chunk, int half_off) {
+__device__ __forceinline__ void decode_rows(const uint32_t (&v)[2 * K + 1], const uint32_t (&addr)[8]) {
     if constexpr (R < 16) {
         const uint32_t p0 = prod_hi<0 * 16 * K + K * R>(v), p1 = prod_hi<1 * 16 * K + K * R>(v);
         const uint32_t p2 = prod_hi<2 * 16 * K + K * R>(v), p3 = prod_hi<3 * 16 * K + K * R>(v);
         const uint32_t ab = hadd2_u32(prmt(p0, p1, 0x4602u), prmt(p0, p1, 0x5713u));
         const uint32_t cd = hadd2_u32(prmt(p2, p3, 0x4602u), prmt(p2, p3, 0x5713u));
-        const int m = row0 + R;
-        *reinterpret_cast<uint2 *>(a_stage + m * 128 + ((chunk ^ (m & 7)) << 4) + half_off) = make_uint2(ab, cd);
-        decode_rows<K, R + 1>(v, a_stage, row0, chunk, half_off);
+        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr[R & 7] + (R >> 3) * 1024), "r"(ab), "r"(cd)
+                     : "memory");
+        decode_rows<K, R + 1>(v, addr);
     }
 }
 
-// Decode one stage: thread (wl, lane) of a 4-warp group handles strip slot sig,
-// column tile j of the K-block, columns 4*t4..4*t4+3, all 16 rows.
+// Decode one (strip slot, column tile, lane quarter) cell of a K-block: 16 rows x 4
+// columns into the swizzled A stage of its weight tile.
 template <int K>
-__device__ __forceinline__ void decode_stage(const unsigned char *bits_stage, unsigned char *a_stage, int wl,
-                                             int lane) {
+__device__ __forceinline__ void decode_cell(const unsigned char *bits_stage, uint32_t a_tile_s, int sig_in_tile,
+                                            int sig, int j, int t4) {
     constexpr int TB = 32 * K;
-    const int pair = wl * 8 + (lane >> 2);
-    const int sig = pair >> 2, j = pair & 3, t4 = lane & 3;
     const unsigned char *tile = bits_stage + sig * kGBitsSlot + j * TB;
     uint32_t v[2 * K + 1];
     if constexpr (K == 2) {
@@ -184,8 +191,24 @@ __device__ __forceinline__ void decode_stage(const unsigned char *bits_stage, un
         v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     }
     v[2 * K] = *reinterpret_cast<const uint32_t *>(tile + 8 * K * ((t4 + 1) & 3));
-    const int kc = 16 * j + 4 * t4;   // first K column of the lane within the stage
-    decode_rows<K, 0>(v, a_stage, 16 * sig, kc >> 3, (kc & 7) * 2);
+    const int kc = 16 * j + 4 * t4;   // first K column of the lane within the K-block
+    const int chunk = kc >> 3, half_off = (kc & 7) * 2;
+    uint32_t addr[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) addr[r] = a_tile_s + (16 * sig_in_tile + r) * 128 + ((chunk ^ r) << 4) + half_off;
+    decode_rows<K, 0>(v, addr);
+}
+
+// Decode one K-block (16 strips x 4 column tiles) with a 4-warp group: thread (wl, lane)
+// takes strip slots 2*wl + {0, 1} ... as two cells (one per weight tile).
+template <int K>
+__device__ __forceinline__ void decode_stage(const unsigned char *bits_stage, uint32_t a_group_s, int wl,
+                                             int lane) {
+    const int cell = wl * 8 + (lane >> 2);   // 0..31 within a weight tile: (strip, column tile)
+    const int sig = cell >> 2, j = cell & 3, t4 = lane & 3;
+#pragma unroll 1
+    for (int t = 0; t < kGTiles; ++t)
+        decode_cell<K>(bits_stage, a_group_s + t * (kGBM * kGBK * 2), sig, 8 * t + sig, j, t4);
 }
 
 // ------------------------------------------------------------------------------ kernel
@@ -203,8 +226,11 @@ template <bool GATEUP>
 __global__ void __launch_bounds__(kGThreads, 1)
     moe_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs args) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    // the stage buffers need 1024-byte alignment (128-byte swizzle atoms)
-    GemmSmem &sm = *reinterpret_cast<GemmSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // The stage buffers need 1024-byte alignment (128-byte swizzle atoms).  Offset the
+    // __shared__ array itself (no round trip through an integer) so that the compiler
+    // keeps shared-memory instructions for every access derived from it.
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    GemmSmem &sm = *reinterpret_cast<GemmSmem *>(smem_raw + pad);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const tq_moe_layer &L = args.L;
 
@@ -226,128 +252,141 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int tiles_per_strip = args.kdim / 16;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kGStages; ++s) {
-            mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.decoded[s], 4);
-            mbar_init(&sm.empty[s], 1);
+        for (int i = 0; i < kGBitsStages; ++i) {
+            mbar_init(&sm.bits_full[i], 1);
+            mbar_init(&sm.bits_empty[i], 4);
+        }
+        for (int i = 0; i < kGBStages; ++i) {
+            mbar_init(&sm.b_full[i], 1);
+            mbar_init(&sm.b_empty[i], 1);
+        }
+        for (int i = 0; i < kGGroups; ++i) {
+            mbar_init(&sm.a_full[i], 4);
+            mbar_init(&sm.a_empty[i], 1);
         }
         mbar_init(&sm.acc_full, 1);
         mbar_init(&sm.mma_done, 1);
         sm.abort = 0;
         fence_barrier_init();
     }
-    if (warp == 1) tmem_alloc(&sm.tmem_base, 256);
+    if (warp == 1) tmem_alloc(&sm.tmem_base, kGTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_d = sm.tmem_base;
+    // a wait that gave up anywhere stops every role: check the shared flag too
+    auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity));
+        if (!ok) sm.abort = 1;
+        return ok && !*(volatile int32_t *)&sm.abort;
+    };
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ bit-stream producer
         const int K = ex.K;
         const int strip_bytes = 4 * 32 * K;
         const uint32_t *strip_base = nullptr;
-        if (lane < 8) {
-            if (GATEUP) strip_base = ((lane & 1) ? ex.up : ex.gate) + (size_t)(mt * 4 + (lane >> 1)) * tiles_per_strip * (8 * K);
-            else strip_base = ex.down + (size_t)(mt * 8 + lane) * tiles_per_strip * (8 * K);
+        if (lane < kGStrips) {
+            // strip slot lane: weight tile lane / 8, slot within the tile lane % 8
+            const int t = lane >> 3, sl = lane & 7;
+            if (GATEUP)
+                strip_base = ((sl & 1) ? ex.up : ex.gate) +
+                             (size_t)((mt * kGTiles + t) * 4 + (sl >> 1)) * tiles_per_strip * (8 * K);
+            else
+                strip_base = ex.down + (size_t)((mt * kGTiles + t) * 8 + sl) * tiles_per_strip * (8 * K);
         }
-        uint32_t parity = 0;
-        bool ok = true;
         int issued = 0;
-        for (int kb = 0; kb < num_kb && ok; ++kb) {
-            const int s = kb % kGStages;
-            if (kb >= kGStages) {
-                ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.empty[s], (parity >> s) & 1u));
-                parity ^= 1u << s;
-                if (!ok || *(volatile int32_t *)&sm.abort) {
-                    ok = false;
-                    break;
-                }
-            }
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.full[s], 8u * strip_bytes + (32u << box) * 128u);
-                tma_load_2d(sm.b[s], &maps.b[box], kb * kGBK, r0 + n0, &sm.full[s]);
-            }
+        for (int kb = 0; kb < num_kb; ++kb) {
+            const int i = kb % kGBitsStages;
+            if (kb >= kGBitsStages && !wait(&sm.bits_empty[i], ((kb / kGBitsStages) - 1) & 1)) break;
+            if (lane == 0) mbar_arrive_expect_tx(&sm.bits_full[i], (uint32_t)kGStrips * strip_bytes);
             __syncwarp();
-            if (lane < 8)
-                bulk_g2s(sm.bits[s] + lane * kGBitsSlot, strip_base + (size_t)kb * 4 * (8 * K), strip_bytes,
-                         &sm.full[s]);
+            if (lane < kGStrips)
+                bulk_g2s(sm.bits[i] + lane * kGBitsSlot, strip_base + (size_t)kb * 4 * (8 * K), strip_bytes,
+                         &sm.bits_full[i]);
             ++issued;
         }
-        if (!ok) {
-            sm.abort = 1;
-            // drain: wait (bounded) for every stage this warp filled last
-            for (int kb = max(0, issued - kGStages); kb < issued; ++kb) {
-                const int s = kb % kGStages;
-                const uint32_t ph = ((kb / kGStages) & 1u);
-                mbar_wait_bounded(&sm.full[s], ph);
+        // drain: every issued copy has landed before the CTA can exit
+        for (int kb = max(0, issued - kGBitsStages); kb < issued; ++kb)
+            mbar_wait_sleep(&sm.bits_full[kb % kGBitsStages], (kb / kGBitsStages) & 1);
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ activation producer
+        int issued = 0;
+        for (int kb = 0; kb < num_kb; ++kb) {
+            const int i = kb % kGBStages;
+            if (kb >= kGBStages && !wait(&sm.b_empty[i], ((kb / kGBStages) - 1) & 1)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.b_full[i], (32u << box) * 128u);
+                tma_load_2d(sm.b[i], &maps.b[box], kb * kGBK, r0 + n0, &sm.b_full[i]);
             }
+            __syncwarp();
+            ++issued;
         }
+        for (int kb = max(0, issued - kGBStages); kb < issued; ++kb)
+            mbar_wait_sleep(&sm.b_full[kb % kGBStages], (kb / kGBStages) & 1);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         const uint32_t idesc = umma_idesc_f16(nmma);
-        uint32_t parity = 0;
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
-            const int s = kb % kGStages;
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.decoded[s], (parity >> s) & 1u));
-            parity ^= 1u << s;
-            if (!ok || *(volatile int32_t *)&sm.abort) {
+            const int g = kb % kGGroups, i = kb % kGBStages;
+            if (!wait(&sm.a_full[g], (kb / kGGroups) & 1) || !wait(&sm.b_full[i], (kb / kGBStages) & 1)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+                const uint32_t b0 = smem_u32(sm.b[i]);
 #pragma unroll
-                for (int k = 0; k < kGBK / 16; ++k)
-                    umma_f16(tmem_d, umma_desc_sw128(a0 + 32 * k), umma_desc_sw128(b0 + 32 * k), idesc,
-                             (kb | k) != 0);
-                umma_commit(&sm.empty[s]);
+                for (int t = 0; t < kGTiles; ++t) {
+                    const uint32_t a0 = smem_u32(sm.a[g][t]);
+#pragma unroll
+                    for (int k = 0; k < kGBK / 16; ++k)
+                        umma_f16(tmem_d + t * kGBN, umma_desc_sw128(a0 + 32 * k), umma_desc_sw128(b0 + 32 * k),
+                                 idesc, (kb | k) != 0);
+                }
+                umma_commit(&sm.a_empty[g]);
+                umma_commit(&sm.b_empty[i]);
             }
             __syncwarp();
         }
         if (lane == 0) umma_commit(ok ? &sm.acc_full : &sm.mma_done);
         __syncwarp();
-        if (!ok) {
-            sm.abort = 1;
-            mbar_wait_bounded(&sm.mma_done, 0);
-        }
+        if (!ok) mbar_wait_sleep(&sm.mma_done, 0);
     } else {
         // ------------------------------------------------------------ decoders
-        const int dw = warp - 2;
+        const int dw = warp - kGFirstDecodeWarp;
         const int group = dw >> 2, wl = dw & 3;
-        uint32_t parity = 0;
-        bool ok = true;
-        for (int kb = group; kb < num_kb; kb += 2) {
-            const int s = kb % kGStages;
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[s], (parity >> s) & 1u));
-            parity ^= 1u << s;
-            if (!ok || *(volatile int32_t *)&sm.abort) {
-                ok = false;
-                break;
-            }
-            unsigned char *a_stage = reinterpret_cast<unsigned char *>(sm.a[s]);
-            if (ex.K == 2) decode_stage<2>(sm.bits[s], a_stage, wl, lane);
-            else if (ex.K == 3) decode_stage<3>(sm.bits[s], a_stage, wl, lane);
-            else decode_stage<4>(sm.bits[s], a_stage, wl, lane);
+        const uint32_t a_s = smem_u32(sm.a[group][0]);
+        for (int kb = group; kb < num_kb; kb += kGGroups) {
+            const int i = kb % kGBitsStages;
+            if (!wait(&sm.bits_full[i], (kb / kGBitsStages) & 1)) break;
+            if (kb >= kGGroups && !wait(&sm.a_empty[group], ((kb / kGGroups) - 1) & 1)) break;
+            if (ex.K == 2) decode_stage<2>(sm.bits[i], a_s, wl, lane);
+            else if (ex.K == 3) decode_stage<3>(sm.bits[i], a_s, wl, lane);
+            else decode_stage<4>(sm.bits[i], a_s, wl, lane);
             fence_proxy_async();      // make the generic-proxy writes visible to the MMA
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.decoded[s]);
+            if (lane == 0) {
+                mbar_arrive(&sm.a_full[group]);
+                mbar_arrive(&sm.bits_empty[i]);
+            }
         }
-        if (!ok) sm.abort = 1;
         // ------------------------------------------------------------ epilogue
-        if (group == 1) {
-            const int q = warp & 3;             // tensor-memory lane quarter of this warp
-            const bool acc_ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.acc_full, 0));
-            if (acc_ok && !*(volatile int32_t *)&sm.abort) {
+        // group t reads weight tile t's accumulator (columns t*256...), one warp per
+        // tensor-memory lane quarter
+        {
+            const int tt = group;
+            const int q = warp & 3;
+            if (wait(&sm.acc_full, 0)) {
                 tc_fence_after();
-                const int row = 32 * q + lane;  // weight row of the tile = tensor-memory lane
+                const int row = 32 * q + lane;  // weight row of tile tt = tensor-memory lane
+                const int mtile = mt * kGTiles + tt;
                 for (int c0 = 0; c0 < nmma; c0 += 16) {
                     uint32_t v[16];
-                    tmem_ld16(tmem_d + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+                    tmem_ld16(tmem_d + ((uint32_t)(32 * q) << 16) + (uint32_t)(tt * kGBN + c0), v);
                     if (GATEUP) {
-                        const int f = (mt * 4 + q) * 16 + (lane & 15);
+                        const int f = (mtile * 4 + q) * 16 + (lane & 15);
                         const float sg = __half2float(ex.s_gate[f]), su = __half2float(ex.s_up[f]);
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
@@ -363,7 +402,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                             }
                         }
                     } else {
-                        const int d = mt * kGBM + row;
+                        const int d = mtile * kGBM + row;
                         const float sd = __half2float(ex.s_down[d]);
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
@@ -384,7 +423,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_d, 256);
+        tmem_dealloc(tmem_d, kGTmemCols);
     }
 }
 
@@ -556,14 +595,14 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
 
     const size_t smem = sizeof(GemmSmem) + 1024;
     {
-        LaunchScope ls(s, kStageGemmGateUp);
+        LaunchScope ls(s, kStageGemmPrep);
         gemm_tile_list_kernel<<<1, 1024, 0, s>>>(offsets, active_ids, n_active, max_tiles, tiles);
     }
     st = launch_status();
     if (st) return st;
     {
         // x_rot is already rotated: copy its rows to their route rows (+ row sums)
-        LaunchScope ls(s, kStageGemmGateUp);
+        LaunchScope ls(s, kStageGemmPrep);
         route_rows_kernel<__half, false><<<(R * 32 + 255) / 256, 256, 0, s>>>(x_rot, R, L->D, perm, k, T, xp, sxp);
     }
     st = launch_status();
@@ -571,7 +610,7 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     {
         GemmArgs a{*L, offsets, tiles, sxp, h, L->D};
         LaunchScope ls(s, kStageGemmGateUp);
-        moe_gemm_kernel<true><<<dim3(L->F / 64, max_tiles), kGThreads, smem, s>>>(maps_x, a);
+        moe_gemm_kernel<true><<<dim3(L->F / (64 * kGTiles), max_tiles), kGThreads, smem, s>>>(maps_x, a);
     }
     st = launch_status();
     if (st) return st;
@@ -584,7 +623,7 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     {
         GemmArgs a{*L, offsets, tiles, shr, y_perm, L->F};
         LaunchScope ls(s, kStageGemmDown);
-        moe_gemm_kernel<false><<<dim3(L->D / kGBM, max_tiles), kGThreads, smem, s>>>(maps_h, a);
+        moe_gemm_kernel<false><<<dim3(L->D / (kGBM * kGTiles), max_tiles), kGThreads, smem, s>>>(maps_h, a);
     }
     return launch_status();
 }
@@ -601,6 +640,7 @@ TQ_API int moe_trellis_gemm(const tq_moe_layer *layer, const uint16_t *x_rot, co
     int st = moe_validate_call(layer, x_rot, offsets, perm, active_ids, n_active, T, k, y_perm, ws, ws_bytes);
     if (st || T == 0) return st;
     if (ws_bytes < tq::gemm_workspace_bytes(layer, T, k)) return TQ_ERR_WORKSPACE;
+    if (layer->D % (tq::kGBM * tq::kGTiles)) return TQ_ERR_UNSUPPORTED;   // down: 256-row CTAs
     if ((long long)T * k / tq::kGBN + layer->E + 1 > 65535) return TQ_ERR_UNSUPPORTED;
     return tq::run_moe_gemm(layer, reinterpret_cast<const __half *>(x_rot), offsets, perm, active_ids, n_active,
                             T, k, y_perm, ws, (cudaStream_t)stream);
