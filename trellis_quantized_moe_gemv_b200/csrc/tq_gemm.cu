@@ -29,6 +29,7 @@
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <string.h>
 
 namespace tq {
 
@@ -65,6 +66,11 @@ struct __align__(1024) GemmSmem {
 
 struct GemmMaps {
     CUtensorMap b[kGBoxes];               // route-ordered activations, box rows 32..256
+    // bit streams of each width group as [expert][strip][words] (uint32), box
+    // {4 tiles, 8 or 16 strips, 1}: gate/up launch: first = gate, second = up (8
+    // strips each); down launch: first = down (16 strips).
+    CUtensorMap bits_first[3];
+    CUtensorMap bits_second[3];
 };
 
 // ------------------------------------------------------------------------------ PTX
@@ -78,6 +84,14 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
         "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -174,9 +188,9 @@ __device__ __forceinline__ void decode_rows(const uint32_t (&v)[2 * K + 1], cons
 // columns into the swizzled A stage of its weight tile.
 template <int K>
 __device__ __forceinline__ void decode_cell(const unsigned char *bits_stage, uint32_t a_tile_s, int sig_in_tile,
-                                            int sig, int j, int t4) {
+                                            int row, int j, int t4) {
     constexpr int TB = 32 * K;
-    const unsigned char *tile = bits_stage + sig * kGBitsSlot + j * TB;
+    const unsigned char *tile = bits_stage + row * (4 * TB) + j * TB;   // rows packed by the tensor copy
     uint32_t v[2 * K + 1];
     if constexpr (K == 2) {
         uint4 a = *reinterpret_cast<const uint4 *>(tile + 16 * t4);
@@ -200,15 +214,19 @@ __device__ __forceinline__ void decode_cell(const unsigned char *bits_stage, uin
 }
 
 // Decode one K-block (16 strips x 4 column tiles) with a 4-warp group: thread (wl, lane)
-// takes strip slots 2*wl + {0, 1} ... as two cells (one per weight tile).
-template <int K>
+// takes one (strip slot, column tile, quarter) cell in each of the two weight tiles.
+// Rows of the bit-stream stage: gate/up: [8 gate strips][8 up strips] of the tile pair
+// (tile t, slot sl -> row (sl & 1) * 8 + 4t + (sl >> 1)); down: 16 consecutive strips.
+template <int K, bool GATEUP>
 __device__ __forceinline__ void decode_stage(const unsigned char *bits_stage, uint32_t a_group_s, int wl,
                                              int lane) {
     const int cell = wl * 8 + (lane >> 2);   // 0..31 within a weight tile: (strip, column tile)
     const int sig = cell >> 2, j = cell & 3, t4 = lane & 3;
 #pragma unroll 1
-    for (int t = 0; t < kGTiles; ++t)
-        decode_cell<K>(bits_stage, a_group_s + t * (kGBM * kGBK * 2), sig, 8 * t + sig, j, t4);
+    for (int t = 0; t < kGTiles; ++t) {
+        const int row = GATEUP ? (sig & 1) * 8 + 4 * t + (sig >> 1) : 8 * t + sig;
+        decode_cell<K>(bits_stage, a_group_s + t * (kGBM * kGBK * 2), sig, row, j, t4);
+    }
 }
 
 // ------------------------------------------------------------------------------ kernel
@@ -284,26 +302,24 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ bit-stream producer
         const int K = ex.K;
-        const int strip_bytes = 4 * 32 * K;
-        const uint32_t *strip_base = nullptr;
-        if (lane < kGStrips) {
-            // strip slot lane: weight tile lane / 8, slot within the tile lane % 8
-            const int t = lane >> 3, sl = lane & 7;
-            if (GATEUP)
-                strip_base = ((sl & 1) ? ex.up : ex.gate) +
-                             (size_t)((mt * kGTiles + t) * 4 + (sl >> 1)) * tiles_per_strip * (8 * K);
-            else
-                strip_base = ex.down + (size_t)((mt * kGTiles + t) * 8 + sl) * tiles_per_strip * (8 * K);
-        }
+        const int row_bytes = 4 * 32 * K;                     // 4 column tiles of one strip
+        const CUtensorMap *m1 = &maps.bits_first[ex.group], *m2 = &maps.bits_second[ex.group];
+        const int strip0 = GATEUP ? mt * 8 : mt * 16;         // first strip of the CTA
         int issued = 0;
         for (int kb = 0; kb < num_kb; ++kb) {
             const int i = kb % kGBitsStages;
             if (kb >= kGBitsStages && !wait(&sm.bits_empty[i], ((kb / kGBitsStages) - 1) & 1)) break;
-            if (lane == 0) mbar_arrive_expect_tx(&sm.bits_full[i], (uint32_t)kGStrips * strip_bytes);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.bits_full[i], (uint32_t)kGStrips * row_bytes);
+                const int x = kb * 4 * 8 * K;                 // word offset of the K-block
+                if (GATEUP) {
+                    tma_load_3d(sm.bits[i], m1, x, strip0, ex.index, &sm.bits_full[i]);
+                    tma_load_3d(sm.bits[i] + 8 * row_bytes, m2, x, strip0, ex.index, &sm.bits_full[i]);
+                } else {
+                    tma_load_3d(sm.bits[i], m1, x, strip0, ex.index, &sm.bits_full[i]);
+                }
+            }
             __syncwarp();
-            if (lane < kGStrips)
-                bulk_g2s(sm.bits[i] + lane * kGBitsSlot, strip_base + (size_t)kb * 4 * (8 * K), strip_bytes,
-                         &sm.bits_full[i]);
             ++issued;
         }
         // drain: every issued copy has landed before the CTA can exit
@@ -362,9 +378,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int i = kb % kGBitsStages;
             if (!wait(&sm.bits_full[i], (kb / kGBitsStages) & 1)) break;
             if (kb >= kGGroups && !wait(&sm.a_empty[group], ((kb / kGGroups) - 1) & 1)) break;
-            if (ex.K == 2) decode_stage<2>(sm.bits[i], a_s, wl, lane);
-            else if (ex.K == 3) decode_stage<3>(sm.bits[i], a_s, wl, lane);
-            else decode_stage<4>(sm.bits[i], a_s, wl, lane);
+            if (ex.K == 2) decode_stage<2, GATEUP>(sm.bits[i], a_s, wl, lane);
+            else if (ex.K == 3) decode_stage<3, GATEUP>(sm.bits[i], a_s, wl, lane);
+            else decode_stage<4, GATEUP>(sm.bits[i], a_s, wl, lane);
             fence_proxy_async();      // make the generic-proxy writes visible to the MMA
             __syncwarp();
             if (lane == 0) {
@@ -545,6 +561,34 @@ static int make_maps(const __half *base, int rows, int cols, GemmMaps &maps) {
     return TQ_OK;
 }
 
+// Bit streams of every width group for one projection as a 3D uint32 tensor
+// [n_experts][n_strips][words_per_strip], box {4 tiles, box_strips, 1}.
+static int make_bits_maps(const tq_moe_layer *L, bool gateup, GemmMaps &maps) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return record_error("cuTensorMapEncodeTiled entry point not found");
+    for (int g = 0; g < 3; ++g) {
+        for (int which = 0; which < 2; ++which) {
+            CUtensorMap *dst = which ? &maps.bits_second[g] : &maps.bits_first[g];
+            memset(dst, 0, sizeof(CUtensorMap));
+            if (g >= L->n_groups || L->groups[g].n_experts == 0 || (!gateup && which)) continue;
+            const tq_width_group &G = L->groups[g];
+            const uint32_t *base = gateup ? (which ? G.up : G.gate) : G.down;
+            const int n_strips = gateup ? L->F / 16 : L->D / 16;
+            const int tiles = gateup ? L->D / 16 : L->F / 16;
+            const cuuint64_t words = (cuuint64_t)tiles * 8 * G.K;
+            cuuint64_t dims[3] = {words, (cuuint64_t)n_strips, (cuuint64_t)G.n_experts};
+            cuuint64_t strides[2] = {words * 4, words * 4 * (cuuint64_t)n_strips};
+            cuuint32_t box[3] = {(cuuint32_t)(4 * 8 * G.K), (cuuint32_t)(gateup ? 8 : 16), 1};
+            cuuint32_t estr[3] = {1, 1, 1};
+            CUresult r = enc(dst, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, (void *)base, dims, strides, box, estr,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS) return record_error("cuTensorMapEncodeTiled (bit streams) failed");
+        }
+    }
+    return TQ_OK;
+}
+
 static size_t align256_g(size_t b) { return (b + 255) & ~(size_t)255; }
 
 static int gemm_max_tiles(int T, int k, int E) {
@@ -591,6 +635,10 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     int st = make_maps(xp, R, L->D, maps_x);
     if (st) return st;
     st = make_maps(hr, R, L->F, maps_h);
+    if (st) return st;
+    st = make_bits_maps(L, true, maps_x);
+    if (st) return st;
+    st = make_bits_maps(L, false, maps_h);
     if (st) return st;
 
     const size_t smem = sizeof(GemmSmem) + 1024;

@@ -255,6 +255,7 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
 
 struct ExpertRef {
     int K;
+    int group, index;             // width group and position inside it
     const uint32_t *gate, *up, *down;
     const __half *s_gate, *s_up, *s_down;
 };
@@ -269,6 +270,8 @@ __device__ __forceinline__ bool expert_ref(const tq_moe_layer &L, int e, ExpertR
     if (idx >= G.n_experts) return false;
     const size_t words_proj = (size_t)(L.D / 16) * (L.F / 16) * 8 * G.K;
     r.K = G.K;
+    r.group = gi;
+    r.index = idx;
     r.gate = G.gate + (size_t)idx * words_proj;
     r.up = G.up + (size_t)idx * words_proj;
     r.down = G.down + (size_t)idx * words_proj;
