@@ -168,14 +168,15 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t pa
 
 // Wait for the phase with the given parity, letting the hardware suspend the thread
 // between polls (no spinning that would take issue slots from working warps), and give
-// up after kWaitSeconds of wall time (device flag bit 1).
+// up after kWaitNs of wall time (device flag bit 1).  The timer is read only every 64
+// polls.
 constexpr uint64_t kWaitNs = 4000000000ull;
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity) {
-    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    while (true) {
-        if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
-        if (global_timer_ns() - t0 > kWaitNs) break;
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait_suspend(bar, parity, 1000000u)) return true;
+        if ((n & 63u) == 0 && global_timer_ns() - t0 > kWaitNs) break;
     }
     raise_flag(2);
     return false;

@@ -37,10 +37,11 @@ constexpr int kGBM = 128;          // weight rows per MMA tile (one accumulator)
 constexpr int kGTiles = 2;         // weight tiles per CTA: both share every activation slab
 constexpr int kGBN = 256;          // max routes per CTA
 constexpr int kGBK = 64;           // K columns per K-block
-constexpr int kGGroups = 2;        // decode groups of 4 warps; K-block kb -> group kb % 2
+constexpr int kGGroups = 2;        // K-block slots: K-block kb is decoded into A slot kb % 2
+constexpr int kGDecodeGroups = 2 * kGGroups;   // 4-warp groups: (K-block parity, weight tile)
 constexpr int kGBitsStages = 6;    // bit-stream ring (multiple of kGGroups)
 constexpr int kGBStages = 3;       // activation (B) ring
-constexpr int kGDecodeWarps = 4 * kGGroups;
+constexpr int kGDecodeWarps = 4 * kGDecodeGroups;
 constexpr int kGFirstDecodeWarp = 3;   // warp 0: bit-stream producer, 1: MMA, 2: B producer
 constexpr int kGThreads = (kGFirstDecodeWarp + kGDecodeWarps) * 32;
 constexpr int kGStrips = 8 * kGTiles;  // 16-row strips per CTA
@@ -53,10 +54,10 @@ struct __align__(1024) GemmSmem {
     __half b[kGBStages][kGBN * kGBK];          // 32 KB per stage
     unsigned char bits[kGBitsStages][kGStrips * kGBitsSlot];
     uint64_t bits_full[kGBitsStages];          // producer -> decoders (count 1 + bytes)
-    uint64_t bits_empty[kGBitsStages];         // decoders -> producer (count 4)
+    uint64_t bits_empty[kGBitsStages];         // decoders -> producer (count 8)
     uint64_t b_full[kGBStages];                // B producer -> MMA (count 1 + bytes)
     uint64_t b_empty[kGBStages];               // MMA -> B producer (commit)
-    uint64_t a_full[kGGroups];                 // decoders -> MMA (count 4)
+    uint64_t a_full[kGGroups];                 // decoders -> MMA (count 8)
     uint64_t a_empty[kGGroups];                // MMA -> decoders (commit)
     uint64_t acc_full;                         // MMA -> epilogue
     uint64_t mma_done;                         // MMA drain on early exit
@@ -186,25 +187,41 @@ __device__ __forceinline__ void decode_rows(const uint32_t (&v)[2 * K + 1], cons
 
 // Decode one (strip slot, column tile, lane quarter) cell of a K-block: 16 rows x 4
 // columns into the swizzled A stage of its weight tile.
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
 template <int K>
-__device__ __forceinline__ void decode_cell(const unsigned char *bits_stage, uint32_t a_tile_s, int sig_in_tile,
-                                            int row, int j, int t4) {
+__device__ __forceinline__ void decode_cell(uint32_t bits_stage_s, uint32_t a_tile_s, int sig_in_tile, int row,
+                                            int j, int t4) {
     constexpr int TB = 32 * K;
-    const unsigned char *tile = bits_stage + row * (4 * TB) + j * TB;   // rows packed by the tensor copy
+    const uint32_t tile = bits_stage_s + row * (4 * TB) + j * TB;   // rows packed by the tensor copy
     uint32_t v[2 * K + 1];
     if constexpr (K == 2) {
-        uint4 a = *reinterpret_cast<const uint4 *>(tile + 16 * t4);
+        uint4 a = lds128(tile + 16 * t4);
         v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     } else if constexpr (K == 3) {
-        const uint2 *q = reinterpret_cast<const uint2 *>(tile + 24 * t4);
-        uint2 a = q[0], b = q[1], c = q[2];
+        const uint32_t q = tile + 24 * t4;
+        uint2 a = lds64(q), b = lds64(q + 8), c = lds64(q + 16);
         v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y; v[4] = c.x; v[5] = c.y;
     } else {
-        const uint4 *q = reinterpret_cast<const uint4 *>(tile + 32 * t4);
-        uint4 a = q[0], b = q[1];
+        const uint32_t q = tile + 32 * t4;
+        uint4 a = lds128(q), b = lds128(q + 16);
         v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     }
-    v[2 * K] = *reinterpret_cast<const uint32_t *>(tile + 8 * K * ((t4 + 1) & 3));
+    v[2 * K] = lds32(tile + 8 * K * ((t4 + 1) & 3));
     const int kc = 16 * j + 4 * t4;   // first K column of the lane within the K-block
     const int chunk = kc >> 3, half_off = (kc & 7) * 2;
     uint32_t addr[8];
@@ -213,20 +230,16 @@ __device__ __forceinline__ void decode_cell(const unsigned char *bits_stage, uin
     decode_rows<K, 0>(v, addr);
 }
 
-// Decode one K-block (16 strips x 4 column tiles) with a 4-warp group: thread (wl, lane)
-// takes one (strip slot, column tile, quarter) cell in each of the two weight tiles.
-// Rows of the bit-stream stage: gate/up: [8 gate strips][8 up strips] of the tile pair
-// (tile t, slot sl -> row (sl & 1) * 8 + 4t + (sl >> 1)); down: 16 consecutive strips.
+// Decode weight tile t of one K-block (8 strips x 4 column tiles) with a 4-warp group:
+// thread (wl, lane) takes one (strip slot, column tile, quarter) cell.  Rows of the
+// bit-stream stage: gate/up: [8 gate strips][8 up strips] of the tile pair (tile t,
+// slot sl -> row (sl & 1) * 8 + 4t + (sl >> 1)); down: 16 consecutive strips.
 template <int K, bool GATEUP>
-__device__ __forceinline__ void decode_stage(const unsigned char *bits_stage, uint32_t a_group_s, int wl,
-                                             int lane) {
-    const int cell = wl * 8 + (lane >> 2);   // 0..31 within a weight tile: (strip, column tile)
+__device__ __forceinline__ void decode_tile(uint32_t bits_stage_s, uint32_t a_tile_s, int t, int wl, int lane) {
+    const int cell = wl * 8 + (lane >> 2);   // 0..31: (strip slot, column tile)
     const int sig = cell >> 2, j = cell & 3, t4 = lane & 3;
-#pragma unroll 1
-    for (int t = 0; t < kGTiles; ++t) {
-        const int row = GATEUP ? (sig & 1) * 8 + 4 * t + (sig >> 1) : 8 * t + sig;
-        decode_cell<K>(bits_stage, a_group_s + t * (kGBM * kGBK * 2), sig, row, j, t4);
-    }
+    const int row = GATEUP ? (sig & 1) * 8 + 4 * t + (sig >> 1) : 8 * t + sig;
+    decode_cell<K>(bits_stage_s, a_tile_s, sig, row, j, t4);
 }
 
 // ------------------------------------------------------------------------------ kernel
@@ -272,14 +285,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kGBitsStages; ++i) {
             mbar_init(&sm.bits_full[i], 1);
-            mbar_init(&sm.bits_empty[i], 4);
+            mbar_init(&sm.bits_empty[i], 8);
         }
         for (int i = 0; i < kGBStages; ++i) {
             mbar_init(&sm.b_full[i], 1);
             mbar_init(&sm.b_empty[i], 1);
         }
         for (int i = 0; i < kGGroups; ++i) {
-            mbar_init(&sm.a_full[i], 4);
+            mbar_init(&sm.a_full[i], 8);
             mbar_init(&sm.a_empty[i], 1);
         }
         mbar_init(&sm.acc_full, 1);
@@ -371,34 +384,39 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (!ok) mbar_wait_sleep(&sm.mma_done, 0);
     } else {
         // ------------------------------------------------------------ decoders
+        // group dg: K-blocks of parity dg >> 1 (A slot), weight tile dg & 1
         const int dw = warp - kGFirstDecodeWarp;
-        const int group = dw >> 2, wl = dw & 3;
-        const uint32_t a_s = smem_u32(sm.a[group][0]);
-        for (int kb = group; kb < num_kb; kb += kGGroups) {
+        const int dg = dw >> 2, wl = dw & 3;
+        const int slot = dg >> 1, tile = dg & 1;
+        const uint32_t a_s = smem_u32(sm.a[slot][tile]);
+        for (int kb = slot; kb < num_kb; kb += kGGroups) {
             const int i = kb % kGBitsStages;
             if (!wait(&sm.bits_full[i], (kb / kGBitsStages) & 1)) break;
-            if (kb >= kGGroups && !wait(&sm.a_empty[group], ((kb / kGGroups) - 1) & 1)) break;
-            if (ex.K == 2) decode_stage<2, GATEUP>(sm.bits[i], a_s, wl, lane);
-            else if (ex.K == 3) decode_stage<3, GATEUP>(sm.bits[i], a_s, wl, lane);
-            else decode_stage<4, GATEUP>(sm.bits[i], a_s, wl, lane);
+            if (kb >= kGGroups && !wait(&sm.a_empty[slot], ((kb / kGGroups) - 1) & 1)) break;
+            const uint32_t bits_s = smem_u32(sm.bits[i]);
+            if (ex.K == 2) decode_tile<2, GATEUP>(bits_s, a_s, tile, wl, lane);
+            else if (ex.K == 3) decode_tile<3, GATEUP>(bits_s, a_s, tile, wl, lane);
+            else decode_tile<4, GATEUP>(bits_s, a_s, tile, wl, lane);
             fence_proxy_async();      // make the generic-proxy writes visible to the MMA
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&sm.a_full[group]);
+                mbar_arrive(&sm.a_full[slot]);
                 mbar_arrive(&sm.bits_empty[i]);
             }
         }
         // ------------------------------------------------------------ epilogue
-        // group t reads weight tile t's accumulator (columns t*256...), one warp per
-        // tensor-memory lane quarter
+        // group dg reads half (dg >> 1) of the columns of weight tile dg & 1, one warp
+        // per tensor-memory lane quarter
         {
-            const int tt = group;
+            const int tt = tile;
             const int q = warp & 3;
             if (wait(&sm.acc_full, 0)) {
                 tc_fence_after();
                 const int row = 32 * q + lane;  // weight row of tile tt = tensor-memory lane
                 const int mtile = mt * kGTiles + tt;
-                for (int c0 = 0; c0 < nmma; c0 += 16) {
+                const int half_cols = ((nmma / 16 + 1) / 2) * 16;
+                const int cb = slot * half_cols, ce = min(nmma, cb + half_cols);
+                for (int c0 = cb; c0 < ce; c0 += 16) {
                     uint32_t v[16];
                     tmem_ld16(tmem_d + ((uint32_t)(32 * q) << 16) + (uint32_t)(tt * kGBN + c0), v);
                     if (GATEUP) {
