@@ -53,6 +53,20 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", 0)))
 
 
+def aggregate_ranks(ms_local, tokens_per_rank, world, device=None):
+    """Whole-job throughput of independent replicas: every rank's timed milliseconds are
+    reduced with MAX over ranks (the job ends when its slowest replica ends) and the
+    tokens of all ranks are divided by that time.  Returns (ms_max, tokens_per_s)."""
+    ms_max = float(ms_local)
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    return ms_max, tokens_per_rank * world / (ms_max * 1e-3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -326,11 +340,7 @@ def run_ours(args, rank, world, local_rank):
     if flags:
         raise RuntimeError("device anomaly flags %d during the timed region" % flags)
 
-    ms_max = ms_total
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max, value = aggregate_ranks(ms_total, T * args.steps, world, device)
 
     # ---- the dominant kernel (gate/up) per launch: algorithmic bytes (decode GEMV,
     # HBM-bound) or FLOPs (prefill GEMM, tensor-bound) over its average duration; the
@@ -394,11 +404,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms, e2e_value = aggregate_ranks(e0.elapsed_time(e1), T * args.steps, world, device)
     h2d = T * D * 2 + T * E * 4
     d2h = T * D * 4
 
@@ -406,10 +412,9 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w0, routes=16, name=args.workload)
 
-    tokens = T * args.steps * world
     line = {
         "metric": METRIC,
-        "value": tokens / (ms_max * 1e-3),
+        "value": value,
         "unit": "tok/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -433,7 +438,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline,
         "stage_avg_launch_ms": stage_avg,
         "gpu_launches": launches,
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "clocks": sampler.summary(t_wall0, t_wall1),
         "cpu_baseline": cpu,
