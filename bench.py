@@ -35,7 +35,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=None,
+                   help="timed steps (default: 500 decode, 50 prefill: about 0.15-0.2 s timed)")
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="moe_decode_t16", choices=["moe_decode_t16", "moe_prefill_t8192"])
@@ -76,10 +77,11 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def csrc_digest():
+def csrc_digest(files=None):
+    """Digest of the kernel sources a profile was taken on (all of csrc/ by default)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "trellis_quantized_moe_gemv_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files or os.listdir(d)):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -97,13 +99,14 @@ def profile_traffic(name):
             if "=" in line and not line.lstrip().startswith("#"):
                 k, v = line.split("=", 1)
                 kv[k.strip()] = v.strip()
-    if kv.get("csrc_digest") != csrc_digest() or "dram_bytes_per_unit" not in kv:
+    files = kv.get("csrc_files", "").split() or None
+    if kv.get("csrc_digest") != csrc_digest(files) or "dram_bytes_per_unit" not in kv:
         return None
     return kv
 
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML every 10 ms."""
+    """Samples SM clock and clock-event reasons through NVML every 2 ms."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -137,7 +140,7 @@ class ClockSampler:
                 self.samples.append((time.time(), mhz, rs))
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.002)
 
     def start(self):
         if self.ok:
@@ -235,7 +238,7 @@ def gateup_flops(layer, T, k):
 
 WORKLOADS = {
     "moe_decode_t16": dict(T=16, path="gemv", stage="gemv_gateup",
-                           kernel="moe_gemv_items_kernel<1> (gate/up GEMV + SiLU)",
+                           kernel="moe_gemv_items_kernel<1> (gate/up GEMV, int8 tensor cores)",
                            widths="368/15/1 experts at K=2/3/4", routing="top-8 of N(0,1) logits"),
     "moe_prefill_t8192": dict(T=8192, path="gemm", stage="gemm_gateup",
                               kernel="moe_gemm_kernel<1> (gate/up tcgen05 GEMM + SiLU)",
@@ -285,13 +288,17 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     api.device_status(clear=True)
 
-    # One CUDA graph per layer copy; the library's per-launch profiling events are
-    # captured with the kernels, so every replay re-records them.
+    # One CUDA graph per layer copy.  The library's profiling events are captured with
+    # the kernels (every replay re-records them); the timed graphs carry the events of
+    # the dominant kernel only, a second set of graphs, replayed after the timed region,
+    # those of every stage.
     api.profile_enable(64 * NL)
+    api.profile_stages([wl["stage"]])
     api.profile_collect()
     launches0 = api.launch_count()
-    graphs = []
-    if not args.eager:
+
+    def capture_graphs():
+        out = []
         side = torch.cuda.Stream()
         side.wait_stream(stream)
         with torch.cuda.stream(side):
@@ -299,9 +306,14 @@ def run_ours(args, rank, world, local_rank):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=side):
                     eager_step(c)
-                graphs.append(g)
+                out.append(g)
         stream.wait_stream(side)
         torch.cuda.synchronize()
+        return out
+
+    graphs = []
+    if not args.eager:
+        graphs = capture_graphs()
         launches_per_step = (api.launch_count() - launches0) // NL
         for i in range(args.warmup):
             graphs[i % NL].replay()
@@ -333,8 +345,18 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     launches = (api.launch_count() - launches0) if args.eager else launches_per_step * args.steps
     stages = api.profile_collect()
-    api.profile_disable()
     sampler.stop()
+    # per-stage breakdown, outside the timed region
+    api.profile_stages(None)
+    if args.eager:
+        for i in range(NL):
+            eager_step(i)
+    else:
+        for g in capture_graphs():
+            g.replay()
+    torch.cuda.synchronize()
+    stage_breakdown = api.profile_collect()
+    api.profile_disable()
     ms_total = ev0.elapsed_time(ev1)
     flags = api.device_status()
     if flags:
@@ -348,7 +370,7 @@ def run_ours(args, rank, world, local_rank):
     counts = [b.routing.counts.cpu().numpy() for b in bufs]
     g_ms, g_n = stages[wl["stage"]]
     g_avg_ms = g_ms / max(g_n, 1)
-    stage_avg = {k_: v[0] / v[1] for k_, v in stages.items() if v[1]}
+    stage_avg = {k_: v[0] / v[1] for k_, v in stage_breakdown.items() if v[1]}
     peaks, peak_src = load_peaks()
     if wl["path"] == "gemv":
         per_copy_bytes = [gateup_algorithmic_bytes(L, c) for L, c in zip(layers, counts)]
@@ -532,6 +554,11 @@ def main():
     rank, world, local_rank = dist_env()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.steps is None:
+        if args.impl == "reference":
+            args.steps = 16
+        else:
+            args.steps = 500 if args.workload == "moe_decode_t16" else 50
     if args.impl == "reference":
         run_reference(args, rank, world)
     else:

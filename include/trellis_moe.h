@@ -98,7 +98,7 @@ int tq_device_status(int32_t *flags_out, int clear);
  *   0 route_topk, 1 route_permute, 2 hadamard128 of the input, 3 GEMV gate/up+SiLU,
  *   4 rotation of h, 5 GEMV down, 6 route_unpermute, 7 trellis_decode, 8 trellis_gemv,
  *   9 GEMM gate/up+SiLU, 10 GEMM down, 11 GEMM preparation (tile list, route-ordered
- *   activation rows).
+ *   activation rows), 12 GEMV activation quantisation (x' rows to 16-bit fixed point).
  * tq_profile_enable creates 2*max_launches events (host-side CUDA resources; call it
  * outside graph capture); launches beyond max_launches are not recorded.  A launch made
  * during stream capture records its events as external event-record nodes of the graph,
@@ -106,9 +106,13 @@ int tq_device_status(int32_t *flags_out, int clear);
  * tq_profile_collect waits for the recorded events, writes per-stage summed
  * milliseconds and launch counts into the host arrays stage_ms[n_stages] /
  * stage_launches[n_stages] (skipping events never recorded), and clears the record.
+ * tq_profile_stages restricts recording to the stages whose bit is set in stage_mask
+ * (bit i = stage i; all stages after tq_profile_enable), so that a timed run can carry
+ * the events of one kernel only; TQ_ERR_INVALID_ARG while profiling is off.
  */
 unsigned long long tq_launch_count(void);
 int tq_profile_enable(int max_launches);
+int tq_profile_stages(uint32_t stage_mask);
 int tq_profile_disable(void);
 int tq_profile_collect(double *stage_ms, int32_t *stage_launches, int n_stages);
 
@@ -143,10 +147,18 @@ int hadamard128(const void *x, int x_dtype, int64_t rows, int64_t cols, uint16_t
  *   scales : [rows] fp16.
  *   x_rot  : [batch][cols] fp16 (already rotated, e.g. by hadamard128), 16-byte aligned.
  *   y      : [batch][rows] fp32.
- *   rows % 16 == 0, cols % 128 == 0, 0 <= batch <= 256, K in {2, 3, 4}.
+ *   ws     : device workspace of at least trellis_gemv_workspace_size(rows, cols, batch)
+ *            bytes, 16-byte aligned (TQ_ERR_WORKSPACE otherwise).
+ *   rows % 16 == 0, cols % 128 == 0, cols <= 16384, K in {2, 3, 4}.
+ * Numerics: each row of x_rot enters the tensor-core contraction as 16-bit fixed point
+ * with one power-of-two scale per row (|x_q| <= 32639, rounded to nearest), codes
+ * exactly; sums are exact in int32 and the scales are applied in double.  Elements
+ * smaller than 1/32 of their row's largest are rounded to that row's step.
  */
+size_t trellis_gemv_workspace_size(int rows, int cols, int batch);
 int trellis_gemv(const uint32_t *bits, const uint16_t *scales, int K, int rows, int cols,
-                 const uint16_t *x_rot, int batch, float *y, tq_stream stream);
+                 const uint16_t *x_rot, int batch, float *y, void *ws, size_t ws_bytes,
+                 tq_stream stream);
 
 /*
  * route_topk -- top-k experts of every token and their route weights ("top-8 softmax
@@ -206,9 +218,11 @@ typedef struct {
 } tq_moe_layer;
 
 /*
- * Workspace bytes moe_trellis_gemv / moe_trellis_gemm need for T tokens and k routes:
- * the SwiGLU activations h of every route ([T*k][F] fp32) and their rotation h'
- * ([T*k][F] fp16), 256-byte aligned.  Returns 0 on invalid arguments.
+ * Workspace bytes moe_trellis_gemv and moe_trellis_gemm need for T tokens and k routes
+ * (the larger of the two).  GEMV: the gate and up results of every route ([T*k][2][F]
+ * fp32), the rotated SwiGLU activations h' and the rotated
+ * tokens x' as 16-bit fixed point (two half-words per value plus 8 bytes per row).  GEMM: route-ordered fp16 activation rows, row sums,
+ * h and h' and the tile list.  Returns 0 on invalid arguments.
  */
 size_t moe_trellis_workspace_size(const tq_moe_layer *layer, int T, int k);
 
@@ -224,7 +238,10 @@ size_t moe_trellis_workspace_size(const tq_moe_layer *layer, int T, int k);
  *   y_perm   : [T*k][D] fp32, expert-grouped route order.
  *   ws       : device workspace of at least moe_trellis_workspace_size() bytes.
  *   Mixed widths run in one launch per stage; routes of an expert are processed
- *   together, each weight decoded once per 16 of its routes.
+ *   together, each weight decoded once per 4 of its routes.  x' and h' enter the
+ *   tensor-core contraction as 16-bit fixed point with one power-of-two scale per row
+ *   (as in trellis_gemv); h' is rotated from fp32 h without an fp16 rounding.
+ *   D, F <= 16384.
  */
 int moe_trellis_gemv(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
                      const int32_t *perm, const int32_t *active_ids, const int32_t *n_active,
@@ -239,8 +256,9 @@ int moe_trellis_gemv(const tq_moe_layer *layer, const uint16_t *x_rot, const int
  * counterpart: this is a packaging of the same computation.
  *   Same arguments and result as moe_trellis_gemv, minus ws / ws_bytes.  The workspace
  *   is a 4 MiB array compiled into the library (a __device__ array every GPU that loads
- *   the library holds until exit), so T * k * F may be at most 699,050 (T * k <= 682 for
- *   F = 1024); larger calls return TQ_ERR_WORKSPACE without doing anything.
+ *   the library holds until exit), so the GEMV workspace, 12 * T * k * F + 4 * T * D
+ *   bytes plus 8 bytes per row (T <= 36 at k = 8, D = 4096, F = 1024), must fit in it;
+ *   larger calls return TQ_ERR_WORKSPACE without doing anything.
  *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress,
  *   once per device, with that device current); make that first call before any stream

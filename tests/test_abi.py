@@ -68,10 +68,19 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.hadamard128(FAKE, 7, 4, 128, FAKE, None) == 1            # dtype
     assert lib.hadamard128(MISALIGNED, 0, 4, 128, FAKE, None) == 3
     assert lib.hadamard128(FAKE, 0, 0, 128, FAKE, None) == 0
-    assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 64, FAKE, 1, FAKE, None) == 1   # cols % 128
-    assert lib.trellis_gemv(FAKE, FAKE, 1, 16, 128, FAKE, 1, FAKE, None) == 1  # K
-    assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 128, FAKE, 257, FAKE, None) == 1
-    assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 128, FAKE, 0, FAKE, None) == 0
+    big = ctypes.c_size_t(1 << 40)
+    assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 64, FAKE, 1, FAKE, FAKE, big, None) == 1   # cols % 128
+    assert lib.trellis_gemv(FAKE, FAKE, 1, 16, 128, FAKE, 1, FAKE, FAKE, big, None) == 1  # K
+    assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 32768, FAKE, 1, FAKE, FAKE, big, None) == 2  # cols
+    assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 128, FAKE, 70000, FAKE, FAKE, big, None) == 2
+    assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 128, FAKE, 0, FAKE, None, 0, None) == 0
+    # workspace: quantised rows (two half-words per value), 8 bytes per row, 8 per output
+    need = lib.trellis_gemv_workspace_size(32, 256, 3)
+    assert need == 3 * 2 * 256 * 2 + 256 + 32 * 3 * 8
+    assert lib.trellis_gemv(FAKE, FAKE, 2, 32, 256, FAKE, 3, FAKE, FAKE, ctypes.c_size_t(need - 1),
+                            None) == 4
+    assert lib.trellis_gemv(FAKE, FAKE, 2, 32, 256, FAKE, 3, FAKE, MISALIGNED, ctypes.c_size_t(need),
+                            None) == 3
     assert lib.route_topk(FAKE, 4, 384, 0, FAKE, FAKE, None) == 1
     assert lib.route_topk(FAKE, 4, 4, 8, FAKE, FAKE, None) == 1         # k > E
     assert lib.route_topk(FAKE, 0, 384, 8, FAKE, FAKE, None) == 0
@@ -96,7 +105,9 @@ def _layer_struct(K=2, E=16, D=256, F=128, n_groups=1):
 def test_moe_workspace_and_layer_validation(lib):
     st = _layer_struct()
     need = lib.moe_trellis_workspace_size(ctypes.byref(st), 16, 8)
-    gemv_need = 128 * 128 * 4 + 128 * 128 * 2
+    # GEMV: per-route gate and up results (fp32), h' and x' as 16-bit fixed point (two
+    # half-words per value) and their per-row (exponent, sum)
+    gemv_need = 128 * 2 * 128 * 4 + 128 * 2 * 128 * 2 + 128 * 8 + 16 * 2 * 256 * 2 + 256
     # the GEMM path also holds route-ordered activations (fp16), their row sums, h, h'
     # and its tile list
     gemm_need = 128 * 256 * 2 + 512 + 128 * 128 * 4 + 128 * 128 * 2 + 512 + 256

@@ -124,16 +124,19 @@ def test_gemv_ragged_shapes(api, K, rows, cols, batch):
 
 
 def test_gemv_constant_stream_closed_form(api):
+    # All-zero streams: every code is T16(0) - 255 = -255, so y = s * 2^-12 * (-255) * sum x'.
     rows, cols = 64, 512
     bits = np.zeros(inputs.words_per_matrix(rows, cols, 2), dtype=np.uint32)
     rng = np.random.default_rng(77)
     s = inputs.random_scales(rng, rows)
     x = inputs.random_activations(rng, (3, cols), "bf16")
     x_rot = api.hadamard128(dev_bf16(x))
-    y = api.trellis_gemv(dev_bits(bits), dev_f16(s), 2, rows, cols, x_rot).cpu().numpy()
-    xs = x_rot.float().cpu().numpy().astype(np.float64).sum(1)
-    expect = s.astype(np.float64)[None, :] * 2.0 ** -12 * (-255) * xs[:, None]
-    np.testing.assert_allclose(y, expect, rtol=1e-5, atol=1e-6)
+    y = api.trellis_gemv(dev_bits(bits), dev_f16(s), 2, rows, cols, x_rot).cpu().numpy().astype(np.float64)
+    xr = OL.rotate(x.astype(np.float64))
+    s64 = s.astype(np.float64)[None, :]
+    expect = s64 * 2.0 ** -12 * (-255) * xr.sum(1)[:, None]
+    bound = s64 * 2.0 ** -12 * 255 * np.abs(xr).sum(1)[:, None]
+    _check_projection(y, expect, bound)
 
 
 # ----------------------------------------------------------------------------- routing

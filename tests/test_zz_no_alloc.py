@@ -69,7 +69,7 @@ def test_noalloc_matches_workspace_entry_point_twice(api):
 def test_noalloc_rejects_sizes_beyond_its_scratch(api):
     layer = inputs.small_layer(5, E=12, D=256, F=128)
     dl = api.DeviceLayer.from_synthetic(layer)
-    T, k = 6000, 1          # 6000 routes * 128 * 6 bytes > 4 MiB
+    T, k = 6000, 1          # 6000 routes x F = 128 x 12 bytes of workspace > 4 MiB
     x_rot = torch.zeros((T, 256), dtype=torch.float16, device="cuda")
     routing = api.Routing.empty(T, k, 12, "cuda")
     y = torch.empty((T * k, 256), dtype=torch.float32, device="cuda")

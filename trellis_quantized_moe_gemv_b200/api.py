@@ -51,11 +51,13 @@ SIGNATURES = {
     "tq_device_status": ([_VP, _I], _I),
     "tq_launch_count": ([], ctypes.c_ulonglong),
     "tq_profile_enable": ([_I], _I),
+    "tq_profile_stages": ([ctypes.c_uint32], _I),
     "tq_profile_disable": ([], _I),
     "tq_profile_collect": ([_VP, _VP, _I], _I),
     "trellis_decode": ([_VP, _I, _I, _I, _VP, _VP], _I),
     "hadamard128": ([_VP, _I, _I64, _I64, _VP, _VP], _I),
-    "trellis_gemv": ([_VP, _VP, _I, _I, _I, _VP, _I, _VP, _VP], _I),
+    "trellis_gemv_workspace_size": ([_I, _I, _I], _SZ),
+    "trellis_gemv": ([_VP, _VP, _I, _I, _I, _VP, _I, _VP, _VP, _SZ, _VP], _I),
     "route_topk": ([_VP, _I, _I, _I, _VP, _VP, _VP], _I),
     "route_permute": ([_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "route_unpermute": ([_VP, _VP, _VP, _I, _I, _I, _VP, _VP], _I),
@@ -136,7 +138,8 @@ def device_status(clear: bool = False) -> int:
 
 
 STAGES = ("route_topk", "route_permute", "rotate_x", "gemv_gateup", "rotate_h", "gemv_down",
-          "route_unpermute", "trellis_decode", "trellis_gemv", "gemm_gateup", "gemm_down", "gemm_prep")
+          "route_unpermute", "trellis_decode", "trellis_gemv", "gemm_gateup", "gemm_down", "gemm_prep",
+          "gemv_quant")
 
 
 def launch_count() -> int:
@@ -146,6 +149,12 @@ def launch_count() -> int:
 
 def profile_enable(max_launches: int = 65536):
     _check(_fn("tq_profile_enable")(max_launches), "tq_profile_enable")
+
+
+def profile_stages(names=None):
+    """Record only the launches of the named stages (all stages when names is None)."""
+    mask = 0xFFFFFFFF if names is None else sum(1 << STAGES.index(n) for n in names)
+    _check(_fn("tq_profile_stages")(mask), "tq_profile_stages")
 
 
 def profile_disable():
@@ -184,8 +193,13 @@ def hadamard128(x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None
     return out
 
 
+def trellis_gemv_workspace_size(rows: int, cols: int, batch: int) -> int:
+    return int(_fn("trellis_gemv_workspace_size")(rows, cols, batch))
+
+
 def trellis_gemv(bits: torch.Tensor, scales: torch.Tensor, K: int, rows: int, cols: int,
-                 x_rot: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                 x_rot: torch.Tensor, out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
     _require(bits, torch.int32, "bits")
     _require(scales, torch.float16, "scales")
     _require(x_rot, torch.float16, "x_rot")
@@ -193,8 +207,11 @@ def trellis_gemv(bits: torch.Tensor, scales: torch.Tensor, K: int, rows: int, co
     if out is None:
         out = torch.empty((batch, rows), dtype=torch.float32, device=x_rot.device)
     _require(out, torch.float32, "out")
-    _check(_fn("trellis_gemv")(_p(bits), _p(scales), K, rows, cols, _p(x_rot), batch, _p(out),
-                               _stream(stream)), "trellis_gemv")
+    if ws is None:
+        ws = torch.empty(max(trellis_gemv_workspace_size(rows, cols, batch), 16), dtype=torch.uint8,
+                         device=x_rot.device)
+    _check(_fn("trellis_gemv")(_p(bits), _p(scales), K, rows, cols, _p(x_rot), batch, _p(out), _p(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)), "trellis_gemv")
     return out
 
 

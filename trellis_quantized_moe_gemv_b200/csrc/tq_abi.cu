@@ -52,6 +52,7 @@ namespace tq {
 
 struct Profiler {
     bool on = false;
+    uint32_t stage_mask = 0xFFFFFFFFu;   // stages whose launches are recorded
     int capacity = 0;
     int used = 0;
     cudaEvent_t *events = nullptr;   // 2 per recorded launch
@@ -72,7 +73,7 @@ static void record_event(cudaEvent_t ev, cudaStream_t s) {
 
 LaunchScope::LaunchScope(cudaStream_t s, int st) : stream(s), slot(-1) {
     ++g_launches;
-    if (g_prof.on && g_prof.used < g_prof.capacity) {
+    if (g_prof.on && g_prof.used < g_prof.capacity && st >= 0 && st < 32 && ((g_prof.stage_mask >> st) & 1u)) {
         slot = g_prof.used++;
         g_prof.stage[slot] = st;
         record_event(g_prof.events[2 * slot], s);
@@ -108,6 +109,12 @@ TQ_API int tq_profile_enable(int max_launches) {
     }
     tq::g_prof.capacity = max_launches;
     tq::g_prof.on = true;
+    return TQ_OK;
+}
+
+TQ_API int tq_profile_stages(uint32_t stage_mask) {
+    if (!tq::g_prof.on) return TQ_ERR_INVALID_ARG;
+    tq::g_prof.stage_mask = stage_mask;
     return TQ_OK;
 }
 

@@ -6,305 +6,103 @@
 // (column-major 16x16 tiles), item 4 (per-output scales); gate/up/SiLU/down of the
 // routed experts with fused gate/up post-processing ("October 25 runtime checkpoint").
 //
-// Decode in registers, contraction on the tensor cores (mma.sync, fp16 x fp16 -> fp32):
-//   * A warp walks 8 strips (16 output rows each) at once: lane group g = lane/4 owns
-//     strip g, so every lane decodes the same tile-relative bit offsets (compile-time
-//     shifts) of its own tile; lane t = lane%4 owns columns 4t..4t+3 of each tile.
-//   * Window -> product: R = bottom16(window) * 0x3A2F0000 + 0x6464 is one IMAD and
-//     leaves [0x64, 0x64, lo, hi] (bytes 0..3) with lo/hi the two bytes of
-//     (window*0x3A2F) mod 2^16.  One PRMT per weight interleaves lo (or hi) of two
-//     weights with the 0x64 bytes: fp16 values 1024+lo, 1024+hi (exact).
-//   * Two MMAs per tile (the lo plane and the hi plane) accumulate
-//     sum_j (2048 + t_j) x_j in fp32; a third MMA with A = 1.0 accumulates sum_j x_j,
-//     and the epilogue forms s * 2^-12 * (D - 2303 * sum_j x_j) = s * 2^-12 * sum_j c_j x_j.
-//   * The 4 lanes of a strip split the tile's 8K words; the word after a lane's
-//     quarter (tail-biting for the last quarter) comes from its neighbour by shuffle.
+// Decode in registers, contraction on the tensor cores with integer MMAs
+// (mma.sync m16n8k32, u8 weights x s8 activations -> s32, exact):
+//   * Activations enter as 16-bit fixed point, one power of two per row:
+//     x_q = round(x / 2^e), |x_q| <= 32639, split into two signed bytes
+//     x_q = 256 xh + xl (xl in [-128, 127]).  quantize_rows_kernel writes each byte
+//     twice into a half-word (one row of xh half-words, one of xl half-words) and e
+//     and sum_j x_q of every row.
+//   * A warp walks 8 strips (16 output rows each): lane group g = lane/4 owns strip g
+//     and lane t = lane%4 owns columns 4t..4t+3 of each tile, so every lane decodes the
+//     same tile-relative bit offsets (compile-time shifts).
+//   * Window -> A operand: one funnel shift brings the window to bit 0 (none when it
+//     starts a word) and one integer multiply by 0x3A2F0000 leaves bytes [0, 0, lo, hi],
+//     lo/hi the two bytes of (window * 0x3A2F) mod 2^16.  One A register is one weight
+//     spread over 4 k-slots; its two zero slots meet whatever the activation word holds
+//     there, so the MMA adds (lo + hi) * x = t * x with no byte shuffling.
+//   * The MMA's 8 columns are 4 routes x 2 limbs (column 2r: route r's xh, 2r+1: its
+//     xl).  |partial sums| <= 510 * 128 * cols < 2^31 for cols <= 16384.
+//   * Epilogue, in double: y = s * 2^-12 * 2^e * (256 H + L - 255 sum_j x_q), H and L
+//     the two limb sums; sum_j c_j x_j = sum_j t_j x_j - 255 sum_j x_j.
+//   * Bit streams reach shared memory by bulk copies into a per-warp ring of stages
+//     (one mbarrier per stage, bounded waits); activations come from L2, one tile
+//     ahead.
 #include "tq_common.cuh"
 
 namespace tq {
 
-constexpr int kGemvWarps = 8;
-constexpr int kGemvThreads = kGemvWarps * 32;
-constexpr uint32_t kSelLo = 0x4602u;   // [A.b2, A.b0, B.b2, B.b0] -> (1024+lo_A, 1024+lo_B)
-constexpr uint32_t kSelHi = 0x5713u;   // [A.b3, A.b1, B.b3, B.b1] -> (1024+hi_A, 1024+hi_B)
-constexpr uint32_t kOneH2 = 0x3C003C00u;
-constexpr float kOffset = 2.0f * 1024.0f + 255.0f;   // (1024+lo)+(1024+hi) = c + 2303
-
-// Packed T16 product of the window at compile-time bit offset O of the lane's span.
-template <int O, int NS>
-__device__ __forceinline__ uint32_t t16_pack(const uint32_t (&v)[NS]) {
-    constexpr int wi = O >> 5, sh = O & 31;
-    uint32_t bottom;
-    if constexpr (sh == 0) bottom = v[wi];
-    else bottom = funnel_r(v[wi], v[wi + 1], sh);
-    return bottom * (kT16Mult << 16) + 0x6464u;
-}
-
-template <int NG>
-struct Acc {
-    float d[8][NG][4];   // [row pair][token group][fragment]
-    float s[NG][4];      // sum of x per token (ones MMA)
-};
-
-// One column tile of the lane's strip: decode 64 windows (rows 0..15 x the lane's 4
-// columns) and issue the MMAs for every token group.
-template <int K, int NG, int P>
-__device__ __forceinline__ void tile_pairs(const uint32_t (&v)[2 * K + 1], const uint2 (&xb)[NG],
-                                           Acc<NG> &acc) {
-    if constexpr (P < 8) {
-        constexpr int r0 = P, r1 = P + 8;
-        const uint32_t R00 = t16_pack<0 * 16 * K + K * r0>(v), R01 = t16_pack<1 * 16 * K + K * r0>(v);
-        const uint32_t R02 = t16_pack<2 * 16 * K + K * r0>(v), R03 = t16_pack<3 * 16 * K + K * r0>(v);
-        const uint32_t R10 = t16_pack<0 * 16 * K + K * r1>(v), R11 = t16_pack<1 * 16 * K + K * r1>(v);
-        const uint32_t R12 = t16_pack<2 * 16 * K + K * r1>(v), R13 = t16_pack<3 * 16 * K + K * r1>(v);
-        const uint32_t l0 = prmt(R00, R01, kSelLo), l1 = prmt(R10, R11, kSelLo);
-        const uint32_t l2 = prmt(R02, R03, kSelLo), l3 = prmt(R12, R13, kSelLo);
-        const uint32_t h0 = prmt(R00, R01, kSelHi), h1 = prmt(R10, R11, kSelHi);
-        const uint32_t h2 = prmt(R02, R03, kSelHi), h3 = prmt(R12, R13, kSelHi);
-#pragma unroll
-        for (int g = 0; g < NG; ++g) {
-            mma_f16_16816(acc.d[P][g], l0, l1, l2, l3, xb[g].x, xb[g].y);
-            mma_f16_16816(acc.d[P][g], h0, h1, h2, h3, xb[g].x, xb[g].y);
-        }
-        tile_pairs<K, NG, P + 1>(v, xb, acc);
-    }
-}
-
-template <int K>
-__device__ __forceinline__ void load_quarter(const uint32_t *p, uint32_t (&w)[2 * K]) {
-    if constexpr (K == 2) {
-        uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
-        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-    } else if constexpr (K == 3) {
-        uint2 a = __ldg(reinterpret_cast<const uint2 *>(p));
-        uint2 b = __ldg(reinterpret_cast<const uint2 *>(p + 2));
-        uint2 c = __ldg(reinterpret_cast<const uint2 *>(p + 4));
-        w[0] = a.x; w[1] = a.y; w[2] = b.x; w[3] = b.y; w[4] = c.x; w[5] = c.y;
-    } else {
-        uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
-        uint4 b = __ldg(reinterpret_cast<const uint4 *>(p + 4));
-        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-    }
-}
-
-// Accumulate column tiles [jb, je) of the lane's strip (tile 0 of the strip at
-// `strip0`, tiles 8K words apart) against the lane's token rows xr[g] (fp16, may be
-// null: contributes zero).  Loads run PF tiles ahead.
-template <int K, int NG>
-__device__ __forceinline__ void accumulate(const uint32_t *__restrict__ strip0, int jb, int je,
-                                           const __half *const (&xr)[NG], Acc<NG> &acc) {
-    constexpr int PF = 2;
-    constexpr int WPT = 8 * K;
-    const int lane = threadIdx.x & 31, t4 = lane & 3;
-    const int src = (lane & ~3) | ((lane + 1) & 3);
-    const uint32_t *q0 = strip0 + 2 * K * t4;
-    uint32_t buf[PF][2 * K];
-    uint2 xb[PF][NG];
-#pragma unroll
-    for (int s = 0; s < PF; ++s) {
-        if (jb + s < je) {
-            load_quarter<K>(q0 + (size_t)(jb + s) * WPT, buf[s]);
-#pragma unroll
-            for (int g = 0; g < NG; ++g)
-                xb[s][g] = xr[g] ? __ldg(reinterpret_cast<const uint2 *>(xr[g] + 16 * (jb + s) + 4 * t4))
-                                 : make_uint2(0u, 0u);
-        }
-    }
-    for (int j = jb; j < je; j += PF) {
-#pragma unroll
-        for (int s = 0; s < PF; ++s) {
-            if (j + s < je) {
-                uint32_t v[2 * K + 1];
-#pragma unroll
-                for (int i = 0; i < 2 * K; ++i) v[i] = buf[s][i];
-                v[2 * K] = __shfl_sync(0xffffffffu, buf[s][0], src);
-                uint2 x[NG];
-#pragma unroll
-                for (int g = 0; g < NG; ++g) x[g] = xb[s][g];
-                const int jn = j + s + PF;
-                if (jn < je) {
-                    load_quarter<K>(q0 + (size_t)jn * WPT, buf[s]);
-#pragma unroll
-                    for (int g = 0; g < NG; ++g)
-                        xb[s][g] = xr[g] ? __ldg(reinterpret_cast<const uint2 *>(xr[g] + 16 * jn + 4 * t4))
-                                         : make_uint2(0u, 0u);
-                }
-                tile_pairs<K, NG, 0>(v, x, acc);
-#pragma unroll
-                for (int g = 0; g < NG; ++g)
-                    mma_f16_16816(acc.s[g], kOneH2, kOneH2, kOneH2, kOneH2, x[g].x, x[g].y);
-            }
-        }
-    }
-}
-
-template <int NG>
-__device__ __forceinline__ void zero(Acc<NG> &acc) {
-#pragma unroll
-    for (int p = 0; p < 8; ++p)
-#pragma unroll
-        for (int g = 0; g < NG; ++g)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc.d[p][g][i] = 0.f;
-#pragma unroll
-    for (int g = 0; g < NG; ++g)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc.s[g][i] = 0.f;
-}
-
-// Shared-memory reduction buffers of one CTA.
-template <int NG>
-struct RedSmem {
-    float d[kGemvWarps][NG][8][16][8];   // [warp][group][strip][row][token]
-    float s[kGemvWarps][NG][8];          // [warp][group][token]
-};
-
-// Store the warp's partials: fragment (row g -> strip g row r0, row g+8 -> row r1,
-// tokens 2t, 2t+1).
-template <int NG>
-__device__ __forceinline__ void store_partials(const Acc<NG> &acc, RedSmem<NG> &red) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int gq = lane >> 2, t4 = lane & 3;
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            red.d[warp][g][gq][p][2 * t4] = acc.d[p][g][0];
-            red.d[warp][g][gq][p][2 * t4 + 1] = acc.d[p][g][1];
-            red.d[warp][g][gq][p + 8][2 * t4] = acc.d[p][g][2];
-            red.d[warp][g][gq][p + 8][2 * t4 + 1] = acc.d[p][g][3];
-        }
-        if (gq == 0) {
-            red.s[warp][g][2 * t4] = acc.s[g][0];
-            red.s[warp][g][2 * t4 + 1] = acc.s[g][1];
-        }
-    }
-}
-
-// Sum over warps in fixed order: raw accumulation of (strip, row, token, group).
-template <int NG>
-__device__ __forceinline__ float red_d(const RedSmem<NG> &red, int g, int strip, int row, int tok) {
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < kGemvWarps; ++w) v += red.d[w][g][strip][row][tok];
-    return v;
-}
-template <int NG>
-__device__ __forceinline__ float red_s(const RedSmem<NG> &red, int g, int tok) {
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < kGemvWarps; ++w) v += red.s[w][g][tok];
-    return v;
-}
-
-__device__ __forceinline__ float finish(float d, float sx, float scale) {
-    return scale * kKappa * (d - kOffset * sx);
-}
-
-// Subnormal planes: D = 2^-24 * sum_j t_j x_j, so sum_j c_j x_j = 2^24 D - 255 sum_j x_j.
-__device__ __forceinline__ float finish_sub(float d, float sx, float scale) {
-    return scale * kKappa * fmaf(16777216.0f, d, -255.0f * sx);
-}
-
-__device__ __forceinline__ void split_range(int n, int part, int parts, int &b, int &e) {
-    const int per = (n + parts - 1) / parts;
-    b = min(n, part * per);
-    e = min(n, b + per);
-}
-
-// --------------------------------------------------------------------------- single GEMV
-
-// CTA = one group of 8 strips (128 rows) x a batch pass of 8*NG tokens; the 8 warps
-// split the column tiles.
-template <int K, int NG>
-__global__ void __launch_bounds__(kGemvThreads, 2)
-    trellis_gemv_kernel(const uint32_t *__restrict__ bits, const __half *__restrict__ scales, int rows,
-                        int cols, const __half *__restrict__ x, int batch, float *__restrict__ y) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    RedSmem<NG> &red = *reinterpret_cast<RedSmem<NG> *>(smem_raw);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2;
-    const int n_strips = rows / 16, tiles = cols / 16;
-    const int strip = blockIdx.x * 8 + gq;
-    const int tok0 = blockIdx.y * 8 * NG;
-    const uint32_t *strip0 =
-        bits + (size_t)min(strip, n_strips - 1) * tiles * (8 * K);  // clamp: rows beyond are dropped
-    const __half *xr[NG];
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-        const int b = tok0 + 8 * g + gq;
-        xr[g] = b < batch ? x + (size_t)b * cols : nullptr;
-    }
-    Acc<NG> acc;
-    zero(acc);
-    int jb, je;
-    split_range(tiles, warp, kGemvWarps, jb, je);
-    accumulate<K, NG>(strip0, jb, je, xr, acc);
-    store_partials(acc, red);
-    __syncthreads();
-    for (int i = threadIdx.x; i < NG * 8 * 16 * 8; i += kGemvThreads) {
-        const int tok = i & 7, row = (i >> 3) & 15, st = (i >> 7) & 7, g = i >> 10;
-        const int b = tok0 + 8 * g + tok, r = (blockIdx.x * 8 + st) * 16 + row;
-        if (b < batch && r < rows)
-            y[(size_t)b * rows + r] =
-                finish(red_d(red, g, st, row, tok), red_s(red, g, tok), __half2float(scales[r]));
-    }
-}
-
-// --------------------------------------------------------------------------- MoE GEMV
-
-struct ExpertRef {
-    int K;
-    int group, index;             // width group and position inside it
-    const uint32_t *gate, *up, *down;
-    const __half *s_gate, *s_up, *s_down;
-};
-
-__device__ __forceinline__ bool expert_ref(const tq_moe_layer &L, int e, ExpertRef &r) {
-    if (e < 0 || e >= L.E) return false;
-    const int slot = L.expert_slot[e];
-    if (slot < 0) return false;
-    const int gi = slot >> 16, idx = slot & 0xFFFF;
-    if (gi >= L.n_groups) return false;
-    const tq_width_group &G = L.groups[gi];
-    if (idx >= G.n_experts) return false;
-    const size_t words_proj = (size_t)(L.D / 16) * (L.F / 16) * 8 * G.K;
-    r.K = G.K;
-    r.group = gi;
-    r.index = idx;
-    r.gate = G.gate + (size_t)idx * words_proj;
-    r.up = G.up + (size_t)idx * words_proj;
-    r.down = G.down + (size_t)idx * words_proj;
-    r.s_gate = reinterpret_cast<const __half *>(G.s_gate) + (size_t)idx * L.F;
-    r.s_up = reinterpret_cast<const __half *>(G.s_up) + (size_t)idx * L.F;
-    r.s_down = reinterpret_cast<const __half *>(G.s_down) + (size_t)idx * L.D;
-    return true;
-}
-
-// ----------------------------------------------------------------------------- MoE items
-//
-// MoE GEMV work item = one CTA of kItemWarps warps: (active expert, 8 strips of 16
-// rows, 8 of the expert's routes).  The warps split the column tiles into contiguous
-// ranges; each streams its range of the 8 strips through its own ring of shared-memory
-// stages filled by bulk copies (lanes 0..7 copy one strip each, completing on one
-// mbarrier per stage; consumers poll with a bound), and the warps' MMA partial sums
-// are added in shared memory in a fixed order at the end of the item.
-//
-// Per weight: one funnel shift brings the window to bit 0 (none for windows that start
-// a word), one integer multiply by 0x3A2F0000 leaves the T16 product's bytes lo, hi in
-// bytes 2 and 3 with zeros below, and one PRMT pairs the lo (or hi) bytes of two
-// weights with zero bytes: fp16 subnormals lo * 2^-24 and hi * 2^-24, exact operands.
-// The MMA accumulates D = 2^-24 * sum_j t_j x_j in fp32 (no offset to cancel).
-
+constexpr int kMaxCols = 16384;        // keeps every int32 partial sum in range
+constexpr int kQMax = 32639;           // 127 * 256 + 127: both bytes stay signed
 constexpr int kItemWarps = 4;
 constexpr int kItemThreads = kItemWarps * 32;
 constexpr int kStages = 2;
-constexpr int kSlotBytes = 576;               // per strip per stage: >= 8*64, 5*96, 4*128 B,
-                                              // 64 B pad so 2 strips share no bank in a phase
+constexpr int kSlotBytes = 576;        // per strip per stage: >= 8*64, 5*96, 4*128 B,
+                                       // 64 B pad so 2 strips share no bank in a phase
 constexpr int kStageBytes = 8 * kSlotBytes;
 
 template <int K>
 constexpr int tiles_per_stage() { return K == 2 ? 8 : (K == 3 ? 5 : 4); }
+
+__device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// T16 product of the window at compile-time bit offset O of the lane's span, in the
+// high half of the result (low half zero): bytes [0, 0, lo, hi].
+template <int O, int NS>
+__device__ __forceinline__ uint32_t t16_product_hi(const uint32_t (&v)[NS]) {
+    constexpr int wi = O >> 5, sh = O & 31;
+    uint32_t bottom;
+    if constexpr (sh == 0) bottom = v[wi];
+    else bottom = funnel_r(v[wi], v[wi + 1], sh);
+    return bottom * (kT16Mult << 16);
+}
+
+// Integer accumulators of NB blocks of 4 routes: [row pair P][block][fragment];
+// fragment 0/1 = (row P, route t, limb h/l), 2/3 = (row P + 8, ...).
+template <int NB>
+struct AccI {
+    int d[8][NB][4];
+};
+
+template <int NB>
+__device__ __forceinline__ void zero(AccI<NB> &acc) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc.d[p][b][i] = 0;
+}
+
+// Rows P and P + 8 of the lane's tile against its 4 columns: 8 windows, 2 MMAs per
+// block (columns 4t, 4t+1 as k-slot groups t, 4+t; then columns 4t+2, 4t+3).
+template <int K, int NB, int P>
+__device__ __forceinline__ void tile_rows(const uint32_t (&v)[2 * K + 1], const uint4 (&xb)[NB], AccI<NB> &acc) {
+    if constexpr (P < 8) {
+        constexpr int r0 = P, r1 = P + 8;
+        const uint32_t R00 = t16_product_hi<0 * 16 * K + K * r0>(v);
+        const uint32_t R01 = t16_product_hi<1 * 16 * K + K * r0>(v);
+        const uint32_t R02 = t16_product_hi<2 * 16 * K + K * r0>(v);
+        const uint32_t R03 = t16_product_hi<3 * 16 * K + K * r0>(v);
+        const uint32_t R10 = t16_product_hi<0 * 16 * K + K * r1>(v);
+        const uint32_t R11 = t16_product_hi<1 * 16 * K + K * r1>(v);
+        const uint32_t R12 = t16_product_hi<2 * 16 * K + K * r1>(v);
+        const uint32_t R13 = t16_product_hi<3 * 16 * K + K * r1>(v);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            imma_16832(acc.d[P][b], R00, R10, R01, R11, xb[b].x, xb[b].y);
+            imma_16832(acc.d[P][b], R02, R12, R03, R13, xb[b].z, xb[b].w);
+        }
+        tile_rows<K, NB, P + 1>(v, xb, acc);
+    }
+}
 
 // A warp's ring: its stage buffers and one mbarrier per stage.  The barriers live in a
 // region of their own (ItemSmem::bar) that nothing else ever writes: an mbarrier's
@@ -318,37 +116,6 @@ struct __align__(128) ItemSmem {
     unsigned char buf[kItemWarps][kStages][kStageBytes];
     uint64_t bar[kItemWarps][kStages];
 };
-
-// T16 product of the window at compile-time bit offset O of the lane's span, in the
-// high half of the result (low half zero): bytes [0, 0, lo, hi].
-template <int O, int NS>
-__device__ __forceinline__ uint32_t t16_product_hi(const uint32_t (&v)[NS]) {
-    constexpr int wi = O >> 5, sh = O & 31;
-    uint32_t bottom;
-    if constexpr (sh == 0) bottom = v[wi];
-    else bottom = funnel_r(v[wi], v[wi + 1], sh);
-    return bottom * (kT16Mult << 16);
-}
-
-template <int K, int P>
-__device__ __forceinline__ void tile_pairs_sub(const uint32_t (&v)[2 * K + 1], uint2 xb, Acc<1> &acc) {
-    if constexpr (P < 8) {
-        constexpr int r0 = P, r1 = P + 8;
-        const uint32_t R00 = t16_product_hi<0 * 16 * K + K * r0>(v);
-        const uint32_t R01 = t16_product_hi<1 * 16 * K + K * r0>(v);
-        const uint32_t R02 = t16_product_hi<2 * 16 * K + K * r0>(v);
-        const uint32_t R03 = t16_product_hi<3 * 16 * K + K * r0>(v);
-        const uint32_t R10 = t16_product_hi<0 * 16 * K + K * r1>(v);
-        const uint32_t R11 = t16_product_hi<1 * 16 * K + K * r1>(v);
-        const uint32_t R12 = t16_product_hi<2 * 16 * K + K * r1>(v);
-        const uint32_t R13 = t16_product_hi<3 * 16 * K + K * r1>(v);
-        mma_f16_16816(acc.d[P][0], prmt(R00, R01, kSelLo), prmt(R10, R11, kSelLo), prmt(R02, R03, kSelLo),
-                      prmt(R12, R13, kSelLo), xb.x, xb.y);
-        mma_f16_16816(acc.d[P][0], prmt(R00, R01, kSelHi), prmt(R10, R11, kSelHi), prmt(R02, R03, kSelHi),
-                      prmt(R12, R13, kSelHi), xb.x, xb.y);
-        tile_pairs_sub<K, P + 1>(v, xb, acc);
-    }
-}
 
 __device__ __forceinline__ void ring_init(const WarpRing &ring) {
     const int lane = threadIdx.x & 31;
@@ -377,17 +144,28 @@ __device__ __forceinline__ void ring_issue(const WarpRing &ring, int st, int c, 
     if (lane < 8) bulk_g2s(ring.buf[st] + lane * kSlotBytes, strip_lane + (size_t)jb * (8 * K), nt * TB, &ring.bar[st]);
 }
 
-// Stream tiles [j0, je) of the 8 strips against the lane's token row xr (fp16 or null).
-// Returns false, after draining its copies, if a bounded wait gave up.
-template <int K>
+// Activation half-words of the lane's 4 columns of tile j (null row: zeros): each
+// 16-bit value holds one signed byte twice, so a 32-bit word [x_c x_c x_c+1 x_c+1]
+// is the B operand of column c+1 (bytes 2, 3) and, shifted left by 16, of column c.
+__device__ __forceinline__ uint2 x_halves(const uint16_t *xw, int j, int t4) {
+    return xw ? __ldg(reinterpret_cast<const uint2 *>(xw + 16 * j + 4 * t4)) : make_uint2(0u, 0u);
+}
+
+// Stream tiles [j0, je) of the 8 strips against the lane's activation rows xw[b] (the
+// lane's limb of route 4b + g/2 of the pass, or null); activations are loaded one tile
+// ahead.  Returns false, after draining its copies, if a bounded wait gave up.
+template <int K, int NB>
 __device__ __forceinline__ bool stream_range(const WarpRing &ring, uint32_t &parity, int j0, int je,
-                                          const uint32_t *strip_lane, const __half *xr, Acc<1> &acc) {
+                                             const uint32_t *strip_lane, const uint16_t *const (&xw)[NB],
+                                             AccI<NB> &acc) {
     constexpr int S = tiles_per_stage<K>();
     constexpr int TB = 32 * K;
     const int lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
     const int n_chunks = (je - j0 + S - 1) / S;
     for (int c = 0; c < min(kStages, n_chunks); ++c) ring_issue<K>(ring, c, c, j0, je, strip_lane);
-    uint2 xn = (xr && j0 < je) ? __ldg(reinterpret_cast<const uint2 *>(xr + 16 * j0 + 4 * t4)) : make_uint2(0u, 0u);
+    uint2 xn[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) xn[b] = j0 < je ? x_halves(xw[b], j0, t4) : make_uint2(0u, 0u);
     for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kStages;
         const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&ring.bar[st], (parity >> st) & 1u));
@@ -420,12 +198,17 @@ __device__ __forceinline__ bool stream_range(const WarpRing &ring, uint32_t &par
                 v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
                 v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
             }
+            // word after the lane's quarter: the next quarter's first (tail-biting)
             v[2 * K] = *reinterpret_cast<const uint32_t *>(tile + 8 * K * ((t4 + 1) & 3));
-            const uint2 x = xn;
+            uint4 x[NB];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) x[b] = make_uint4(xn[b].x << 16, xn[b].x, xn[b].y << 16, xn[b].y);
             const int jn = jb + t + 1;
-            if (xr && jn < je) xn = __ldg(reinterpret_cast<const uint2 *>(xr + 16 * jn + 4 * t4));
-            tile_pairs_sub<K, 0>(v, x, acc);
-            mma_f16_16816(acc.s[0], kOneH2, kOneH2, kOneH2, kOneH2, x.x, x.y);
+            if (jn < je) {
+#pragma unroll
+                for (int b = 0; b < NB; ++b) xn[b] = x_halves(xw[b], jn, t4);
+            }
+            tile_rows<K, NB, 0>(v, x, acc);
         }
         __syncwarp();
         if (c + kStages < n_chunks) ring_issue<K>(ring, st, c + kStages, j0, je, strip_lane);
@@ -433,32 +216,234 @@ __device__ __forceinline__ bool stream_range(const WarpRing &ring, uint32_t &par
     return true;
 }
 
+template <int NB>
+__device__ __forceinline__ bool stream_any(int K, const WarpRing &ring, uint32_t &parity, int j0, int je,
+                                           const uint32_t *strip_lane, const uint16_t *const (&xw)[NB],
+                                           AccI<NB> &acc) {
+    if (K == 2) return stream_range<2, NB>(ring, parity, j0, je, strip_lane, xw, acc);
+    if (K == 3) return stream_range<3, NB>(ring, parity, j0, je, strip_lane, xw, acc);
+    return stream_range<4, NB>(ring, parity, j0, je, strip_lane, xw, acc);
+}
+
 // Shared-memory partials of the CTA's warps; aliases the stage buffers (never the
 // barriers) once every warp has consumed its last stage.
+template <int NB>
 struct ItemRed {
-    float d[kItemWarps][8][16][8];   // [warp][strip][row][token]
-    float s[kItemWarps][8];          // [warp][token]
+    int d[kItemWarps][8][16][4 * NB][2];   // [warp][strip][row][route][limb]
 };
-static_assert(sizeof(ItemRed) <= sizeof(ItemSmem::buf), "reduction buffer must fit in the stage buffers");
+static_assert(sizeof(ItemRed<2>) <= sizeof(ItemSmem::buf), "reduction buffer must fit in the stage buffers");
 
-// GATEUP: item = (active expert, 64 intermediate rows: strips 0..3 of gate, 0..3 of up),
-//         out = h [routes][F] fp32, h = silu(gate x') * (up x').
-// !GATEUP: item = (active expert, 128 output rows), xsrc = h' [routes][F] fp16,
-//          out = y [routes][D] fp32.
+template <int NB>
+__device__ __forceinline__ void store_partials(const AccI<NB> &acc, ItemRed<NB> &red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            *reinterpret_cast<int2 *>(red.d[warp][gq][p][4 * b + t4]) = make_int2(acc.d[p][b][0], acc.d[p][b][1]);
+            *reinterpret_cast<int2 *>(red.d[warp][gq][p + 8][4 * b + t4]) = make_int2(acc.d[p][b][2], acc.d[p][b][3]);
+        }
+}
+
+// Sum over warps in fixed order (exact): limb sums of (strip, row, route).
+template <int NB>
+__device__ __forceinline__ int2 red_sum(const ItemRed<NB> &red, int strip, int row, int route) {
+    int h = 0, l = 0;
+#pragma unroll
+    for (int w = 0; w < kItemWarps; ++w) {
+        h += red.d[w][strip][row][route][0];
+        l += red.d[w][strip][row][route][1];
+    }
+    return make_int2(h, l);
+}
+
+// y = s * 2^-12 * 2^e * (256 H + L - 255 sum x_q), formed in double.
+__device__ __forceinline__ float finish_q(int H, int L, int2 meta, float scale) {
+    const double a = 256.0 * (double)H + (double)L - 255.0 * (double)meta.y;
+    return (float)(a * ldexp((double)scale * (double)kKappa, meta.x));
+}
+
+__device__ __forceinline__ void split_range(int n, int part, int parts, int &b, int &e) {
+    const int per = (n + parts - 1) / parts;
+    b = min(n, part * per);
+    e = min(n, b + per);
+}
+
+// ------------------------------------------------------------------ activation rows
+//
+// One CTA of 8 warps per row of `cols` values (a multiple of 128): take the row from
+// its source (optionally rotating every 128-chunk with fwht128_warp, the hadamard128
+// transform), take max |v| over the row, pick e with max / 2^e <= 32639
+// (e = ilogb(max) - 14, one more if the mantissa is too large), and write
+// x_q = rint(v / 2^e) as its two signed bytes, each held twice in a half-word:
+// xq[row][0][col] = xh * 0x0101, xq[row][1][col] = xl * 0x0101.
+// meta[row] = (e, sum_j x_q).  The row is read again in the second pass instead of
+// being kept in registers, so any row length works.
+
+// Plain rows x[row][cols].
+template <typename T>
+struct RowSrc {
+    const T *x;
+    int cols;
+    __device__ __forceinline__ void load(int row, int c, int lane, float (&v)[4]) const {
+        const float4 f = load4<T>(x + (size_t)row * cols + (size_t)c * 128 + 4 * lane);
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    }
+};
+
+// SwiGLU of the gate/up GEMV's column-split partial sums: h = silu(sum_s g_s) * sum_s u_s
+// from gu[row][s][0][cols] (gate) and gu[row][s][1][cols] (up).
+struct SwigluSrc {
+    const float *gu;
+    int cols, splits;
+    __device__ __forceinline__ void load(int row, int c, int lane, float (&v)[4]) const {
+        const float *p = gu + (size_t)row * splits * 2 * cols + (size_t)c * 128 + 4 * lane;
+        float4 g = *reinterpret_cast<const float4 *>(p), u = *reinterpret_cast<const float4 *>(p + cols);
+        for (int sp = 1; sp < splits; ++sp) {
+            const float4 g2 = *reinterpret_cast<const float4 *>(p + (size_t)sp * 2 * cols);
+            const float4 u2 = *reinterpret_cast<const float4 *>(p + (size_t)sp * 2 * cols + cols);
+            g.x += g2.x; g.y += g2.y; g.z += g2.z; g.w += g2.w;
+            u.x += u2.x; u.y += u2.y; u.z += u2.z; u.w += u2.w;
+        }
+        v[0] = silu_f32(g.x) * u.x;
+        v[1] = silu_f32(g.y) * u.y;
+        v[2] = silu_f32(g.z) * u.z;
+        v[3] = silu_f32(g.w) * u.w;
+    }
+};
+
+template <typename Src, bool ROTATE>
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int cols, uint16_t *__restrict__ xq,
+                                                            int2 *__restrict__ meta) {
+    __shared__ float s_max[8];
+    __shared__ int s_sum[8];
+    const int row = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int chunks = cols / 128;
+    float m = 0.f;
+    for (int c = warp; c < chunks; c += 8) {
+        float v[4];
+        src.load(row, c, lane, v);
+        if constexpr (ROTATE) fwht128_warp(v, lane);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = fmaxf(m, fabsf(v[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) s_max[warp] = m;
+    __syncthreads();
+    m = s_max[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, s_max[w]);
+    int e = 0;
+    if (m > 0.f) {                   // a NaN or infinite max is not supported
+        e = ilogbf(m) - 14;
+        if (ldexpf(m, -e) > (float)kQMax) ++e;
+    }
+    uint16_t *qh = xq + (size_t)row * 2 * cols, *ql = qh + cols;
+    int sum = 0;
+    for (int c = warp; c < chunks; c += 8) {
+        float v[4];
+        src.load(row, c, lane, v);
+        if constexpr (ROTATE) fwht128_warp(v, lane);
+        uint32_t wh[4], wl[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int q = __float2int_rn(ldexpf(v[i], -e));
+            q = max(-kQMax, min(kQMax, q));
+            sum += q;
+            const int lo = ((q + 128) & 255) - 128;
+            const int hi = (q - lo) >> 8;
+            wh[i] = (uint32_t)(hi & 255) * 0x0101u;
+            wl[i] = (uint32_t)(lo & 255) * 0x0101u;
+        }
+        const size_t off = (size_t)c * 128 + 4 * lane;
+        *reinterpret_cast<uint2 *>(qh + off) = make_uint2(wh[0] | (wh[1] << 16), wh[2] | (wh[3] << 16));
+        *reinterpret_cast<uint2 *>(ql + off) = make_uint2(wl[0] | (wl[1] << 16), wl[2] | (wl[3] << 16));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) s_sum[warp] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int total = 0;
+        for (int w = 0; w < 8; ++w) total += s_sum[w];
+        meta[row] = make_int2(e, total);
+    }
+}
+
+template <bool ROTATE, typename Src>
+int launch_quantize_rows(const Src &src, long long rows, int cols, uint16_t *xq, int2 *meta, cudaStream_t s,
+                         int stage) {
+    if (rows <= 0) return TQ_OK;
+    if (rows > 0x7fffffffll) return TQ_ERR_UNSUPPORTED;
+    LaunchScope ls(s, stage);
+    quantize_rows_kernel<Src, ROTATE><<<(unsigned)rows, 256, 0, s>>>(src, cols, xq, meta);
+    return launch_status();
+}
+
+// --------------------------------------------------------------------------- MoE GEMV
+
+struct ExpertRef {
+    int K;
+    int group, index;             // width group and position inside it
+    const uint32_t *gate, *up, *down;
+    const __half *s_gate, *s_up, *s_down;
+};
+
+__device__ __forceinline__ bool expert_ref(const tq_moe_layer &L, int e, ExpertRef &r) {
+    if (e < 0 || e >= L.E) return false;
+    const int slot = L.expert_slot[e];
+    if (slot < 0) return false;
+    const int gi = slot >> 16, idx = slot & 0xFFFF;
+    if (gi >= L.n_groups) return false;
+    const tq_width_group &G = L.groups[gi];
+    if (idx >= G.n_experts) return false;
+    const size_t words_proj = (size_t)(L.D / 16) * (L.F / 16) * 8 * G.K;
+    r.K = G.K;
+    r.group = gi;
+    r.index = idx;
+    r.gate = G.gate + (size_t)idx * words_proj;
+    r.up = G.up + (size_t)idx * words_proj;
+    r.down = G.down + (size_t)idx * words_proj;
+    r.s_gate = reinterpret_cast<const __half *>(G.s_gate) + (size_t)idx * L.F;
+    r.s_up = reinterpret_cast<const __half *>(G.s_up) + (size_t)idx * L.F;
+    r.s_down = reinterpret_cast<const __half *>(G.s_down) + (size_t)idx * L.D;
+    return true;
+}
+
+// MoE GEMV work item = one CTA of kItemWarps warps: (active expert, 8 strips of 16
+// rows, column range, passes of 4 of the expert's routes).  The warps split the item's
+// column tiles into contiguous ranges; each streams its range of the 8 strips through
+// its own ring, and the warps' integer partial sums are added in shared memory at the
+// end of a pass.
+//
+// GATEUP: item = (active expert, 64 intermediate rows: strips 0..3 of gate, 0..3 of
+//         up, column split sp of kGateUpSplits); activations = the tokens' quantised
+//         rotated rows (xq, xmeta indexed by token); out = gu [routes][split][2][F]
+//         fp32, the split's share of gate x' and up x' (the SwiGLU is applied when h
+//         is rotated and quantised).  More than one split multiplies the CTAs of a
+//         small batch; measured on the 16-token decode layer it gains nothing, so the
+//         columns are not split.
+// !GATEUP: item = (active expert, 128 output rows); activations = quantised h'
+//          (indexed by route); out = y [routes][D] fp32.
+constexpr int kGateUpSplits = 1;
+
 template <bool GATEUP>
 __global__ void __launch_bounds__(kItemThreads, 5)
-    moe_gemv_items_kernel(const tq_moe_layer L, const __half *__restrict__ xsrc,
+    moe_gemv_items_kernel(const tq_moe_layer L, const uint16_t *__restrict__ xq, const int2 *__restrict__ xmeta,
                           const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm,
                           const int32_t *__restrict__ active_ids, const int32_t *__restrict__ n_active_p,
                           int k, int n_routes, float *__restrict__ out) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     ItemSmem &sm_items = *reinterpret_cast<ItemSmem *>(smem_raw);
-    ItemRed &red = *reinterpret_cast<ItemRed *>(smem_raw);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2, t4 = lane & 3;
-    const int per_expert = GATEUP ? L.F / 64 : L.D / 128;
+    ItemRed<1> &red = *reinterpret_cast<ItemRed<1> *>(smem_raw);
+    __shared__ int s_row[4];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2;
+    constexpr int splits = GATEUP ? kGateUpSplits : 1;
+    const int per_expert = (GATEUP ? L.F / 64 : L.D / 128) * splits;
     const int item = blockIdx.x;
     if (item >= *n_active_p * per_expert) return;
-    const int a = item / per_expert, sub = item % per_expert;
+    const int a = item / per_expert, sub = (item % per_expert) / splits, sp = item % splits;
     const int e = active_ids[a];
     ExpertRef ex;
     if (!expert_ref(L, e, ex)) {
@@ -469,10 +454,14 @@ __global__ void __launch_bounds__(kItemThreads, 5)
     ring_init(ring);
     uint32_t parity = 0;
 
+    const int cols = GATEUP ? L.D : L.F;
     const int r0 = offsets[e], ne = offsets[e + 1] - r0;
-    const int tiles = GATEUP ? L.D / 16 : L.F / 16;
-    int jb, je;
-    split_range(tiles, warp, kItemWarps, jb, je);
+    const int tiles = cols / 16;
+    int cb, ce, jb, je;
+    split_range(tiles, sp, splits, cb, ce);
+    split_range(ce - cb, warp, kItemWarps, jb, je);
+    jb += cb;
+    je += cb;
     const int cs = lane & 7;
     const uint32_t *strip_lane;
     if (GATEUP)
@@ -480,72 +469,120 @@ __global__ void __launch_bounds__(kItemThreads, 5)
     else
         strip_lane = ex.down + (size_t)(sub * 8 + cs) * tiles * (8 * ex.K);
 
-    for (int tb = 0; tb < ne; tb += 8) {
-        const int tt = tb + gq;
-        const __half *xr = nullptr;
-        if (tt < ne) {
-            if (GATEUP) {
-                const int pr = perm[r0 + tt];
-                if (pr >= 0 && pr < n_routes) xr = xsrc + (size_t)(pr / k) * L.D;
-            } else {
-                xr = xsrc + (size_t)(r0 + tt) * L.F;
+    for (int tb = 0; tb < ne; tb += 4) {
+        // activation row of each route of the pass (-1: none)
+        if (threadIdx.x < 4) {
+            const int tt = tb + threadIdx.x;
+            int row = -1;            // -1: no route; -2: route with an invalid index
+            if (tt < ne) {
+                if (GATEUP) {
+                    const int pr = perm[r0 + tt];
+                    row = (pr >= 0 && pr < n_routes) ? pr / k : -2;
+                } else {
+                    row = r0 + tt;
+                }
             }
-        }
-        Acc<1> acc;
-        zero(acc);
-        bool ok;
-        if (ex.K == 2) ok = stream_range<2>(ring, parity, jb, je, strip_lane, xr, acc);
-        else if (ex.K == 3) ok = stream_range<3>(ring, parity, jb, je, strip_lane, xr, acc);
-        else ok = stream_range<4>(ring, parity, jb, je, strip_lane, xr, acc);
-        ok = __syncthreads_and(ok);
-        if (!ok) return;   // every warp drained its copies; the item is left unwritten
-        // partials -> shared memory (the rings are idle now)
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            red.d[warp][gq][p][2 * t4] = acc.d[p][0][0];
-            red.d[warp][gq][p][2 * t4 + 1] = acc.d[p][0][1];
-            red.d[warp][gq][p + 8][2 * t4] = acc.d[p][0][2];
-            red.d[warp][gq][p + 8][2 * t4 + 1] = acc.d[p][0][3];
-        }
-        if (gq == 0) {
-            red.s[warp][2 * t4] = acc.s[0][0];
-            red.s[warp][2 * t4 + 1] = acc.s[0][1];
+            s_row[threadIdx.x] = row;
         }
         __syncthreads();
+        const int my_row = s_row[gq >> 1];
+        const uint16_t *xw[1] = {my_row >= 0 ? xq + (size_t)my_row * 2 * cols + (gq & 1) * cols : nullptr};
+        AccI<1> acc;
+        zero(acc);
+        bool ok = stream_any<1>(ex.K, ring, parity, jb, je, strip_lane, xw, acc);
+        ok = __syncthreads_and(ok);
+        if (!ok) return;   // every warp drained its copies; the item is left unwritten
+        store_partials(acc, red);   // the rings are idle now
+        __syncthreads();
         if (GATEUP) {
-            for (int i = threadIdx.x; i < 4 * 16 * 8; i += kItemThreads) {
-                const int tok = i & 7, row = (i >> 3) & 15, st = i >> 7;
-                const int t2 = tb + tok;
-                if (t2 >= ne) continue;
-                float dg = 0.f, du = 0.f, sx = 0.f;
-#pragma unroll
-                for (int w = 0; w < kItemWarps; ++w) {
-                    dg += red.d[w][st][row][tok];
-                    du += red.d[w][st + 4][row][tok];
-                    sx += red.s[w][tok];
-                }
+            for (int i = threadIdx.x; i < 4 * 16 * 4; i += kItemThreads) {
+                const int rt = i & 3, row = (i >> 2) & 15, st = i >> 6;
+                const int xrow = s_row[rt];
+                if (xrow == -1) continue;
                 const int f = (sub * 4 + st) * 16 + row;
-                const float gv = finish_sub(dg, sx, __half2float(ex.s_gate[f]));
-                const float uv = finish_sub(du, sx, __half2float(ex.s_up[f]));
-                out[(size_t)(r0 + t2) * L.F + f] = silu_f32(gv) * uv;
+                float gv = 0.f, uv = 0.f;    // a route with an invalid index: h = 0
+                if (xrow >= 0) {
+                    int2 m = xmeta[xrow];
+                    if (sp) m.y = 0;         // the -255 sum x term is added once, by split 0
+                    const int2 g = red_sum(red, st, row, rt), u = red_sum(red, st + 4, row, rt);
+                    gv = finish_q(g.x, g.y, m, __half2float(ex.s_gate[f]));
+                    uv = finish_q(u.x, u.y, m, __half2float(ex.s_up[f]));
+                }
+                float *o = out + ((size_t)(r0 + tb + rt) * splits + sp) * 2 * L.F + f;
+                o[0] = gv;
+                o[L.F] = uv;
             }
         } else {
-            for (int i = threadIdx.x; i < 8 * 16 * 8; i += kItemThreads) {
-                const int tok = i & 7, row = (i >> 3) & 15, st = i >> 7;
-                const int t2 = tb + tok;
-                if (t2 >= ne) continue;
-                float dd = 0.f, sx = 0.f;
-#pragma unroll
-                for (int w = 0; w < kItemWarps; ++w) {
-                    dd += red.d[w][st][row][tok];
-                    sx += red.s[w][tok];
-                }
+            for (int i = threadIdx.x; i < 8 * 16 * 4; i += kItemThreads) {
+                const int rt = i & 3, row = (i >> 2) & 15, st = i >> 6;
+                const int xrow = s_row[rt];
+                if (xrow < 0) continue;
+                const int2 y = red_sum(red, st, row, rt);
                 const int d = (sub * 8 + st) * 16 + row;
-                out[(size_t)(r0 + t2) * L.D + d] = finish_sub(dd, sx, __half2float(ex.s_down[d]));
+                out[(size_t)xrow * L.D + d] = finish_q(y.x, y.y, xmeta[xrow], __half2float(ex.s_down[d]));
             }
         }
-        __syncthreads();   // the rings are reused by the next pass
+        __syncthreads();   // the rings and s_row are reused by the next pass
     }
+}
+
+// ------------------------------------------------------------------------ single GEMV
+//
+// CTA = (group of 8 strips = 128 rows, column split, pass of 4*NB tokens); the 4 warps
+// split the CTA's column tiles.  The integer partial sums of all CTAs of a row group
+// are added into acc [batch][rows][2] with atomics (exact, so order-independent), and
+// gemv_finish_kernel applies the scales.
+template <int NB>
+__global__ void __launch_bounds__(kItemThreads, 4)
+    trellis_gemv_kernel(const uint32_t *__restrict__ bits, int K, int rows, int cols, const uint16_t *__restrict__ xq,
+                        int batch, int col_splits, int *__restrict__ acc_out) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    ItemSmem &sm_items = *reinterpret_cast<ItemSmem *>(smem_raw);
+    ItemRed<NB> &red = *reinterpret_cast<ItemRed<NB> *>(smem_raw);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2;
+    const int n_strips = rows / 16, tiles = cols / 16;
+    const WarpRing ring{sm_items.buf[warp], sm_items.bar[warp]};
+    ring_init(ring);
+    uint32_t parity = 0;
+    int cb, ce, jb, je;
+    split_range(tiles, blockIdx.y, col_splits, cb, ce);
+    split_range(ce - cb, warp, kItemWarps, jb, je);
+    jb += cb;
+    je += cb;
+    const int strip = min((int)blockIdx.x * 8 + (lane & 7), n_strips - 1);   // rows beyond are dropped
+    const uint32_t *strip_lane = bits + (size_t)strip * tiles * (8 * K);
+    const int tok0 = blockIdx.z * 4 * NB;
+    const uint16_t *xw[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const int t = tok0 + 4 * b + (gq >> 1);
+        xw[b] = t < batch ? xq + (size_t)t * 2 * cols + (gq & 1) * cols : nullptr;
+    }
+    AccI<NB> acc;
+    zero(acc);
+    bool ok = stream_any<NB>(K, ring, parity, jb, je, strip_lane, xw, acc);
+    ok = __syncthreads_and(ok);
+    if (!ok) return;
+    store_partials(acc, red);
+    __syncthreads();
+    for (int i = threadIdx.x; i < 8 * 16 * 4 * NB; i += kItemThreads) {
+        const int rt = i % (4 * NB), row = (i / (4 * NB)) & 15, st = i / (64 * NB);
+        const int t = tok0 + rt, r = (blockIdx.x * 8 + st) * 16 + row;
+        if (t >= batch || r >= rows) continue;
+        const int2 v = red_sum(red, st, row, rt);
+        int *dst = acc_out + ((size_t)t * rows + r) * 2;
+        atomicAdd(dst, v.x);
+        atomicAdd(dst + 1, v.y);
+    }
+}
+
+__global__ void gemv_finish_kernel(const int *__restrict__ acc, const int2 *__restrict__ meta,
+                                   const __half *__restrict__ scales, int rows, int batch, float *__restrict__ y) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (size_t)rows * batch) return;
+    const int t = (int)(i / rows), r = (int)(i % rows);
+    const int2 hl = reinterpret_cast<const int2 *>(acc)[i];
+    y[i] = finish_q(hl.x, hl.y, meta[t], __half2float(scales[r]));
 }
 
 template <typename Kern>
@@ -558,10 +595,63 @@ inline int set_smem(Kern kern, size_t bytes) {
 
 inline size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
+// Workspace of the single GEMV: quantised rows, their (e, sum), integer sums.
+struct GemvWs {
+    uint16_t *xq;
+    int2 *meta;
+    int *acc;
+};
+
+size_t gemv_ws_bytes(int rows, int cols, int batch) {
+    return align256((size_t)batch * 2 * cols * 2) + align256((size_t)batch * 8) + align256((size_t)rows * batch * 8);
+}
+
+GemvWs gemv_ws(void *ws, int rows, int cols, int batch) {
+    char *p = reinterpret_cast<char *>(ws);
+    GemvWs w;
+    w.xq = reinterpret_cast<uint16_t *>(p);
+    p += align256((size_t)batch * 2 * cols * 2);
+    w.meta = reinterpret_cast<int2 *>(p);
+    p += align256((size_t)batch * 8);
+    w.acc = reinterpret_cast<int *>(p);
+    return w;
+}
+
+template <int NB>
+int run_gemv(const uint32_t *bits, const __half *scales, int K, int rows, int cols, const __half *x, int batch,
+             float *y, const GemvWs &w, cudaStream_t s) {
+    const size_t smem = sizeof(ItemSmem);
+    static bool configured = false;
+    if (!configured) {
+        if (set_smem(trellis_gemv_kernel<NB>, smem)) return TQ_ERR_CUDA;
+        configured = true;
+    }
+    int st = launch_quantize_rows<false>(RowSrc<__half>{x, cols}, batch, cols, w.xq, w.meta, s, kStageGemvQuant);
+    if (st) return st;
+    if (cudaMemsetAsync(w.acc, 0, (size_t)rows * batch * 8, s) != cudaSuccess) return record_cuda_error("cudaMemsetAsync");
+    const int groups = (rows / 16 + 7) / 8, passes = (batch + 4 * NB - 1) / (4 * NB), tiles = cols / 16;
+    const int want = (4 * num_sms() + groups * passes - 1) / (groups * passes);
+    const int splits = max(1, min(want, tiles / (2 * kItemWarps)));
+    {
+        LaunchScope ls(s, kStageGemv);
+        trellis_gemv_kernel<NB><<<dim3(groups, splits, passes), kItemThreads, smem, s>>>(bits, K, rows, cols, w.xq,
+                                                                                         batch, splits, w.acc);
+    }
+    st = launch_status();
+    if (st) return st;
+    const size_t n = (size_t)rows * batch;
+    LaunchScope ls(s, kStageGemv);
+    gemv_finish_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w.acc, w.meta, scales, rows, batch, y);
+    return launch_status();
+}
+
+// ------------------------------------------------------------------------ MoE launch
+
 int validate_layer(const tq_moe_layer *L) {
     if (!L) return TQ_ERR_INVALID_ARG;
     if (L->E < 1 || L->E > 1024 || L->D < 128 || L->F < 128 || L->D % 128 || L->F % 128)
         return TQ_ERR_INVALID_ARG;
+    if (L->D > kMaxCols || L->F > kMaxCols) return TQ_ERR_UNSUPPORTED;
     if (L->n_groups < 1 || L->n_groups > 3 || !L->expert_slot) return TQ_ERR_INVALID_ARG;
     for (int g = 0; g < L->n_groups; ++g) {
         const tq_width_group &G = L->groups[g];
@@ -573,13 +663,38 @@ int validate_layer(const tq_moe_layer *L) {
     return TQ_OK;
 }
 
+// Workspace of the MoE GEMV: gate/up partial sums gu [routes][splits][2][F] fp32,
+// quantised h' [routes][2][F] half-words and its (e, sum) per route, quantised x'
+// [T][2][D] half-words and its (e, sum) per token.
+struct MoeGemvWs {
+    float *gu;
+    uint16_t *hq;
+    int2 *hmeta;
+    uint16_t *xq;
+    int2 *xmeta;
+};
+
 size_t workspace_bytes(const tq_moe_layer *L, int T, int k) {
     const size_t routes = (size_t)T * k;
-    return align256(routes * L->F * sizeof(float)) + align256(routes * L->F * sizeof(__half));
+    return align256(routes * kGateUpSplits * 2 * L->F * 4) + align256(routes * 2 * L->F * 2) + align256(routes * 8) +
+           align256((size_t)T * 2 * L->D * 2) + align256((size_t)T * 8);
 }
 
-int launch_hadamard128(const void *x, int x_dtype, long long rows, long long cols, __half *out,
-                       cudaStream_t s, int stage);
+MoeGemvWs moe_gemv_ws(const tq_moe_layer *L, int T, int k, void *ws) {
+    const size_t routes = (size_t)T * k;
+    char *p = reinterpret_cast<char *>(ws);
+    MoeGemvWs w;
+    w.gu = reinterpret_cast<float *>(p);
+    p += align256(routes * kGateUpSplits * 2 * L->F * 4);
+    w.hq = reinterpret_cast<uint16_t *>(p);
+    p += align256(routes * 2 * L->F * 2);
+    w.hmeta = reinterpret_cast<int2 *>(p);
+    p += align256(routes * 8);
+    w.xq = reinterpret_cast<uint16_t *>(p);
+    p += align256((size_t)T * 2 * L->D * 2);
+    w.xmeta = reinterpret_cast<int2 *>(p);
+    return w;
+}
 
 int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offsets, const int32_t *perm,
                  const int32_t *active_ids, const int32_t *n_active, int T, int k, float *y_perm,
@@ -592,39 +707,25 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
         configured = true;
     }
     const int routes = T * k;
-    float *h = reinterpret_cast<float *>(ws);
-    __half *h_rot = reinterpret_cast<__half *>(reinterpret_cast<char *>(ws) +
-                                               align256((size_t)routes * L->F * sizeof(float)));
+    const MoeGemvWs w = moe_gemv_ws(L, T, k, ws);
     const int max_active = min(L->E, routes);
-    const int gu_items = max_active * (L->F / 64);
+    const int gu_items = max_active * (L->F / 64) * kGateUpSplits;
     const int dn_items = max_active * (L->D / 128);
+    int st = launch_quantize_rows<false>(RowSrc<__half>{x_rot, L->D}, T, L->D, w.xq, w.xmeta, s, kStageGemvQuant);
+    if (st) return st;
     {
         LaunchScope ls(s, kStageGemvGateUp);
-        moe_gemv_items_kernel<true><<<gu_items, kItemThreads, smem, s>>>(*L, x_rot, offsets, perm, active_ids,
-                                                                          n_active, k, routes, h);
+        moe_gemv_items_kernel<true><<<gu_items, kItemThreads, smem, s>>>(*L, w.xq, w.xmeta, offsets, perm, active_ids,
+                                                                          n_active, k, routes, w.gu);
     }
-    int st = launch_status();
+    st = launch_status();
     if (st) return st;
-    st = launch_hadamard128(h, TQ_DTYPE_F32, routes, L->F, h_rot, s, kStageRotateH);
+    st = launch_quantize_rows<true>(SwigluSrc{w.gu, L->F, kGateUpSplits}, routes, L->F, w.hq, w.hmeta, s,
+                                    kStageRotateH);
     if (st) return st;
     LaunchScope ls(s, kStageGemvDown);
-    moe_gemv_items_kernel<false><<<dn_items, kItemThreads, smem, s>>>(*L, h_rot, offsets, perm, active_ids,
+    moe_gemv_items_kernel<false><<<dn_items, kItemThreads, smem, s>>>(*L, w.hq, w.hmeta, offsets, perm, active_ids,
                                                                        n_active, k, routes, y_perm);
-    return launch_status();
-}
-
-template <int K, int NG>
-int run_gemv(const uint32_t *bits, const __half *scales, int rows, int cols, const __half *x, int batch,
-             float *y, cudaStream_t s) {
-    const size_t smem = sizeof(RedSmem<NG>);
-    static bool configured = false;
-    if (!configured) {
-        if (set_smem(trellis_gemv_kernel<K, NG>, smem)) return TQ_ERR_CUDA;
-        configured = true;
-    }
-    dim3 grid((rows / 16 + 7) / 8, (batch + 8 * NG - 1) / (8 * NG));
-    LaunchScope ls(s, kStageGemv);
-    trellis_gemv_kernel<K, NG><<<grid, kGemvThreads, smem, s>>>(bits, scales, rows, cols, x, batch, y);
     return launch_status();
 }
 
@@ -632,29 +733,28 @@ int run_gemv(const uint32_t *bits, const __half *scales, int rows, int cols, con
 
 using namespace tq;
 
+TQ_API size_t trellis_gemv_workspace_size(int rows, int cols, int batch) {
+    if (rows < 0 || cols < 0 || batch < 0 || rows % 16 || cols % 128 || cols > kMaxCols) return 0;
+    return gemv_ws_bytes(rows, cols, batch);
+}
+
 TQ_API int trellis_gemv(const uint32_t *bits, const uint16_t *scales, int K, int rows, int cols,
-                        const uint16_t *x_rot, int batch, float *y, tq_stream stream) {
-    if (K < 2 || K > 4 || rows < 0 || cols < 0 || rows % 16 || cols % 128 || batch < 0 || batch > 256)
+                        const uint16_t *x_rot, int batch, float *y, void *ws, size_t ws_bytes, tq_stream stream) {
+    if (K < 2 || K > 4 || rows < 0 || cols < 0 || rows % 16 || cols % 128 || batch < 0)
         return TQ_ERR_INVALID_ARG;
+    if (cols > kMaxCols || batch > 65535) return TQ_ERR_UNSUPPORTED;
     if (rows == 0 || batch == 0) return TQ_OK;
     if (cols == 0) return TQ_ERR_INVALID_ARG;
     if (!bits || !scales || !x_rot || !y) return TQ_ERR_INVALID_ARG;
     if (!aligned16(bits) || !aligned16(x_rot)) return TQ_ERR_ALIGNMENT;
+    if (!ws || ws_bytes < gemv_ws_bytes(rows, cols, batch)) return TQ_ERR_WORKSPACE;
+    if (!aligned16(ws)) return TQ_ERR_ALIGNMENT;
     cudaStream_t s = (cudaStream_t)stream;
     const __half *sc = reinterpret_cast<const __half *>(scales);
     const __half *x = reinterpret_cast<const __half *>(x_rot);
-    if (batch <= 8) {
-        switch (K) {
-            case 2: return run_gemv<2, 1>(bits, sc, rows, cols, x, batch, y, s);
-            case 3: return run_gemv<3, 1>(bits, sc, rows, cols, x, batch, y, s);
-            default: return run_gemv<4, 1>(bits, sc, rows, cols, x, batch, y, s);
-        }
-    }
-    switch (K) {
-        case 2: return run_gemv<2, 2>(bits, sc, rows, cols, x, batch, y, s);
-        case 3: return run_gemv<3, 2>(bits, sc, rows, cols, x, batch, y, s);
-        default: return run_gemv<4, 2>(bits, sc, rows, cols, x, batch, y, s);
-    }
+    const GemvWs w = gemv_ws(ws, rows, cols, batch);
+    if (batch <= 4) return run_gemv<1>(bits, sc, K, rows, cols, x, batch, y, w, s);
+    return run_gemv<2>(bits, sc, K, rows, cols, x, batch, y, w, s);
 }
 
 namespace tq {
