@@ -46,6 +46,9 @@ def parse_args():
     p.add_argument("--eager", action="store_true", help="launch every step from the host instead of a CUDA graph")
     p.add_argument("--tokens", type=int, default=None, help="override the workload's token count (profiling runs)")
     p.add_argument("--experts", type=int, default=None, help="override the workload's expert count (profiling runs)")
+    p.add_argument("--sweep", action="store_true",
+                   help="batch sweep of the mixed-width decode layer (T = 1 .. 16384, uniform top-8): "
+                        "device time of the GEMV and the GEMM path at every T, one JSON line each")
     return p.parse_args()
 
 
@@ -549,6 +552,68 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+SWEEP_T = (1, 8, 64, 256, 384, 512, 1024, 2048, 16384)   # the configured sizes plus three near the crossover
+
+
+def run_sweep(args, local_rank):
+    """Both expert paths on the mixed-width 384-expert layer at every sweep size: CUDA-graph
+    replays of the whole layer (routing to combine) cycled over 4 layer copies (4.9 GB of
+    bit streams, beyond L2), timed with CUDA events after warm-up."""
+    import torch
+    from trellis_quantized_moe_gemv_b200 import api, inputs
+    from trellis_quantized_moe_gemv_b200 import build as tqbuild
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    tqbuild.build()
+    api.lib()
+    w0, layers, _ = build_decode_workload(api, inputs, torch, device, 0, 4)
+    host_layer, k = w0["layer"], 8
+    stream = torch.cuda.current_stream()
+    results = []
+    for T in SWEEP_T:
+        w = inputs.moe_sweep_tokens(T, layer=host_layer)
+        x = torch.from_numpy(w["x"]).to(torch.bfloat16).to(device)
+        lg = torch.from_numpy(w["logits"]).to(device)
+        row = {"sweep": "moe_sweep_tokens", "tokens": T, "top_k": k, "routing": "top-8 of N(0,1) logits"}
+        for path in ("gemv", "gemm"):
+            bufs = [api.MoeBuffers(L, T, k) for L in layers]
+            for c, L in enumerate(layers):
+                api.moe_layer(L, x, lg, k, bufs=bufs[c], path=path)
+            torch.cuda.synchronize()
+            graphs = []
+            side = torch.cuda.Stream()
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                for c, L in enumerate(layers):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=side):
+                        api.moe_layer(L, x, lg, k, bufs=bufs[c], path=path)
+                    graphs.append(g)
+            stream.wait_stream(side)
+            for i in range(8):
+                graphs[i % 4].replay()
+            torch.cuda.synchronize()
+            steps = max(8, min(400, int(4e5 / max(T, 1))))
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(steps):
+                graphs[i % 4].replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / steps
+            row[path + "_ms"] = ms
+            row[path + "_tok_s"] = T / (ms * 1e-3)
+            del graphs, bufs
+            torch.cuda.empty_cache()
+        row["faster"] = "gemv" if row["gemv_ms"] <= row["gemm_ms"] else "gemm"
+        results.append(row)
+        print(json.dumps(row), flush=True)
+    cross = next((r["tokens"] for r in results if r["faster"] == "gemm"), None)
+    print(json.dumps({"sweep": "moe_sweep_tokens", "gemm_faster_from_tokens": cross,
+                      "library_switch_tokens": api.GEMM_MIN_TOKENS}), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local_rank = dist_env()
@@ -559,7 +624,10 @@ def main():
             args.steps = 16
         else:
             args.steps = 500 if args.workload == "moe_decode_t16" else 50
-    if args.impl == "reference":
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args, local_rank)
+    elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
         run_ours(args, rank, world, local_rank)
