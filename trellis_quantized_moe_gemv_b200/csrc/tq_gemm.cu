@@ -280,7 +280,6 @@ __global__ void __launch_bounds__(kGThreads, 1)
     while ((32 << box) < n) ++box;          // box rows 32 << box >= n
     const int nmma = max(16, (n + 15) & ~15);
     const int num_kb = args.kdim / kGBK;
-    const int tiles_per_strip = args.kdim / 16;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kGBitsStages; ++i) {
@@ -309,7 +308,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
         const bool ok = __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity));
         if (!ok) sm.abort = 1;
-        return ok && !*(volatile int32_t *)&sm.abort;
+        // one answer for the whole warp, so that its lanes leave their loops together
+        return ok && !__any_sync(0xffffffffu, *(volatile int32_t *)&sm.abort != 0);
     };
 
     if (warp == 0) {
