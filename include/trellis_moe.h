@@ -110,6 +110,15 @@ int tq_device_status(int32_t *flags_out, int clear);
  * (bit i = stage i; all stages after tq_profile_enable), so that a timed run can carry
  * the events of one kernel only; TQ_ERR_INVALID_ARG while profiling is off.
  */
+/*
+ * tq_selftest_bounded_wait -- failure-detection check (no counterpart on the pages):
+ * one warp runs the library's bounded mbarrier wait on a barrier that nothing arrives
+ * on.  After limit_us microseconds (1 .. 10,000,000) the wait gives up, raises device
+ * flag bit 1 (read it with tq_device_status) and the kernel returns; nothing traps and
+ * the context stays usable.  Asynchronous on `stream`, like every entry point.
+ */
+int tq_selftest_bounded_wait(uint32_t limit_us, tq_stream stream);
+
 unsigned long long tq_launch_count(void);
 int tq_profile_enable(int max_launches);
 int tq_profile_stages(uint32_t stage_mask);

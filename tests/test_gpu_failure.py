@@ -1,0 +1,56 @@
+"""Failure detection without a GPU fault: the library's bounded device wait, run on an
+mbarrier that nothing arrives on, gives up after its limit, raises device flag bit 1 and
+returns; the context stays usable (a layer computed right after matches the oracle)."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import layer as OL
+from trellis_quantized_moe_gemv_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    import trellis_quantized_moe_gemv_b200.build as b
+    b.build()
+    from trellis_quantized_moe_gemv_b200 import api as A
+    A.device_status(clear=True)
+    return A
+
+
+def test_bounded_wait_gives_up_and_flags(api):
+    api.device_status(clear=True)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    api.selftest_bounded_wait(20000)          # 20 ms
+    torch.cuda.synchronize()
+    elapsed = time.time() - t0
+    assert api.device_status(clear=True) == 2
+    assert 0.015 <= elapsed < 5.0
+
+
+def test_context_usable_after_a_wait_gave_up(api):
+    api.selftest_bounded_wait(5000)
+    torch.cuda.synchronize()
+    assert api.device_status(clear=True) == 2
+    layer = inputs.small_layer(808, E=12, D=256, F=128)
+    rng = np.random.default_rng(809)
+    x = inputs.random_activations(rng, (6, 256), "bf16")
+    logits = inputs.normal_logits(rng, 6, 12)
+    dl = api.DeviceLayer.from_synthetic(layer)
+    out = api.moe_layer(dl, torch.from_numpy(x).to(torch.bfloat16).cuda(), torch.from_numpy(logits).cuda(), 4,
+                        path="gemv")
+    torch.cuda.synchronize()
+    res = OL.moe_layer(layer, x, logits, 4)
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - res["out"]) <= res["bound"] + 1e-6 * np.abs(res["out"]) + 1e-12)
+    assert api.device_status() == 0
+
+
+def test_selftest_rejects_bad_limits(api):
+    with pytest.raises(api.TQError, match="INVALID"):
+        api.selftest_bounded_wait(0)

@@ -52,6 +52,7 @@ SIGNATURES = {
     "tq_launch_count": ([], ctypes.c_ulonglong),
     "tq_profile_enable": ([_I], _I),
     "tq_profile_stages": ([ctypes.c_uint32], _I),
+    "tq_selftest_bounded_wait": ([ctypes.c_uint32, _VP], _I),
     "tq_profile_disable": ([], _I),
     "tq_profile_collect": ([_VP, _VP, _I], _I),
     "trellis_decode": ([_VP, _I, _I, _I, _VP, _VP], _I),
@@ -149,6 +150,12 @@ def launch_count() -> int:
 
 def profile_enable(max_launches: int = 65536):
     _check(_fn("tq_profile_enable")(max_launches), "tq_profile_enable")
+
+
+def selftest_bounded_wait(limit_us: int, stream=None):
+    """Run the library's bounded device wait on a barrier nothing arrives on (gives up
+    after limit_us and raises device flag bit 1)."""
+    _check(_fn("tq_selftest_bounded_wait")(limit_us, _stream(stream)), "tq_selftest_bounded_wait")
 
 
 def profile_stages(names=None):

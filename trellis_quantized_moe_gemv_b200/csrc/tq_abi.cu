@@ -147,3 +147,25 @@ TQ_API int tq_profile_collect(double *stage_ms, int32_t *stage_launches, int n_s
     tq::g_prof.used = 0;
     return TQ_OK;
 }
+
+// ---------------------------------------------------------------------- failure check
+namespace tq {
+// One warp waits, with the library's bounded wait, for a phase of a fresh mbarrier that
+// nothing ever arrives on: the wait gives up after limit_ns, raises device flag bit 1
+// and the kernel returns normally.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    mbar_wait_sleep(&bar, 0, limit_ns);
+}
+}  // namespace tq
+
+TQ_API int tq_selftest_bounded_wait(uint32_t limit_us, tq_stream stream) {
+    if (limit_us < 1 || limit_us > 10000000u) return TQ_ERR_INVALID_ARG;
+    tq::selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_us * 1000ull);
+    return tq::launch_status();
+}

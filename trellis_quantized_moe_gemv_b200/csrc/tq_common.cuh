@@ -169,15 +169,17 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t pa
 
 // Wait for the phase with the given parity, letting the hardware suspend the thread
 // between polls (no spinning that would take issue slots from working warps), and give
-// up after kWaitNs of wall time (device flag bit 1).  The timer is read only every 64
-// polls.
+// up after limit_ns of wall time (device flag bit 1).  Each poll may suspend for up to
+// limit_ns / 256 (at most 1 ms); the timer is read every 8 polls.
 constexpr uint64_t kWaitNs = 4000000000ull;
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, uint64_t limit_ns = kWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+    const uint64_t h = limit_ns / 256;
+    const uint32_t hint_ns = h > 1000000ull ? 1000000u : (h < 1000ull ? 1000u : (uint32_t)h);
     for (uint32_t n = 1;; ++n) {
-        if (mbar_try_wait_suspend(bar, parity, 1000000u)) return true;
-        if ((n & 63u) == 0 && global_timer_ns() - t0 > kWaitNs) break;
+        if (mbar_try_wait_suspend(bar, parity, hint_ns)) return true;
+        if ((n & 7u) == 0 && global_timer_ns() - t0 > limit_ns) break;
     }
     raise_flag(2);
     return false;
