@@ -41,6 +41,7 @@ constexpr int kGGroups = 2;        // K-block slots: K-block kb is decoded into 
 constexpr int kGDecodeGroups = 2 * kGGroups;   // 4-warp groups: (K-block parity, weight tile)
 constexpr int kGBitsStages = 6;    // bit-stream ring (multiple of kGGroups)
 constexpr int kGBStages = 3;       // activation (B) ring
+constexpr int kGKbRing = 4;        // K-block barrier ring: > the A and B reuse distances
 constexpr int kGDecodeWarps = 4 * kGDecodeGroups;
 constexpr int kGFirstDecodeWarp = 3;   // warp 0: bit-stream producer, 1: MMA, 2: B producer
 constexpr int kGThreads = (kGFirstDecodeWarp + kGDecodeWarps) * 32;
@@ -55,10 +56,13 @@ struct __align__(1024) GemmSmem {
     unsigned char bits[kGBitsStages][kGStrips * kGBitsSlot];
     uint64_t bits_full[kGBitsStages];          // producer -> decoders (count 1 + bytes)
     uint64_t bits_empty[kGBitsStages];         // decoders -> producer (count 8)
-    uint64_t b_full[kGBStages];                // B producer -> MMA (count 1 + bytes)
-    uint64_t b_empty[kGBStages];               // MMA -> B producer (commit)
-    uint64_t a_full[kGGroups];                 // decoders -> MMA (count 8)
-    uint64_t a_empty[kGGroups];                // MMA -> decoders (commit)
+    // One barrier pair per K-block (ring of kGKbRing): kb_ready completes when the 8
+    // decode warps of the K-block have arrived and its activation slab has landed (the
+    // MMA thread waits once per K-block); kb_done is the MMA commit, waited by the
+    // decoders before reusing the A slot (K-block kb + 2) and by the activation
+    // producer before reusing the slab stage (kb + 3).
+    uint64_t kb_ready[kGKbRing];
+    uint64_t kb_done[kGKbRing];
     uint64_t acc_full;                         // MMA -> epilogue
     uint64_t mma_done;                         // MMA drain on early exit
     uint32_t tmem_base;
@@ -286,13 +290,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
             mbar_init(&sm.bits_full[i], 1);
             mbar_init(&sm.bits_empty[i], 8);
         }
-        for (int i = 0; i < kGBStages; ++i) {
-            mbar_init(&sm.b_full[i], 1);
-            mbar_init(&sm.b_empty[i], 1);
-        }
-        for (int i = 0; i < kGGroups; ++i) {
-            mbar_init(&sm.a_full[i], 8);
-            mbar_init(&sm.a_empty[i], 1);
+        for (int i = 0; i < kGKbRing; ++i) {
+            mbar_init(&sm.kb_ready[i], 8 + 1);   // 8 decode warps + the producer's expect_tx
+            mbar_init(&sm.kb_done[i], 1);
         }
         mbar_init(&sm.acc_full, 1);
         mbar_init(&sm.mma_done, 1);
@@ -343,42 +343,50 @@ __global__ void __launch_bounds__(kGThreads, 1)
         int issued = 0;
         for (int kb = 0; kb < num_kb; ++kb) {
             const int i = kb % kGBStages;
-            if (kb >= kGBStages && !wait(&sm.b_empty[i], ((kb / kGBStages) - 1) & 1)) break;
+            const int pk = kb - kGBStages;    // the K-block that last used stage i
+            if (pk >= 0 && !wait(&sm.kb_done[pk % kGKbRing], (pk / kGKbRing) & 1)) break;
+            uint64_t *ready = &sm.kb_ready[kb % kGKbRing];
             if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.b_full[i], (32u << box) * 128u);
-                tma_load_2d(sm.b[i], &maps.b[box], kb * kGBK, r0 + n0, &sm.b_full[i]);
+                mbar_arrive_expect_tx(ready, (32u << box) * 128u);
+                tma_load_2d(sm.b[i], &maps.b[box], kb * kGBK, r0 + n0, ready);
             }
             __syncwarp();
             ++issued;
         }
+        // drain: the copies land within microseconds (these barriers also count the
+        // decoders, so after an abort they may only complete by the wait's limit)
         for (int kb = max(0, issued - kGBStages); kb < issued; ++kb)
-            mbar_wait_sleep(&sm.b_full[kb % kGBStages], (kb / kGBStages) & 1);
+            mbar_wait_sleep(&sm.kb_ready[kb % kGKbRing], (kb / kGKbRing) & 1);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // One lane runs the loop: one bounded wait per K-block, 2 x 4 MMAs whose
+        // descriptors step by 32 B (2 in 16-byte units) from per-slot bases, one commit.
         const uint32_t idesc = umma_idesc_f16(nmma);
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
-            const int g = kb % kGGroups, i = kb % kGBStages;
-            if (!wait(&sm.a_full[g], (kb / kGGroups) & 1) || !wait(&sm.b_full[i], (kb / kGBStages) & 1)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t b0 = smem_u32(sm.b[i]);
+        if (lane == 0) {
+            // the start-address field holds address >> 4 (14 bits, shared memory < 256 KB)
+            const uint64_t a_desc0 = umma_desc_sw128(smem_u32(sm.a[0][0]));
+            const uint64_t b_desc0 = umma_desc_sw128(smem_u32(sm.b[0]));
+            constexpr uint32_t a_step = sizeof(sm.a[0][0]) >> 4, b_step = sizeof(sm.b[0]) >> 4;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const int g = kb % kGGroups, i = kb % kGBStages;
+                if (!mbar_wait_sleep(&sm.kb_ready[kb % kGKbRing], (kb / kGKbRing) & 1) ||
+                    *(volatile int32_t *)&sm.abort) {
+                    sm.abort = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
 #pragma unroll
-                for (int t = 0; t < kGTiles; ++t) {
-                    const uint32_t a0 = smem_u32(sm.a[g][t]);
+                for (int t = 0; t < kGTiles; ++t)
 #pragma unroll
                     for (int k = 0; k < kGBK / 16; ++k)
-                        umma_f16(tmem_d + t * kGBN, umma_desc_sw128(a0 + 32 * k), umma_desc_sw128(b0 + 32 * k),
-                                 idesc, (kb | k) != 0);
-                }
-                umma_commit(&sm.a_empty[g]);
-                umma_commit(&sm.b_empty[i]);
+                        umma_f16(tmem_d + t * kGBN, a_desc0 + (uint64_t)((g * kGTiles + t) * a_step + 2 * k),
+                                 b_desc0 + (uint64_t)(i * b_step + 2 * k), idesc, (kb | k) != 0);
+                umma_commit(&sm.kb_done[kb % kGKbRing]);
             }
-            __syncwarp();
         }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (lane == 0) umma_commit(ok ? &sm.acc_full : &sm.mma_done);
         __syncwarp();
         if (!ok) mbar_wait_sleep(&sm.mma_done, 0);
@@ -392,7 +400,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
         for (int kb = slot; kb < num_kb; kb += kGGroups) {
             const int i = kb % kGBitsStages;
             if (!wait(&sm.bits_full[i], (kb / kGBitsStages) & 1)) break;
-            if (kb >= kGGroups && !wait(&sm.a_empty[slot], ((kb / kGGroups) - 1) & 1)) break;
+            const int pk = kb - kGGroups;     // the K-block that last used this A slot
+            if (pk >= 0 && !wait(&sm.kb_done[pk % kGKbRing], (pk / kGKbRing) & 1)) break;
             const uint32_t bits_s = smem_u32(sm.bits[i]);
             if (ex.K == 2) decode_tile<2, GATEUP>(bits_s, a_s, tile, wl, lane);
             else if (ex.K == 3) decode_tile<3, GATEUP>(bits_s, a_s, tile, wl, lane);
@@ -400,7 +409,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             fence_proxy_async();      // make the generic-proxy writes visible to the MMA
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&sm.a_full[slot]);
+                mbar_arrive(&sm.kb_ready[kb % kGKbRing]);
                 mbar_arrive(&sm.bits_empty[i]);
             }
         }
