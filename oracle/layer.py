@@ -63,6 +63,19 @@ def rotate(x) -> np.ndarray:
     return out.reshape(x.shape)
 
 
+def rotate_in(x, signs=None) -> np.ndarray:
+    """Input side of a projection: rotate(signs * x) (signs None: rotate(x))."""
+    x = np.asarray(x, dtype=np.float64)
+    return rotate(x if signs is None else x * np.asarray(signs, dtype=np.float64))
+
+
+def rotate_out(v, signs=None) -> np.ndarray:
+    """Output side of a projection in the two-sided transform: signs * rotate(v)
+    (signs None: v unchanged, the input-side-only layer)."""
+    v = np.asarray(v, dtype=np.float64)
+    return v if signs is None else rotate(v) * np.asarray(signs, dtype=np.float64)
+
+
 def dequantize(codes, scales) -> np.ndarray:
     """W[i, j] = s_i * kappa * c[i, j] (fp64); scales are fp16 values."""
     s = np.asarray(scales, dtype=np.float64)
@@ -190,28 +203,63 @@ class ExpertWeights:
         return s[:, None] * KAPPA * codes.astype(np.float64)
 
 
-def expert_forward(weights: ExpertWeights, e: int, x_rot, down_rows=None):
+def expert_forward(weights: ExpertWeights, e: int, x_rot, down_rows=None, signs=None):
     """SwiGLU expert on rotated token rows x_rot [n, D].
 
+    signs: the layer's sign vectors (dict x, gu, h, y) of the two-sided transform, or
+    None (input side only).  Two-sided: g = s_gu * rotate(W_g x'), u likewise,
+    h' = rotate(s_h * h), y = s_y * rotate(W_d h').
     Returns a dict with g, u, h, h_rot (fp64) and y [n, D or len(down_rows)], plus the
-    per-projection tolerance scales bound_g, bound_u, bound_y = |W| . |input|.
+    per-projection tolerance scales bound_g, bound_u, bound_y = |W| . |input| (of the
+    projections before their output rotation).
     """
+    two = signs is not None
     Wg = weights.matrix(e, "gate")
     Wu = weights.matrix(e, "up")
-    g = project(Wg, x_rot)
-    u = project(Wu, x_rot)
+    g_raw = project(Wg, x_rot)
+    u_raw = project(Wu, x_rot)
+    g = rotate_out(g_raw, signs["gu"] if two else None)
+    u = rotate_out(u_raw, signs["gu"] if two else None)
     h = silu(g) * u
-    h_rot = rotate(h)
-    Wd = weights.matrix(e, "down") if down_rows is None else weights.down_rows(e, down_rows)
-    y = project(Wd, h_rot)
-    return dict(g=g, u=u, h=h, h_rot=h_rot, y=y,
+    h_rot = rotate_in(h, signs["h"] if two else None)
+    if down_rows is None:
+        rows = None
+    elif two:
+        # the output rotation mixes 128 consecutive rows: compute whole 128-row chunks
+        chunks = np.unique(np.asarray(down_rows) // HADAMARD_N)
+        rows = (chunks[:, None] * HADAMARD_N + np.arange(HADAMARD_N)[None, :]).reshape(-1)
+    else:
+        rows = np.asarray(down_rows)
+    Wd = weights.matrix(e, "down") if rows is None else weights.down_rows(e, rows)
+    y_raw = project(Wd, h_rot)
+    if two:
+        if rows is None:
+            y = rotate_out(y_raw, signs["y"])
+        else:
+            y_rows = rotate(y_raw) * np.asarray(signs["y"], dtype=np.float64)[rows]
+            pos = {int(r): i for i, r in enumerate(rows)}
+            sel = [pos[int(r)] for r in down_rows]
+            y = y_rows[:, sel]
+    else:
+        y = y_raw
+    return dict(g=g, u=u, h=h, h_rot=h_rot, y=y, two_sided=two, rows=rows, down_rows=down_rows,
                 bound_g=abs_bound(Wg, x_rot), bound_u=abs_bound(Wu, x_rot),
                 bound_y=abs_bound(Wd, h_rot), Wd=Wd)
 
 
+def _rot_abs(v) -> np.ndarray:
+    """Elementwise bound on |rotate(dv)| given |dv| <= v: per 128-chunk, sum / sqrt(128)."""
+    v = np.asarray(v, dtype=np.float64)
+    n = v.shape[-1]
+    chunk = v.reshape(v.shape[:-1] + (n // HADAMARD_N, HADAMARD_N)).sum(-1)
+    return np.repeat(chunk, HADAMARD_N, axis=-1) / np.sqrt(float(HADAMARD_N))
+
+
 def e2e_error_bound(stage, eps_proj: float, w_abs):
     """First-order bound on |out_gpu - out| of one route's contribution, given that each
-    projection meets |dy| <= eps_proj * (|W| . |input|) and h' is rounded to fp16.
+    projection meets |dy| <= eps_proj * (|W| . |input|) (h' rounding included); with
+    the two-sided transform the raw projections' errors are spread by their output
+    rotations (per 128-chunk: sum / sqrt(128)).
 
     stage: the dict of ``expert_forward`` for that route's rows; w_abs: |route weight|.
     Returns the bound for the route's y scaled by its weight.
@@ -219,6 +267,9 @@ def e2e_error_bound(stage, eps_proj: float, w_abs):
     g, u = stage["g"], stage["u"]
     dg = eps_proj * stage["bound_g"]
     du = eps_proj * stage["bound_u"]
+    if stage.get("two_sided"):
+        # errors of the raw projections spread by their output rotation
+        dg, du = _rot_abs(dg), _rot_abs(du)
     # |silu(g+dg)*(u+du) - silu(g)*u| <= |silu'(g)| dg |u| + (|silu(g)| + 1.1 dg) du
     #                                    + 0.25 dg^2 |u|          (|silu''| <= 0.5)
     dh = (np.abs(silu_prime(g)) * dg * np.abs(u)
@@ -227,6 +278,11 @@ def e2e_error_bound(stage, eps_proj: float, w_abs):
     chunk = dh.reshape(dh.shape[:-1] + (n // HADAMARD_N, HADAMARD_N)).sum(-1)
     dh_rot = np.repeat(chunk, HADAMARD_N, axis=-1) / np.sqrt(float(HADAMARD_N))
     dy = np.abs(dh_rot) @ np.abs(stage["Wd"]).T + eps_proj * stage["bound_y"]
+    if stage.get("two_sided"):
+        dy = _rot_abs(dy)
+        if stage.get("down_rows") is not None:
+            pos = {int(r): i for i, r in enumerate(stage["rows"])}
+            dy = dy[:, [pos[int(r)] for r in stage["down_rows"]]]
     return w_abs[:, None] * dy
 
 
@@ -240,15 +296,16 @@ def moe_tokens(layer, x, logits, k: int, token_ids, weights: ExpertWeights = Non
     Returns dict(out [n_tok, D or len(down_rows)], bound [same], topk_ids, topk_w).
     """
     weights = weights or ExpertWeights(layer)
+    signs = getattr(layer, "signs", None)
     ids, w = route_topk(logits, k)
     token_ids = np.asarray(token_ids)
-    x_rot = rotate(np.asarray(x, dtype=np.float64)[token_ids])
+    x_rot = rotate_in(np.asarray(x, dtype=np.float64)[token_ids], signs["x"] if signs is not None else None)
     n_out = layer.D if down_rows is None else len(down_rows)
     out = np.zeros((token_ids.size, n_out))
     bound = np.zeros((token_ids.size, n_out))
     for a, t in enumerate(token_ids):
         for s in range(k):
-            st = expert_forward(weights, int(ids[t, s]), x_rot[a:a + 1], down_rows)
+            st = expert_forward(weights, int(ids[t, s]), x_rot[a:a + 1], down_rows, signs)
             out[a] += w[t, s] * st["y"][0]
             bound[a] += e2e_error_bound(st, eps_proj, np.abs(w[t, s:s + 1]))[0]
     return dict(out=out, bound=bound, topk_ids=ids, topk_w=w)

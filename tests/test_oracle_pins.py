@@ -303,3 +303,61 @@ def test_moe_layer_closed_form_with_constant_streams():
             out += res["topk_w"][t, s] * g.s_down[i].astype(np.float64) * kappa * (-255) * math.sqrt(128) * h0
         np.testing.assert_allclose(res["out"][t], out, rtol=1e-10, atol=1e-14)
         assert np.all(res["bound"][t] > 0)
+
+
+# ----------------------------------------------------------------- two-sided transform
+
+def _dense_rotation(n):
+    """Block-diagonal orthonormal Hadamard of size n from scipy (independent of the
+    oracle's own construction)."""
+    import scipy.linalg
+    H = scipy.linalg.hadamard(128).astype(np.float64) / np.sqrt(128.0)
+    return np.kron(np.eye(n // 128), H)
+
+
+def _two_sided_layer():
+    layer = inputs.small_layer(4242, E=6, D=256, F=256, split={2: 3, 3: 2, 4: 1})
+    return inputs.with_signs(layer, 4243)
+
+
+def test_two_sided_expert_equals_dense_effective_matrices():
+    # g = diag(s_gu) H W_gate H diag(s_x) x and y = diag(s_y) H W_down H diag(s_h) h,
+    # with the rotations as explicit dense matrices.
+    layer = _two_sided_layer()
+    sg = layer.signs
+    w = L.ExpertWeights(layer)
+    rng = np.random.default_rng(4244)
+    x = rng.standard_normal((3, layer.D))
+    HD, HF = _dense_rotation(layer.D), _dense_rotation(layer.F)
+    for e in (0, 3, 5):
+        st = L.expert_forward(w, e, L.rotate_in(x, sg["x"]), signs=sg)
+        Wg_eff = np.diag(sg["gu"].astype(float)) @ HF @ w.matrix(e, "gate") @ HD @ np.diag(sg["x"].astype(float))
+        Wu_eff = np.diag(sg["gu"].astype(float)) @ HF @ w.matrix(e, "up") @ HD @ np.diag(sg["x"].astype(float))
+        np.testing.assert_allclose(st["g"], x @ Wg_eff.T, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(st["u"], x @ Wu_eff.T, rtol=1e-10, atol=1e-12)
+        h = L.silu(x @ Wg_eff.T) * (x @ Wu_eff.T)
+        Wd_eff = np.diag(sg["y"].astype(float)) @ HD @ w.matrix(e, "down") @ HF @ np.diag(sg["h"].astype(float))
+        np.testing.assert_allclose(st["y"], h @ Wd_eff.T, rtol=1e-9, atol=1e-12)
+
+
+def test_two_sided_output_rotation_preserves_chunk_norms():
+    layer = _two_sided_layer()
+    w = L.ExpertWeights(layer)
+    x_rot = L.rotate(np.random.default_rng(7).standard_normal((2, layer.D)))
+    one = L.expert_forward(w, 2, x_rot)
+    two = L.expert_forward(w, 2, x_rot, signs=layer.signs)
+    g1 = one["g"].reshape(2, -1, 128)
+    g2 = two["g"].reshape(2, -1, 128)
+    np.testing.assert_allclose(np.linalg.norm(g2, axis=-1), np.linalg.norm(g1, axis=-1), rtol=1e-12)
+
+
+def test_two_sided_selected_down_rows_match_full_rows():
+    layer = _two_sided_layer()
+    rng = np.random.default_rng(4245)
+    x = rng.standard_normal((2, layer.D))
+    logits = rng.standard_normal((2, layer.E)).astype(np.float32)
+    full = L.moe_tokens(layer, x, logits, 2, [0, 1])
+    rows = np.array([3, 130, 255, 7])
+    part = L.moe_tokens(layer, x, logits, 2, [0, 1], down_rows=rows)
+    np.testing.assert_allclose(part["out"], full["out"][:, rows], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(part["bound"], full["bound"][:, rows], rtol=1e-12, atol=1e-14)

@@ -25,7 +25,7 @@ row-major order, per-width groups with ascending expert ids) are those of the C-
 header; this module only fills such arrays with uniform random words.
 """
 from dataclasses import dataclass, field
-from typing import List
+from typing import Optional, List
 
 import numpy as np
 
@@ -117,6 +117,9 @@ class SyntheticLayer:
     groups: List[WidthGroup] = field(default_factory=list)
     name: str = ""
     seed: int = 0
+    # Layer sign vectors of the two-sided transform (int8, +1/-1), shared by every
+    # expert: x [D], gu [F], h [F], y [D]; None for the input-side-only layer.
+    signs: Optional[dict] = None
 
 
 def width_map(rng: np.random.Generator, E: int, split: dict) -> np.ndarray:
@@ -204,6 +207,19 @@ def moe_sweep_tokens(T: int, seed: int = 1005, layer: SyntheticLayer = None):
     x = random_activations(rng, (T, layer.D), "bf16")
     logits = normal_logits(rng, T, layer.E)
     return dict(layer=layer, x=x, logits=logits, k=TOP_K)
+
+
+def random_signs(rng: np.random.Generator, n: int) -> np.ndarray:
+    """Uniform random +1/-1 (int8) of length n."""
+    return np.where(rng.integers(0, 2, size=n) == 1, 1, -1).astype(np.int8)
+
+
+def with_signs(layer: SyntheticLayer, seed: int) -> SyntheticLayer:
+    """The same layer carrying seeded layer sign vectors (x, gu, h, y)."""
+    rng = np.random.default_rng(seed)
+    layer.signs = dict(x=random_signs(rng, layer.D), gu=random_signs(rng, layer.F),
+                       h=random_signs(rng, layer.F), y=random_signs(rng, layer.D))
+    return layer
 
 
 def small_layer(seed: int, E: int = 12, D: int = 256, F: int = 128, split: dict = None,
