@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 1
+#define TQ_ABI_VERSION 2
 
 typedef enum {
     TQ_OK = 0,
@@ -149,6 +149,13 @@ int hadamard128(const void *x, int x_dtype, int64_t rows, int64_t cols, uint16_t
                 tq_stream stream);
 
 /*
+ * hadamard128_signed -- the input side of the two-sided transform: out = rotate(signs * x)
+ * (signs: device int8 [cols] of +1/-1, 4-byte aligned); otherwise as hadamard128.
+ */
+int hadamard128_signed(const void *x, int x_dtype, int64_t rows, int64_t cols, const int8_t *signs,
+                       uint16_t *out, tq_stream stream);
+
+/*
  * trellis_gemv -- one trellis-coded matrix times a small batch of rotated activations:
  *   y[b][r] = s[r] * 2^-12 * sum_c code[r][c] * x_rot[b][c]
  * (the projection of "How T16 works", items 1, 2 and 4, on decode-sized batches).
@@ -205,6 +212,15 @@ int route_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *counts,
 int route_unpermute(const float *y_perm, const int32_t *inv, const float *topk_w, int T, int k,
                     int D, float *out, tq_stream stream);
 
+/*
+ * route_unpermute_signed -- combine plus the output side of the down projection's
+ * two-sided transform: out[t] = signs_y * rotate(sum_s topk_w[t][s] * y_perm[inv[t*k+s]]),
+ * summed in slot order in fp32 (the rotation is linear, so it is applied once, after the
+ * weighted sum).  D % 128 == 0; signs_y: device int8 [D], 4-byte aligned.
+ */
+int route_unpermute_signed(const float *y_perm, const int32_t *inv, const float *topk_w, int T, int k,
+                           int D, const int8_t *signs_y, float *out, tq_stream stream);
+
 /* One width group of a layer: experts of one K, concatenated in ascending global id. */
 typedef struct {
     int K;                       /* 2, 3 or 4 bits per weight                          */
@@ -218,12 +234,27 @@ typedef struct {
     const uint16_t *s_down;      /* device fp16 [n_experts][D]                         */
 } tq_width_group;
 
-/* A trellis-coded MoE layer: E experts of hidden size D and intermediate size F. */
+/*
+ * A trellis-coded MoE layer: E experts of hidden size D and intermediate size F.
+ * Optional two-sided transform (the exlr8 layout's "128 x 128 Hadamard on both sides"
+ * and layer signs shared by every expert): with the four sign vectors set, every
+ * projection is s_out * rotate(W * rotate(s_in * input)), i.e.
+ *   x' = rotate(sign_x * x)          (the caller: hadamard128_signed)
+ *   g  = sign_gu * rotate(W_gate x'),  u = sign_gu * rotate(W_up x'),  h = silu(g) * u
+ *   h' = rotate(sign_h * h),           y = sign_y * rotate(W_down h')
+ * moe_trellis_gemv / _gemm apply sign_gu and sign_h; their y_perm holds W_down h' before
+ * the output rotation, which route_unpermute_signed applies after the combine.  All four
+ * NULL: the input-side-only layer (x' = rotate(x), h' = rotate(h), y = W_down h').
+ */
 typedef struct {
     int E, D, F;                 /* D % 128 == 0, F % 128 == 0                         */
     int n_groups;                /* 1..3 width groups                                  */
     tq_width_group groups[3];
     const int32_t *expert_slot;  /* device [E]: (group << 16) | index in group, or -1  */
+    const int8_t *sign_x;        /* device [D] +1/-1, 4-byte aligned, or NULL          */
+    const int8_t *sign_gu;       /* device [F]                                         */
+    const int8_t *sign_h;        /* device [F]                                         */
+    const int8_t *sign_y;        /* device [D]                                         */
 } tq_moe_layer;
 
 /*

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     from trellis_quantized_moe_gemv_b200 import api
-    assert api.abi_version() == 1
+    assert api.abi_version() == 2
     for code in range(7):
         assert lib.tq_status_string(code)
     assert b"ALIGNMENT" in lib.tq_status_string(3)
@@ -130,6 +130,19 @@ def test_moe_workspace_and_layer_validation(lib):
     mis = _layer_struct()
     mis.groups[0].gate = 0x10004
     assert lib.moe_trellis_gemv(ctypes.byref(mis), *args, 16, 8, FAKE, FAKE, need, None) == 3
+    # layer sign vectors of the two-sided transform: all four or none, 4-byte aligned
+    part = _layer_struct()
+    part.sign_x = part.sign_gu = 0x10000
+    assert lib.moe_trellis_workspace_size(ctypes.byref(part), 16, 8) == 0
+    assert lib.moe_trellis_gemv(ctypes.byref(part), *args, 16, 8, FAKE, FAKE, need, None) == 1
+    signed = _layer_struct()
+    signed.sign_x = signed.sign_gu = signed.sign_h = signed.sign_y = 0x10000
+    need2 = lib.moe_trellis_workspace_size(ctypes.byref(signed), 16, 8)
+    assert need2 >= need
+    signed.sign_h = 0x10002
+    assert lib.moe_trellis_gemv(ctypes.byref(signed), *args, 16, 8, FAKE, FAKE, need2, None) == 3
+    assert lib.hadamard128_signed(FAKE, 0, 4, 128, None, FAKE, None) == 1
+    assert lib.route_unpermute_signed(FAKE, FAKE, FAKE, 4, 8, 200, FAKE, FAKE, None) == 1
 
 
 def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):

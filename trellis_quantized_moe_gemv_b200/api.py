@@ -37,7 +37,9 @@ class TqWidthGroup(ctypes.Structure):
 class TqMoeLayer(ctypes.Structure):
     _fields_ = [("E", ctypes.c_int), ("D", ctypes.c_int), ("F", ctypes.c_int),
                 ("n_groups", ctypes.c_int), ("groups", TqWidthGroup * 3),
-                ("expert_slot", ctypes.c_void_p)]
+                ("expert_slot", ctypes.c_void_p),
+                ("sign_x", ctypes.c_void_p), ("sign_gu", ctypes.c_void_p),
+                ("sign_h", ctypes.c_void_p), ("sign_y", ctypes.c_void_p)]
 
 
 _lib = None
@@ -57,11 +59,13 @@ SIGNATURES = {
     "tq_profile_collect": ([_VP, _VP, _I], _I),
     "trellis_decode": ([_VP, _I, _I, _I, _VP, _VP], _I),
     "hadamard128": ([_VP, _I, _I64, _I64, _VP, _VP], _I),
+    "hadamard128_signed": ([_VP, _I, _I64, _I64, _VP, _VP, _VP], _I),
     "trellis_gemv_workspace_size": ([_I, _I, _I], _SZ),
     "trellis_gemv": ([_VP, _VP, _I, _I, _I, _VP, _I, _VP, _VP, _SZ, _VP], _I),
     "route_topk": ([_VP, _I, _I, _I, _VP, _VP, _VP], _I),
     "route_permute": ([_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "route_unpermute": ([_VP, _VP, _VP, _I, _I, _I, _VP, _VP], _I),
+    "route_unpermute_signed": ([_VP, _VP, _VP, _I, _I, _I, _VP, _VP, _VP], _I),
     "moe_trellis_workspace_size": ([ctypes.POINTER(TqMoeLayer), _I, _I], _SZ),
     "moe_trellis_gemv": ([ctypes.POINTER(TqMoeLayer), _VP, _VP, _VP, _VP, _VP, _I, _I, _VP, _VP,
                           _SZ, _VP], _I),
@@ -200,6 +204,22 @@ def hadamard128(x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None
     return out
 
 
+def hadamard128_signed(x: torch.Tensor, signs: torch.Tensor, out: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """rotate(signs * x) on every 128-chunk (the input side of the two-sided transform)."""
+    if x.dtype not in TQ_DTYPE:
+        raise TypeError("hadamard128_signed: x must be fp16, bf16 or fp32")
+    _require(x, x.dtype, "x")
+    _require(signs, torch.int8, "signs")
+    rows, cols = (x.shape[0], x.shape[1]) if x.dim() == 2 else (1, x.shape[-1])
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.float16, device=x.device)
+    _require(out, torch.float16, "out")
+    _check(_fn("hadamard128_signed")(_p(x), TQ_DTYPE[x.dtype], rows, cols, _p(signs), _p(out),
+                                     _stream(stream)), "hadamard128_signed")
+    return out
+
+
 def trellis_gemv_workspace_size(rows: int, cols: int, batch: int) -> int:
     return int(_fn("trellis_gemv_workspace_size")(rows, cols, batch))
 
@@ -275,6 +295,23 @@ def route_unpermute(y_perm: torch.Tensor, inv: torch.Tensor, topk_w: torch.Tenso
     return out
 
 
+def route_unpermute_signed(y_perm: torch.Tensor, inv: torch.Tensor, topk_w: torch.Tensor, signs_y: torch.Tensor,
+                           out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Combine, then the down projection's output side: signs_y * rotate(sum_s w * y)."""
+    _require(y_perm, torch.float32, "y_perm")
+    _require(inv, torch.int32, "inv")
+    _require(topk_w, torch.float32, "topk_w")
+    _require(signs_y, torch.int8, "signs_y")
+    T, k = topk_w.shape
+    D = y_perm.shape[1]
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.float32, device=y_perm.device)
+    _require(out, torch.float32, "out")
+    _check(_fn("route_unpermute_signed")(_p(y_perm), _p(inv), _p(topk_w), T, k, D, _p(signs_y), _p(out),
+                                         _stream(stream)), "route_unpermute_signed")
+    return out
+
+
 class DeviceLayer:
     """A trellis-coded MoE layer resident on the GPU, with its C-ABI descriptor.
 
@@ -282,7 +319,7 @@ class DeviceLayer:
     `expert_slot[e] = (group << 16) | index` locates expert e.
     """
 
-    def __init__(self, E: int, D: int, F: int, groups: List[dict], device="cuda"):
+    def __init__(self, E: int, D: int, F: int, groups: List[dict], device="cuda", signs: Optional[dict] = None):
         self.E, self.D, self.F = E, D, F
         self.device = torch.device(device)
         self.groups = []
@@ -315,13 +352,20 @@ class DeviceLayer:
             self.groups.append(t)
         self.expert_slot = torch.from_numpy(slot).to(self.device)
         st.expert_slot = self.expert_slot.data_ptr()
+        # layer sign vectors of the two-sided transform (int8 +1/-1): x, gu, h, y
+        self.signs = None
+        if signs is not None:
+            self.signs = {key: torch.as_tensor(np.asarray(signs[key], dtype=np.int8)).to(self.device).contiguous()
+                          for key in ("x", "gu", "h", "y")}
+            st.sign_x, st.sign_gu = self.signs["x"].data_ptr(), self.signs["gu"].data_ptr()
+            st.sign_h, st.sign_y = self.signs["h"].data_ptr(), self.signs["y"].data_ptr()
         self.struct = st
 
     @staticmethod
     def from_synthetic(layer, device="cuda") -> "DeviceLayer":
         groups = [dict(K=g.K, ids=g.ids, gate=g.gate, up=g.up, down=g.down,
                        s_gate=g.s_gate, s_up=g.s_up, s_down=g.s_down) for g in layer.groups]
-        return DeviceLayer(layer.E, layer.D, layer.F, groups, device)
+        return DeviceLayer(layer.E, layer.D, layer.F, groups, device, getattr(layer, "signs", None))
 
     def compressed_bytes(self, experts) -> int:
         """Bit-stream + scale bytes of the given experts (all three projections)."""
@@ -403,10 +447,16 @@ def moe_layer(layer: DeviceLayer, x: torch.Tensor, logits: torch.Tensor, k: int,
     bufs = bufs or MoeBuffers(layer, T, k)
     route_topk(logits, k, bufs.ids, bufs.w, stream)
     route_permute(bufs.ids, layer.E, bufs.routing, stream)
-    hadamard128(x, bufs.x_rot, stream)
+    if layer.signs is not None:
+        hadamard128_signed(x, layer.signs["x"], bufs.x_rot, stream)
+    else:
+        hadamard128(x, bufs.x_rot, stream)
     use_gemm = path == "gemm" or (path == "auto" and T >= GEMM_MIN_TOKENS
                                   and hasattr(lib(), "moe_trellis_gemm"))
     fn = moe_trellis_gemm if use_gemm else moe_trellis_gemv
     fn(layer, bufs.x_rot, bufs.routing, T, k, bufs.y_perm, bufs.ws, stream)
-    route_unpermute(bufs.y_perm, bufs.routing.inv, bufs.w, bufs.out, stream)
+    if layer.signs is not None:
+        route_unpermute_signed(bufs.y_perm, bufs.routing.inv, bufs.w, layer.signs["y"], bufs.out, stream)
+    else:
+        route_unpermute(bufs.y_perm, bufs.routing.inv, bufs.w, bufs.out, stream)
     return bufs.out

@@ -253,8 +253,9 @@ struct GemmArgs {
     const int32_t *offsets;
     const int32_t *tiles;        // [0] = count, then (expert, first route) pairs
     const float *rowsum;         // [T*k] sum of each route's activation row
-    float *out;                  // gate/up: h [T*k][F]; down: y [T*k][D]
+    float *out;                  // gate/up: h [T*k][F] (raw_gu: g, u [T*k][2][F]); down: y [T*k][D]
     int kdim;                    // D (gate/up) or F (down)
+    int raw_gu;                  // gate/up of the two-sided transform: store g and u, not h
 };
 
 template <bool GATEUP>
@@ -441,7 +442,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
                                 const float sx = args.rowsum[route];
                                 const float g = sg * kKappa * fmaf(16777216.0f, dv, -255.0f * sx);
                                 const float u = su * kKappa * fmaf(16777216.0f, du, -255.0f * sx);
-                                args.out[(size_t)route * L.F + f] = silu_f32(g) * u;
+                                if (args.raw_gu) {
+                                    args.out[(size_t)route * 2 * L.F + f] = g;
+                                    args.out[((size_t)route * 2 + 1) * L.F + f] = u;
+                                } else {
+                                    args.out[(size_t)route * L.F + f] = silu_f32(g) * u;
+                                }
                             }
                         }
                     } else {
@@ -502,6 +508,44 @@ __global__ void __launch_bounds__(256) route_rows_kernel(const T *__restrict__ x
         u.x = *reinterpret_cast<uint32_t *>(&lo);
         u.y = *reinterpret_cast<uint32_t *>(&hi);
         *reinterpret_cast<uint2 *>(dst + (size_t)j * cols + c + 4 * lane) = u;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) rowsum[j] = sum;
+}
+
+// The two-sided transform between the gate/up and down GEMMs, one warp per route row j:
+// g = sign_gu * rotate(g), u likewise (the output side of gate and up), h = silu(g) * u,
+// h' = rotate(sign_h * h) (the input side of down), stored fp16 with its fp32 row sum.
+__global__ void __launch_bounds__(256) swiglu_rows_kernel(const float *__restrict__ gu, int rows, int F,
+                                                          const int8_t *__restrict__ sign_gu,
+                                                          const int8_t *__restrict__ sign_h, __half *__restrict__ dst,
+                                                          float *__restrict__ rowsum) {
+    const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (j >= rows) return;
+    float sum = 0.f;
+    for (int c = 0; c < F; c += 128) {
+        const float4 g4 = load4<float>(gu + (size_t)j * 2 * F + c + 4 * lane);
+        const float4 u4 = load4<float>(gu + ((size_t)j * 2 + 1) * F + c + 4 * lane);
+        float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w}, h[4];
+        fwht128_warp(g, lane);
+        fwht128_warp(u, lane);
+        const char4 so = *reinterpret_cast<const char4 *>(sign_gu + c + 4 * lane);
+        const char4 si = *reinterpret_cast<const char4 *>(sign_h + c + 4 * lane);
+        const float o[4] = {(float)so.x, (float)so.y, (float)so.z, (float)so.w};
+        const float in[4] = {(float)si.x, (float)si.y, (float)si.z, (float)si.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = silu_f32(g[i] * o[i]) * (u[i] * o[i]) * in[i];
+        fwht128_warp(h, lane);
+        __half2 lo = __floats2half2_rn(h[0], h[1]);
+        __half2 hi = __floats2half2_rn(h[2], h[3]);
+        const float2 lf = __half22float2(lo), hf = __half22float2(hi);
+        sum += (lf.x + lf.y) + (hf.x + hf.y);
+        uint2 w;
+        w.x = *reinterpret_cast<uint32_t *>(&lo);
+        w.y = *reinterpret_cast<uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(dst + (size_t)j * F + c + 4 * lane) = w;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
@@ -625,8 +669,9 @@ static int gemm_max_tiles(int T, int k, int E) {
 
 size_t gemm_workspace_bytes(const tq_moe_layer *L, int T, int k) {
     const size_t R = (size_t)T * k;
+    const size_t hcols = L->sign_gu ? 2 : 1;   // two-sided: g and u, else h
     return align256_g(R * L->D * sizeof(__half)) + align256_g(R * sizeof(float)) +
-           align256_g(R * L->F * sizeof(float)) + align256_g(R * L->F * sizeof(__half)) +
+           align256_g(R * hcols * L->F * sizeof(float)) + align256_g(R * L->F * sizeof(__half)) +
            align256_g(R * sizeof(float)) + align256_g((1 + 2 * (size_t)gemm_max_tiles(T, k, L->E)) * sizeof(int32_t));
 }
 
@@ -649,8 +694,9 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     w += align256_g((size_t)R * L->D * sizeof(__half));
     float *sxp = reinterpret_cast<float *>(w);
     w += align256_g((size_t)R * sizeof(float));
-    float *h = reinterpret_cast<float *>(w);
-    w += align256_g((size_t)R * L->F * sizeof(float));
+    const int two = L->sign_gu != nullptr;     // two-sided transform
+    float *h = reinterpret_cast<float *>(w);   // h, or g and u when two-sided
+    w += align256_g((size_t)R * (two ? 2 : 1) * L->F * sizeof(float));
     __half *hr = reinterpret_cast<__half *>(w);
     w += align256_g((size_t)R * L->F * sizeof(__half));
     float *shr = reinterpret_cast<float *>(w);
@@ -683,7 +729,7 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     st = launch_status();
     if (st) return st;
     {
-        GemmArgs a{*L, offsets, tiles, sxp, h, L->D};
+        GemmArgs a{*L, offsets, tiles, sxp, h, L->D, two};
         LaunchScope ls(s, kStageGemmGateUp);
         moe_gemm_kernel<true><<<dim3(L->F / (64 * kGTiles), max_tiles), kGThreads, smem, s>>>(maps_x, a);
     }
@@ -691,12 +737,15 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     if (st) return st;
     {
         LaunchScope ls(s, kStageRotateH);
-        route_rows_kernel<float, true><<<(R * 32 + 255) / 256, 256, 0, s>>>(h, R, L->F, nullptr, 1, R, hr, shr);
+        if (two)
+            swiglu_rows_kernel<<<(R * 32 + 255) / 256, 256, 0, s>>>(h, R, L->F, L->sign_gu, L->sign_h, hr, shr);
+        else
+            route_rows_kernel<float, true><<<(R * 32 + 255) / 256, 256, 0, s>>>(h, R, L->F, nullptr, 1, R, hr, shr);
     }
     st = launch_status();
     if (st) return st;
     {
-        GemmArgs a{*L, offsets, tiles, shr, y_perm, L->F};
+        GemmArgs a{*L, offsets, tiles, shr, y_perm, L->F, 0};
         LaunchScope ls(s, kStageGemmDown);
         moe_gemm_kernel<false><<<dim3(L->D / (kGBM * kGTiles), max_tiles), kGThreads, smem, s>>>(maps_h, a);
     }

@@ -293,9 +293,12 @@ struct RowSrc {
 
 // SwiGLU of the gate/up GEMV's column-split partial sums: h = silu(sum_s g_s) * sum_s u_s
 // from gu[row][s][0][cols] (gate) and gu[row][s][1][cols] (up).
+// sign_gu (optional): the output side of the two-sided transform, applied to g and u
+// before the SwiGLU: g = sign_gu * rotate(g), u likewise.
 struct SwigluSrc {
     const float *gu;
     int cols, splits;
+    const int8_t *sign_gu;
     __device__ __forceinline__ void load(int row, int c, int lane, float (&v)[4]) const {
         const float *p = gu + (size_t)row * splits * 2 * cols + (size_t)c * 128 + 4 * lane;
         float4 g = *reinterpret_cast<const float4 *>(p), u = *reinterpret_cast<const float4 *>(p + cols);
@@ -305,16 +308,26 @@ struct SwigluSrc {
             g.x += g2.x; g.y += g2.y; g.z += g2.z; g.w += g2.w;
             u.x += u2.x; u.y += u2.y; u.z += u2.z; u.w += u2.w;
         }
-        v[0] = silu_f32(g.x) * u.x;
-        v[1] = silu_f32(g.y) * u.y;
-        v[2] = silu_f32(g.z) * u.z;
-        v[3] = silu_f32(g.w) * u.w;
+        float gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w};
+        if (sign_gu) {
+            fwht128_warp(gv, lane);
+            fwht128_warp(uv, lane);
+            const char4 sg = *reinterpret_cast<const char4 *>(sign_gu + c * 128 + 4 * lane);
+            const float s4[4] = {(float)sg.x, (float)sg.y, (float)sg.z, (float)sg.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                gv[i] *= s4[i];
+                uv[i] *= s4[i];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = silu_f32(gv[i]) * uv[i];
     }
 };
 
 template <typename Src, bool ROTATE>
-__global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int cols, uint16_t *__restrict__ xq,
-                                                            int2 *__restrict__ meta) {
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int cols, const int8_t *__restrict__ signs,
+                                                            uint16_t *__restrict__ xq, int2 *__restrict__ meta) {
     __shared__ float s_max[8];
     __shared__ int s_sum[8];
     const int row = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -323,7 +336,13 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int c
     for (int c = warp; c < chunks; c += 8) {
         float v[4];
         src.load(row, c, lane, v);
-        if constexpr (ROTATE) fwht128_warp(v, lane);
+        if constexpr (ROTATE) {
+            if (signs) {   // input side of the two-sided transform: rotate(signs * v)
+                const char4 sg = *reinterpret_cast<const char4 *>(signs + c * 128 + 4 * lane);
+                v[0] *= sg.x; v[1] *= sg.y; v[2] *= sg.z; v[3] *= sg.w;
+            }
+            fwht128_warp(v, lane);
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) m = fmaxf(m, fabsf(v[i]));
     }
@@ -344,7 +363,13 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int c
     for (int c = warp; c < chunks; c += 8) {
         float v[4];
         src.load(row, c, lane, v);
-        if constexpr (ROTATE) fwht128_warp(v, lane);
+        if constexpr (ROTATE) {
+            if (signs) {   // input side of the two-sided transform: rotate(signs * v)
+                const char4 sg = *reinterpret_cast<const char4 *>(signs + c * 128 + 4 * lane);
+                v[0] *= sg.x; v[1] *= sg.y; v[2] *= sg.z; v[3] *= sg.w;
+            }
+            fwht128_warp(v, lane);
+        }
         uint32_t wh[4], wl[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -373,11 +398,11 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int c
 
 template <bool ROTATE, typename Src>
 int launch_quantize_rows(const Src &src, long long rows, int cols, uint16_t *xq, int2 *meta, cudaStream_t s,
-                         int stage) {
+                         int stage, const int8_t *signs = nullptr) {
     if (rows <= 0) return TQ_OK;
     if (rows > 0x7fffffffll) return TQ_ERR_UNSUPPORTED;
     LaunchScope ls(s, stage);
-    quantize_rows_kernel<Src, ROTATE><<<(unsigned)rows, 256, 0, s>>>(src, cols, xq, meta);
+    quantize_rows_kernel<Src, ROTATE><<<(unsigned)rows, 256, 0, s>>>(src, cols, signs, xq, meta);
     return launch_status();
 }
 
@@ -653,6 +678,10 @@ int validate_layer(const tq_moe_layer *L) {
         return TQ_ERR_INVALID_ARG;
     if (L->D > kMaxCols || L->F > kMaxCols) return TQ_ERR_UNSUPPORTED;
     if (L->n_groups < 1 || L->n_groups > 3 || !L->expert_slot) return TQ_ERR_INVALID_ARG;
+    const int n_signs = !!L->sign_x + !!L->sign_gu + !!L->sign_h + !!L->sign_y;
+    if (n_signs != 0 && n_signs != 4) return TQ_ERR_INVALID_ARG;   // all four or none
+    for (const int8_t *sg : {L->sign_x, L->sign_gu, L->sign_h, L->sign_y})
+        if (reinterpret_cast<uintptr_t>(sg) & 3) return TQ_ERR_ALIGNMENT;
     for (int g = 0; g < L->n_groups; ++g) {
         const tq_width_group &G = L->groups[g];
         if (G.K < 2 || G.K > 4 || G.n_experts < 0 || G.n_experts > 0xFFFF) return TQ_ERR_INVALID_ARG;
@@ -720,8 +749,8 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     }
     st = launch_status();
     if (st) return st;
-    st = launch_quantize_rows<true>(SwigluSrc{w.gu, L->F, kGateUpSplits}, routes, L->F, w.hq, w.hmeta, s,
-                                    kStageRotateH);
+    st = launch_quantize_rows<true>(SwigluSrc{w.gu, L->F, kGateUpSplits, L->sign_gu}, routes, L->F, w.hq, w.hmeta, s,
+                                    kStageRotateH, L->sign_h);
     if (st) return st;
     LaunchScope ls(s, kStageGemvDown);
     moe_gemv_items_kernel<false><<<dn_items, kItemThreads, smem, s>>>(*L, w.hq, w.hmeta, offsets, perm, active_ids,

@@ -54,8 +54,11 @@ __device__ __forceinline__ void fwht128_warp(float (&v)[4], int lane) {
     for (int i = 0; i < 4; ++i) v[i] *= kInvSqrt128;
 }
 
+// signs (optional, int8 +1/-1 per column) multiply x before the rotation: the input
+// side of the two-sided transform, x' = rotate(signs * x).
 template <typename T>
 __global__ void __launch_bounds__(256) hadamard128_kernel(const T *__restrict__ x, long long n_chunks,
+                                                          const int8_t *__restrict__ signs, int chunks_per_row,
                                                           __half *__restrict__ out) {
     const long long chunk = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -63,6 +66,11 @@ __global__ void __launch_bounds__(256) hadamard128_kernel(const T *__restrict__ 
     const size_t off = (size_t)chunk * 128 + 4 * lane;
     float4 f = load4<T>(x + off);
     float v[4] = {f.x, f.y, f.z, f.w};
+    if (signs) {
+        const int col = (int)(chunk % chunks_per_row) * 128 + 4 * lane;
+        const char4 sg = *reinterpret_cast<const char4 *>(signs + col);
+        v[0] *= sg.x; v[1] *= sg.y; v[2] *= sg.z; v[3] *= sg.w;
+    }
     fwht128_warp(v, lane);
     __half2 lo = __floats2half2_rn(v[0], v[1]);
     __half2 hi = __floats2half2_rn(v[2], v[3]);
@@ -74,7 +82,7 @@ __global__ void __launch_bounds__(256) hadamard128_kernel(const T *__restrict__ 
 
 // Rotation launcher shared with the MoE path (rotating the SwiGLU activations h).
 int launch_hadamard128(const void *x, int x_dtype, long long rows, long long cols, __half *out,
-                       cudaStream_t s, int stage) {
+                       cudaStream_t s, int stage, const int8_t *signs = nullptr) {
     const long long n_chunks = rows * (cols / 128);
     if (n_chunks == 0) return TQ_OK;
     const int threads = 256;
@@ -83,14 +91,16 @@ int launch_hadamard128(const void *x, int x_dtype, long long rows, long long col
     LaunchScope ls(s, stage);
     switch (x_dtype) {
         case TQ_DTYPE_F16:
-            hadamard128_kernel<__half><<<(unsigned)blocks, threads, 0, s>>>((const __half *)x, n_chunks, out);
+            hadamard128_kernel<__half><<<(unsigned)blocks, threads, 0, s>>>((const __half *)x, n_chunks, signs,
+                                                                            (int)(cols / 128), out);
             break;
         case TQ_DTYPE_BF16:
             hadamard128_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, s>>>(
-                (const __nv_bfloat16 *)x, n_chunks, out);
+                (const __nv_bfloat16 *)x, n_chunks, signs, (int)(cols / 128), out);
             break;
         case TQ_DTYPE_F32:
-            hadamard128_kernel<float><<<(unsigned)blocks, threads, 0, s>>>((const float *)x, n_chunks, out);
+            hadamard128_kernel<float><<<(unsigned)blocks, threads, 0, s>>>((const float *)x, n_chunks, signs,
+                                                                           (int)(cols / 128), out);
             break;
         default:
             return TQ_ERR_INVALID_ARG;
@@ -98,7 +108,68 @@ int launch_hadamard128(const void *x, int x_dtype, long long rows, long long col
     return launch_status();
 }
 
+// Combine with the output side of the two-sided transform of the down projection:
+// out[t] = signs * rotate(sum_s w[t, s] * y_perm[inv[t*k + s]]), summed in slot order (the
+// rotation is linear, so rotating once after the weighted sum equals rotating every
+// route's output).  One warp per (token, 128-chunk).
+__global__ void __launch_bounds__(256) route_unpermute_signed_kernel(
+    const float *__restrict__ y_perm, const int32_t *__restrict__ inv, const float *__restrict__ w, int T, int k,
+    int D, int n_routes, const int8_t *__restrict__ signs, float *__restrict__ out) {
+    const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int chunks = D / 128;
+    if (wid >= (long long)T * chunks) return;
+    const int t = (int)(wid / chunks), c = (int)(wid % chunks);
+    const int col = c * 128 + 4 * lane;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < k; ++s) {
+        const int r = inv[t * k + s];
+        const float ws = w[t * k + s];
+        if (r < 0 || r >= n_routes) {
+            if (lane == 0) raise_flag(1);
+            continue;
+        }
+        const float4 y = *reinterpret_cast<const float4 *>(y_perm + (size_t)r * D + col);
+        v[0] = fmaf(ws, y.x, v[0]);
+        v[1] = fmaf(ws, y.y, v[1]);
+        v[2] = fmaf(ws, y.z, v[2]);
+        v[3] = fmaf(ws, y.w, v[3]);
+    }
+    fwht128_warp(v, lane);
+    const char4 sg = *reinterpret_cast<const char4 *>(signs + col);
+    *reinterpret_cast<float4 *>(out + (size_t)t * D + col) = make_float4(v[0] * sg.x, v[1] * sg.y, v[2] * sg.z, v[3] * sg.w);
+}
+
 }  // namespace tq
+
+TQ_API int route_unpermute_signed(const float *y_perm, const int32_t *inv, const float *topk_w, int T, int k,
+                                  int D, const int8_t *signs_y, float *out, tq_stream stream) {
+    if (T < 0 || k < 1 || D < 128 || D % 128) return TQ_ERR_INVALID_ARG;
+    if (T == 0) return TQ_OK;
+    if (!y_perm || !inv || !topk_w || !out || !signs_y) return TQ_ERR_INVALID_ARG;
+    if (!tq::aligned16(y_perm) || !tq::aligned16(out) || (reinterpret_cast<uintptr_t>(signs_y) & 3))
+        return TQ_ERR_ALIGNMENT;
+    cudaStream_t s = (cudaStream_t)stream;
+    const long long warps = (long long)T * (D / 128);
+    const long long blocks = (warps * 32 + 255) / 256;
+    if (blocks > 0x7fffffffll) return TQ_ERR_UNSUPPORTED;
+    tq::LaunchScope ls(s, tq::kStageUnpermute);
+    tq::route_unpermute_signed_kernel<<<(unsigned)blocks, 256, 0, s>>>(y_perm, inv, topk_w, T, k, D, T * k, signs_y,
+                                                                        out);
+    return tq::launch_status();
+}
+
+TQ_API int hadamard128_signed(const void *x, int x_dtype, int64_t rows, int64_t cols, const int8_t *signs,
+                              uint16_t *out, tq_stream stream) {
+    if (rows < 0 || cols < 0 || cols % 128) return TQ_ERR_INVALID_ARG;
+    if (x_dtype != TQ_DTYPE_F16 && x_dtype != TQ_DTYPE_BF16 && x_dtype != TQ_DTYPE_F32)
+        return TQ_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0) return TQ_OK;
+    if (!x || !out || !signs) return TQ_ERR_INVALID_ARG;
+    if (!tq::aligned16(x) || !tq::aligned16(out) || (reinterpret_cast<uintptr_t>(signs) & 3)) return TQ_ERR_ALIGNMENT;
+    return tq::launch_hadamard128(x, x_dtype, rows, cols, reinterpret_cast<__half *>(out), (cudaStream_t)stream,
+                                  tq::kStageRotateX, signs);
+}
 
 TQ_API int hadamard128(const void *x, int x_dtype, int64_t rows, int64_t cols, uint16_t *out,
                        tq_stream stream) {
