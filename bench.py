@@ -46,6 +46,8 @@ def parse_args():
     p.add_argument("--eager", action="store_true", help="launch every step from the host instead of a CUDA graph")
     p.add_argument("--tokens", type=int, default=None, help="override the workload's token count (profiling runs)")
     p.add_argument("--experts", type=int, default=None, help="override the workload's expert count (profiling runs)")
+    p.add_argument("--two-sided", action="store_true",
+                   help="layers carry the two-sided transform (Hadamard on both sides, layer signs)")
     p.add_argument("--sweep", action="store_true",
                    help="batch sweep of the mixed-width decode layer (T = 1 .. 16384, uniform top-8): "
                         "device time of the GEMV and the GEMM path at every T, one JSON line each")
@@ -176,13 +178,15 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workload
 
-def build_decode_workload(api, inputs, torch, device, rank, n_copies):
+def build_decode_workload(api, inputs, torch, device, rank, n_copies, two_sided=False):
     """Layer copy 0 from the seeded numpy generators (the copy the parity tests check);
     copies 1..3 with the same widths, their bit streams and scales drawn on the device
     from a seeded torch generator; every copy has its own tokens and logits."""
     w0 = inputs.moe_decode_t16(seed=1003 + 100 * rank)
     host_layer = w0["layer"]
     layers, xs, logits = [], [], []
+    if two_sided:
+        inputs.with_signs(host_layer, 8000 + 100 * rank)
     layers.append(api.DeviceLayer.from_synthetic(host_layer, device))
     gen = torch.Generator(device=device)
     for c in range(1, n_copies):
@@ -198,7 +202,12 @@ def build_decode_workload(api, inputs, torch, device, rank, n_copies):
             groups.append(dict(K=g.K, ids=g.ids, gate=rbits(g.gate.shape), up=rbits(g.up.shape),
                                down=rbits(g.down.shape), s_gate=rscale(g.s_gate.shape),
                                s_up=rscale(g.s_up.shape), s_down=rscale(g.s_down.shape)))
-        layers.append(api.DeviceLayer(host_layer.E, host_layer.D, host_layer.F, groups, device))
+        signs = None
+        if two_sided:
+            srng = np.random.default_rng(8000 + 100 * rank + c)
+            signs = {key: inputs.random_signs(srng, n) for key, n in
+                     (("x", host_layer.D), ("gu", host_layer.F), ("h", host_layer.F), ("y", host_layer.D))}
+        layers.append(api.DeviceLayer(host_layer.E, host_layer.D, host_layer.F, groups, device, signs))
     for c in range(n_copies):
         rng = np.random.default_rng(9000 + 100 * rank + c)
         x = w0["x"] if c == 0 else inputs.random_activations(rng, (16, host_layer.D), "bf16")
@@ -225,10 +234,12 @@ def gateup_algorithmic_bytes(layer, counts):
     return total
 
 
-def build_prefill_workload(api, inputs, device, rank, T=8192, E=384):
+def build_prefill_workload(api, inputs, device, rank, T=8192, E=384, two_sided=False):
     """The all-K=3 384-expert layer with 8192 Zipf(1.1)-routed tokens: one step touches
     every expert (1.8 GB of bit streams), far beyond L2, so one layer copy suffices."""
     w0 = inputs.moe_prefill_t8192(seed=1004 + 100 * rank, T=T, E=E)
+    if two_sided:
+        inputs.with_signs(w0["layer"], 8000 + 100 * rank)
     layers = [api.DeviceLayer.from_synthetic(w0["layer"], device)]
     return w0, layers, [(w0["x"], w0["logits"])]
 
@@ -272,10 +283,11 @@ def run_ours(args, rank, world, local_rank):
         if args.tokens or args.experts:
             raise SystemExit("--tokens/--experts apply to the prefill workload")
         NL = args.layers
-        w0, layers, xs = build_decode_workload(api, inputs, torch, device, rank, NL)
+        w0, layers, xs = build_decode_workload(api, inputs, torch, device, rank, NL, args.two_sided)
     else:
         NL = 1
-        w0, layers, xs = build_prefill_workload(api, inputs, device, rank, T=T, E=args.experts or 384)
+        w0, layers, xs = build_prefill_workload(api, inputs, device, rank, T=T, E=args.experts or 384,
+                                                two_sided=args.two_sided)
     E, D, F = layers[0].E, layers[0].D, layers[0].F
     bufs = [api.MoeBuffers(L, T, k) for L in layers]
     x_dev = [torch.from_numpy(x).to(torch.bfloat16).to(device) for x, _ in xs]
@@ -459,6 +471,8 @@ def run_ours(args, rank, world, local_rank):
                   "inputs larger than L2: each step reads all 1.8 GB of bit streams",
             "path": wl["path"], "launch": "eager" if args.eager else "cuda-graph replay per step",
             "parallelism": "replicas" if world > 1 else "single-gpu",
+            "transform": "two-sided (Hadamard on both sides, layer signs)" if args.two_sided
+                         else "input-side Hadamard",
         },
         "roofline": roofline,
         "stage_avg_launch_ms": stage_avg,
