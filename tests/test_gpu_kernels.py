@@ -183,6 +183,44 @@ def test_route_permute_exact(api, T, E, k):
     np.testing.assert_array_equal(r.active_ids.cpu().numpy()[:n_act], active)
 
 
+@pytest.mark.parametrize("T,k,E", [(2048, 8, 384), (2500, 8, 1024), (2051, 8, 7), (40000, 8, 384)])
+def test_route_permute_multi_block_exact(api, T, k, E):
+    # T*k >= 16384 takes the multi-CTA grouping (4096-route blocks, ragged last block);
+    # a few out-of-range ids are dropped (inv = -1) and raise device flag bit 0.
+    rng = np.random.default_rng(T + E)
+    logits = inputs.zipf_gumbel_logits(rng, T, E) if E >= 8 else inputs.normal_logits(rng, T, E)
+    rid, _ = OL.route_topk(logits, min(k, E))
+    if rid.shape[1] < k:
+        rid = np.concatenate([rid, rid[:, :k - rid.shape[1]]], axis=1)
+    bad = rng.choice(rid.size, 5, replace=False)
+    rid_bad = rid.copy().reshape(-1)
+    rid_bad[bad[:3]] = E
+    rid_bad[bad[3:]] = -7
+    rid_bad = rid_bad.reshape(rid.shape)
+    api.device_status(clear=True)
+    r = api.route_permute(torch.from_numpy(rid_bad).cuda(), E)
+    torch.cuda.synchronize()
+    assert api.device_status(clear=True) == 1
+    valid = (rid_bad >= 0) & (rid_bad < E)
+    ref_ids = np.where(valid, rid_bad, 0).reshape(-1)
+    counts = np.bincount(ref_ids[valid.reshape(-1)], minlength=E).astype(np.int32)
+    order = np.argsort(np.where(valid.reshape(-1), ref_ids, E), kind="stable")[:valid.sum()]
+    np.testing.assert_array_equal(r.counts.cpu().numpy(), counts)
+    np.testing.assert_array_equal(r.offsets.cpu().numpy()[1:], np.cumsum(counts))
+    np.testing.assert_array_equal(r.perm.cpu().numpy()[:valid.sum()], order)
+    inv = r.inv.cpu().numpy()
+    assert np.all(inv[~valid.reshape(-1)] == -1)
+    np.testing.assert_array_equal(inv[order], np.arange(order.size))
+    # and, without bad ids, exactly the oracle's grouping
+    r2 = api.route_permute(torch.from_numpy(rid).cuda(), E)
+    c2, o2, p2, i2 = OL.route_permute(rid, E)
+    np.testing.assert_array_equal(r2.perm.cpu().numpy(), p2)
+    np.testing.assert_array_equal(r2.inv.cpu().numpy(), i2)
+    np.testing.assert_array_equal(r2.offsets.cpu().numpy(), o2)
+    n_act = int(r2.n_active.item())
+    np.testing.assert_array_equal(r2.active_ids.cpu().numpy()[:n_act], np.nonzero(c2)[0])
+
+
 @pytest.mark.parametrize("T,k,D", [(1, 8, 4096), (16, 8, 4096), (37, 3, 256)])
 def test_route_unpermute(api, T, k, D):
     rng = np.random.default_rng(T + k + D)

@@ -189,6 +189,188 @@ __global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
     }
 }
 
+// ---------------------------------------------------------------- multi-CTA grouping
+//
+// The same stable grouping for large route counts in four launches, with no workspace:
+// A: each block of kPermBlockRoutes routes counts its experts -> perm[b * E + e];
+// B: one CTA turns those counts into each block's first position per expert
+//    (offsets[e] + routes of e in earlier blocks) -> inv[b * E + e], and writes counts,
+//    offsets and the active-expert list;
+// C: each block reads its starting positions and places its routes exactly as the
+//    single-CTA kernel does (chunks of 1024 in route order, match.any ranks), writing
+//    perm only (inv still holds the starting positions other blocks read);
+// D: inv[perm[j]] = j for the placed routes, -1 for routes with an invalid expert.
+// perm and inv hold T*k >= blocks * E entries whenever T*k >= kPermMultiMin.
+constexpr int kPermBlockRoutes = 4 * kPermThreads;
+constexpr int kPermMultiMin = 16384;
+
+__global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(const int32_t *__restrict__ topk_ids,
+                                                                    int n_routes, int E,
+                                                                    int32_t *__restrict__ block_counts) {
+    extern __shared__ int32_t hist[];
+    const int tid = threadIdx.x;
+    for (int e = tid; e < E; e += kPermThreads) hist[e] = 0;
+    __syncthreads();
+    const int r0 = blockIdx.x * kPermBlockRoutes, r1 = min(n_routes, r0 + kPermBlockRoutes);
+    bool bad = false;
+    for (int i = r0 + tid; i < r1; i += kPermThreads) {
+        const int e = topk_ids[i];
+        if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+        else bad = true;
+    }
+    if (bad) raise_flag(1);
+    __syncthreads();
+    for (int e = tid; e < E; e += kPermThreads) block_counts[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(kPermThreads) permute_scan_kernel(const int32_t *__restrict__ block_counts,
+                                                                    int n_blocks, int E,
+                                                                    int32_t *__restrict__ block_start,
+                                                                    int32_t *__restrict__ counts,
+                                                                    int32_t *__restrict__ offsets,
+                                                                    int32_t *__restrict__ active_ids,
+                                                                    int32_t *__restrict__ n_active) {
+    __shared__ int32_t warp_sum[kPermWarps], warp_sum_a[kPermWarps];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int c = 0;
+    if (tid < E)
+        for (int b = 0; b < n_blocks; ++b) c += block_counts[(size_t)b * E + tid];
+    const int a = c > 0 ? 1 : 0;
+    int incl = c, incl_a = a;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int t1 = __shfl_up_sync(0xffffffffu, incl, off);
+        const int t2 = __shfl_up_sync(0xffffffffu, incl_a, off);
+        if (lane >= off) {
+            incl += t1;
+            incl_a += t2;
+        }
+    }
+    if (lane == 31) {
+        warp_sum[warp] = incl;
+        warp_sum_a[warp] = incl_a;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int sm = warp_sum[lane], sa = warp_sum_a[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int t1 = __shfl_up_sync(0xffffffffu, sm, off);
+            const int t2 = __shfl_up_sync(0xffffffffu, sa, off);
+            if (lane >= off) {
+                sm += t1;
+                sa += t2;
+            }
+        }
+        warp_sum[lane] = sm;
+        warp_sum_a[lane] = sa;
+    }
+    __syncthreads();
+    if (tid < E) {
+        const int ex = (warp > 0 ? warp_sum[warp - 1] : 0) + incl - c;
+        const int ex_a = (warp > 0 ? warp_sum_a[warp - 1] : 0) + incl_a - a;
+        offsets[tid] = ex;
+        counts[tid] = c;
+        if (c > 0) active_ids[ex_a] = tid;
+        if (tid == E - 1) {
+            offsets[E] = ex + c;
+            *n_active = ex_a + a;
+        }
+        // each block's first position for this expert, in block order
+        int run = ex;
+        for (int b = 0; b < n_blocks; ++b) {
+            const int v = block_counts[(size_t)b * E + tid];
+            block_start[(size_t)b * E + tid] = run;
+            run += v;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int32_t *__restrict__ topk_ids,
+                                                                       int n_routes, int E,
+                                                                       const int32_t *__restrict__ block_start,
+                                                                       int32_t *__restrict__ perm) {
+    extern __shared__ int32_t smem[];
+    int32_t *cursor = smem;                 // [E] next position of each expert
+    int32_t *total = cursor + E;            // [E] routes of the current chunk
+    int32_t *wcnt = total + E;              // [kPermWarps][E] per-warp counts of a chunk
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < E; e += kPermThreads) cursor[e] = block_start[(size_t)blockIdx.x * E + e];
+    for (int x = tid; x < kPermWarps * E; x += kPermThreads) wcnt[x] = 0;
+    __syncthreads();
+    const unsigned lt_mask = (1u << lane) - 1u;
+    const int r0 = blockIdx.x * kPermBlockRoutes, r1 = min(n_routes, r0 + kPermBlockRoutes);
+    for (int chunk = r0; chunk < r1; chunk += kPermThreads) {
+        const int i = chunk + tid;
+        const int e = i < r1 ? topk_ids[i] : -1;
+        const bool valid = e >= 0 && e < E;
+        const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+        const int rank = __popc(peers & lt_mask);
+        const bool leader = lane == 31 - __clz(peers);
+        if (valid && leader) wcnt[warp * E + e] = __popc(peers);
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += kPermThreads) {
+            int run = 0;
+            for (int w = 0; w < kPermWarps; ++w) {
+                const int v = wcnt[w * E + ee];
+                wcnt[w * E + ee] = run;
+                run += v;
+            }
+            total[ee] = run;
+        }
+        __syncthreads();
+        if (valid) perm[cursor[e] + wcnt[warp * E + e] + rank] = i;
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += kPermThreads) cursor[ee] += total[ee];
+        for (int x = tid; x < kPermWarps * E; x += kPermThreads) wcnt[x] = 0;
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(256) permute_inverse_kernel(const int32_t *__restrict__ topk_ids, int n_routes,
+                                                              int E, const int32_t *__restrict__ offsets,
+                                                              const int32_t *__restrict__ perm,
+                                                              int32_t *__restrict__ inv) {
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= n_routes) return;
+    if (j < offsets[E]) inv[perm[j]] = j;
+    const int e = topk_ids[j];
+    if (e < 0 || e >= E) inv[j] = -1;
+}
+
+static int route_permute_multi(const int32_t *topk_ids, int R, int E, int32_t *counts, int32_t *offsets,
+                               int32_t *perm, int32_t *inv, int32_t *active_ids, int32_t *n_active,
+                               cudaStream_t s) {
+    static bool configured = false;
+    if (!configured) {
+        if (cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(sizeof(int32_t) * (2 + kPermWarps) * kPermMaxE)) != cudaSuccess)
+            return TQ_ERR_CUDA;
+        configured = true;
+    }
+    const int n_blocks = (R + kPermBlockRoutes - 1) / kPermBlockRoutes;
+    {
+        LaunchScope ls(s, kStagePermute);
+        permute_hist_kernel<<<n_blocks, kPermThreads, sizeof(int32_t) * E, s>>>(topk_ids, R, E, perm);
+    }
+    int st = launch_status();
+    if (st) return st;
+    {
+        LaunchScope ls(s, kStagePermute);
+        permute_scan_kernel<<<1, kPermThreads, 0, s>>>(perm, n_blocks, E, inv, counts, offsets, active_ids, n_active);
+    }
+    if ((st = launch_status())) return st;
+    {
+        LaunchScope ls(s, kStagePermute);
+        permute_scatter_kernel<<<n_blocks, kPermThreads, sizeof(int32_t) * (2 + kPermWarps) * E, s>>>(topk_ids, R, E,
+                                                                                                  inv, perm);
+    }
+    if ((st = launch_status())) return st;
+    LaunchScope ls(s, kStagePermute);
+    permute_inverse_kernel<<<(R + 255) / 256, 256, 0, s>>>(topk_ids, R, E, offsets, perm, inv);
+    return launch_status();
+}
+
 // out[t][d] = sum_s w[t][s] * y_perm[inv[t*k+s]][d], slot order, float4 per thread.
 __global__ void __launch_bounds__(256) route_unpermute_kernel(const float *__restrict__ y_perm,
                                                               const int32_t *__restrict__ inv,
@@ -248,6 +430,8 @@ TQ_API int route_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *
     if (!counts || !offsets || !active_ids || !n_active) return TQ_ERR_INVALID_ARG;
     if (T > 0 && (!topk_ids || !perm || !inv)) return TQ_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
+    if ((long long)T * k >= kPermMultiMin)
+        return route_permute_multi(topk_ids, T * k, E, counts, offsets, perm, inv, active_ids, n_active, s);
     const size_t smem = permute_smem_bytes(E);
     static bool configured = false;
     if (!configured) {
