@@ -221,6 +221,30 @@ int route_unpermute(const float *y_perm, const int32_t *inv, const float *topk_w
 int route_unpermute_signed(const float *y_perm, const int32_t *inv, const float *topk_w, int T, int k,
                            int D, const int8_t *signs_y, float *out, tq_stream stream);
 
+/*
+ * trellis_encode -- T16 bit streams for a target matrix by a tail-biting Viterbi search
+ * ("How T16 works": a QTIP-style bitshift trellis found by a Viterbi search, item 1's
+ * codebook, item 2's column-major tile positions, item 4: a quantizer minimising squared
+ * error).  For every 16x16 tile it minimises sum_p (tau_p - 4 c_p)^2, tau_p =
+ * rint(4 * target_p) clamped to [-1276, 1276] (quarter code units), c_p = t - 255 the
+ * centred code of window p, over tail-biting streams of 256*K bits; the search is one
+ * free pass and, unless its best path already closes, two passes closed on the closure
+ * bits of that path's last and first windows (the cheaper wins; ties to the first, to
+ * the smaller dropped bits, to the smaller final window), so the result is deterministic.
+ *   target : device fp32 [rows][cols], row-major, in code units (the caller divides the
+ *            weights by scale * 2^-12); 4-byte aligned.
+ *   bits   : device [rows/16][cols/16][8K] uint32, the layout trellis_decode and the
+ *            MoE kernels read.
+ *   tile_cost : device uint32 [rows/16][cols/16], each tile's objective, or NULL.
+ *   ws     : device workspace of trellis_encode_workspace_size(K, rows, cols) bytes
+ *            (255 rows of 2^(16-K) backpointer bytes per resident CTA), 16-byte aligned.
+ * rows, cols multiples of 16; K in 2..4.  Integer arithmetic throughout.  Returns
+ * TQ_ERR_INVALID_ARG / TQ_ERR_ALIGNMENT / TQ_ERR_WORKSPACE before launching anything.
+ */
+size_t trellis_encode_workspace_size(int K, int rows, int cols);
+int trellis_encode(const float *target, int K, int rows, int cols, uint32_t *bits,
+                   uint32_t *tile_cost, void *ws, size_t ws_bytes, tq_stream stream);
+
 /* One width group of a layer: experts of one K, concatenated in ascending global id. */
 typedef struct {
     int K;                       /* 2, 3 or 4 bits per weight                          */

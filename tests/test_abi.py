@@ -35,7 +35,7 @@ def test_header_declares_the_boundary():
     for required in ("trellis_decode", "hadamard128", "trellis_gemv", "route_topk", "route_permute",
                      "route_unpermute", "moe_trellis_gemv", "moe_trellis_gemm",
                      "moe_trellis_workspace_size", "tq_status_string", "tq_abi_version",
-                     "tq_device_status"):
+                     "tq_device_status", "trellis_encode", "trellis_encode_workspace_size"):
         assert required in names
 
 
@@ -151,3 +151,19 @@ def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(api.TQError):
         api.lib()
+
+
+def test_encode_validation(lib):
+    # workspace: 255 backpointer rows of 2^(16-K) bytes per resident CTA (one per tile here)
+    assert lib.trellis_encode_workspace_size(2, 32, 32) == 4 * 255 * (1 << 14)
+    assert lib.trellis_encode_workspace_size(4, 16, 16) == 255 * (1 << 12)
+    assert lib.trellis_encode_workspace_size(5, 16, 16) == 0
+    assert lib.trellis_encode_workspace_size(2, 20, 16) == 0
+    assert lib.trellis_encode_workspace_size(3, 0, 16) == 0
+    need = lib.trellis_encode_workspace_size(3, 32, 32)
+    assert lib.trellis_encode(FAKE, 5, 32, 32, FAKE, FAKE, FAKE, need, None) == 1
+    assert lib.trellis_encode(FAKE, 3, 30, 32, FAKE, FAKE, FAKE, need, None) == 1
+    assert lib.trellis_encode(FAKE, 3, 32, 32, FAKE, FAKE, FAKE, need - 1, None) == 4
+    assert lib.trellis_encode(FAKE, 3, 32, 32, FAKE, None, MISALIGNED, need, None) == 3
+    assert lib.trellis_encode(None, 3, 32, 32, FAKE, None, FAKE, need, None) == 1
+    assert lib.trellis_encode(None, 3, 0, 32, None, None, None, 0, None) == 0   # no tiles: no-op

@@ -58,6 +58,8 @@ SIGNATURES = {
     "tq_profile_disable": ([], _I),
     "tq_profile_collect": ([_VP, _VP, _I], _I),
     "trellis_decode": ([_VP, _I, _I, _I, _VP, _VP], _I),
+    "trellis_encode_workspace_size": ([_I, _I, _I], _SZ),
+    "trellis_encode": ([_VP, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP], _I),
     "hadamard128": ([_VP, _I, _I64, _I64, _VP, _VP], _I),
     "hadamard128_signed": ([_VP, _I, _I64, _I64, _VP, _VP, _VP], _I),
     "trellis_gemv_workspace_size": ([_I, _I, _I], _SZ),
@@ -144,7 +146,7 @@ def device_status(clear: bool = False) -> int:
 
 STAGES = ("route_topk", "route_permute", "rotate_x", "gemv_gateup", "rotate_h", "gemv_down",
           "route_unpermute", "trellis_decode", "trellis_gemv", "gemm_gateup", "gemm_down", "gemm_prep",
-          "gemv_quant")
+          "gemv_quant", "trellis_encode")
 
 
 def launch_count() -> int:
@@ -189,6 +191,28 @@ def trellis_decode(bits: torch.Tensor, K: int, rows: int, cols: int,
     _require(out, torch.float16, "out")
     _check(_fn("trellis_decode")(_p(bits), K, rows, cols, _p(out), _stream(stream)), "trellis_decode")
     return out
+
+
+def trellis_encode(target: torch.Tensor, K: int, bits: Optional[torch.Tensor] = None,
+                   cost: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                   stream=None):
+    """T16 bit streams [R/16][C/16][8K] (int32 words) for fp32 targets [R][C] in code units,
+    and each tile's squared error in quarter code units [R/16][C/16] (int32 holding uint32)."""
+    _require(target, torch.float32, "target")
+    rows, cols = target.shape
+    tiles = (rows // 16, cols // 16)
+    if bits is None:
+        bits = torch.empty(tiles + (8 * K,), dtype=torch.int32, device=target.device)
+    if cost is None:
+        cost = torch.empty(tiles, dtype=torch.int32, device=target.device)
+    _require(bits, torch.int32, "bits")
+    _require(cost, torch.int32, "cost")
+    if ws is None:
+        need = _fn("trellis_encode_workspace_size")(K, rows, cols)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=target.device)
+    _check(_fn("trellis_encode")(_p(target), K, rows, cols, _p(bits), _p(cost), _p(ws), ws.numel(),
+                                 _stream(stream)), "trellis_encode")
+    return bits, cost
 
 
 def hadamard128(x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

@@ -7,3 +7,4 @@
 #include "tq_gemv.cu"
 #include "tq_gemm.cu"
 #include "tq_noalloc.cu"
+#include "tq_encode.cu"
