@@ -83,21 +83,38 @@ __device__ void enc_pass(EncSmem<K> &sm, int b, uint8_t *__restrict__ bp, uint32
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const int g = g0 + h;
-                    uint32_t bc = 0, bd = 0;
+                    uint32_t c[S::G];
 #pragma unroll
-                    for (int d = 0; d < S::G; ++d) {
+                    for (int d = 0; d < S::G; d += 4) {   // the group's path costs
                         const uint32_t s = s0 + g * S::G + d;
-                        uint32_t base;
-                        if (p == 0) base = (b < 0 || (int)(s & S::kMask) == b) ? 0u : kEncBig;
-                        else base = prev[m0 + g * S::G + d];
-                        const uint32_t c = base + enc_dist(s, tq);
-                        if (d == 0 || c < bc) {
-                            bc = c;
-                            bd = d;
+                        uint4 base4;
+                        if (p == 0) {   // start: free, or window 0's low bits equal to b
+                            base4.x = (b < 0 || ((s + 0) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
+                            base4.y = (b < 0 || ((s + 1) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
+                            base4.z = (b < 0 || ((s + 2) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
+                            base4.w = (b < 0 || ((s + 3) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
+                        } else {
+                            base4 = *reinterpret_cast<const uint4 *>(prev + m0 + g * S::G + d);
                         }
+                        c[d] = base4.x + enc_dist(s, tq);
+                        c[d + 1] = base4.y + enc_dist(s + 1, tq);
+                        c[d + 2] = base4.z + enc_dist(s + 2, tq);
+                        c[d + 3] = base4.w + enc_dist(s + 3, tq);
                     }
-                    gb[h] = bc;
-                    ga |= bd << (8 * h);
+                    // pairwise minimum, the left (smaller d) kept on a tie
+                    uint32_t a[S::G];
+#pragma unroll
+                    for (int d = 0; d < S::G; ++d) a[d] = d;
+#pragma unroll
+                    for (int w = 1; w < S::G; w <<= 1)
+#pragma unroll
+                        for (int d = 0; d < S::G; d += 2 * w)
+                            if (c[d + w] < c[d]) {
+                                c[d] = c[d + w];
+                                a[d] = a[d + w];
+                            }
+                    gb[h] = c[0];
+                    ga |= a[0] << (8 * h);
                 }
                 *reinterpret_cast<uint4 *>(next + gm + g0) = make_uint4(gb[0], gb[1], gb[2], gb[3]);
                 *reinterpret_cast<uint32_t *>(row + g0) = ga;
