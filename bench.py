@@ -48,6 +48,8 @@ def parse_args():
     p.add_argument("--experts", type=int, default=None, help="override the workload's expert count (profiling runs)")
     p.add_argument("--two-sided", action="store_true",
                    help="layers carry the two-sided transform (Hadamard on both sides, layer signs)")
+    p.add_argument("--encode", action="store_true",
+                   help="time trellis_encode (T16 tail-biting Viterbi) on 1024x4096 Gaussian targets, K = 2, 3, 4")
     p.add_argument("--sweep", action="store_true",
                    help="batch sweep of the mixed-width decode layer (T = 1 .. 16384, uniform top-8): "
                         "device time of the GEMV and the GEMM path at every T, one JSON line each")
@@ -628,6 +630,53 @@ def run_sweep(args, local_rank):
                       "library_switch_tokens": api.GEMM_MIN_TOKENS}), flush=True)
 
 
+def run_encode(args, local_rank):
+    """trellis_encode on a 1024x4096 target of N(0, 100^2) code units per width: device time
+    (CUDA events, after a warm-up call), normalised squared error of the decoded codes
+    against the Gaussian rate-distortion bound 2^(-2K), the least-squares gain that maps
+    the codes back onto the targets, and the oracle's time for one tile on the host."""
+    import torch
+    import numpy as np
+    from trellis_quantized_moe_gemv_b200 import api
+    from trellis_quantized_moe_gemv_b200 import build as tqbuild
+    torch.cuda.set_device(local_rank)
+    tqbuild.build()
+    api.lib()
+    rows, cols, sigma = 1024, 4096, 100.0
+    for K in (2, 3, 4):
+        g = torch.Generator(device="cuda")
+        g.manual_seed(2000 + K)
+        x = torch.randn((rows, cols), generator=g, device="cuda") * sigma
+        ws = torch.empty(api._fn("trellis_encode_workspace_size")(K, rows, cols), dtype=torch.uint8, device="cuda")
+        for _ in range(args.warmup):
+            api.trellis_encode(x[:64], K, ws=ws)
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        bits, cost = api.trellis_encode(x, K, ws=ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        codes = api.trellis_decode(bits, K, rows, cols).float()
+        nmse = ((x - codes) ** 2).mean().item() / sigma ** 2
+        gain = ((x * codes).sum() / (codes * codes).sum()).item()
+        tile = x[:16, :16].cpu().numpy()
+        from oracle import encode as OE
+        OE.code_table()
+        t0 = time.time()
+        OE.encode_tile(tile, K)
+        cpu_s = time.time() - t0
+        print(json.dumps({
+            "metric": "trellis_encode weights/s", "value": rows * cols / (ms * 1e-3), "unit": "weights/s",
+            "n_gpus": 1, "ms": ms, "higher_is_better": True, "dtype": "int32", "data": "synthetic",
+            "config": {"workload": "encode_gaussian_%dx%d_K%d" % (rows, cols, K), "K": K,
+                       "targets": "N(0, %g^2) code units" % sigma, "tiles": rows * cols // 256},
+            "nmse": nmse, "rate_distortion_bound": 2.0 ** (-2 * K), "gain": gain,
+            "cpu_baseline": {"value": 256 / cpu_s, "unit": "weights/s", "cores": 1, "kind": "oracle",
+                             "sample": "one 16x16 tile"}}), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local_rank = dist_env()
@@ -638,7 +687,10 @@ def main():
             args.steps = 16
         else:
             args.steps = 500 if args.workload == "moe_decode_t16" else 50
-    if args.sweep:
+    if args.encode:
+        if rank == 0:
+            run_encode(args, local_rank)
+    elif args.sweep:
         if rank == 0:
             run_sweep(args, local_rank)
     elif args.impl == "reference":

@@ -19,10 +19,10 @@
 //
 // One CTA of 1024 threads per tile (persistent over tiles).  The predecessors of window
 // s are the 2^K windows (m << K) | d with m = s & (2^(16-K) - 1), and they are
-// consecutive, so a step is: every thread forms the path costs of its 64 consecutive
-// windows from best[m] (shared memory, double-buffered) plus (tau_p - 4 c(s))^2, and
-// reduces them group by group into the next best[] and the backpointers (the winning d
-// of every m, one byte, in the CTA's global workspace rows).  The traceback walks the
+// consecutive, so a step is: for each group of 2^K consecutive windows, a thread forms
+// their path costs from best[m] (shared memory, double-buffered) plus
+// (tau_p - 4 c(s))^2 and reduces them into the next best[] and the backpointers (the
+// winning d of every m, one byte, in the CTA's global workspace rows).  The traceback walks the
 // backpointer rows from the chosen final window; the stream bits are assembled with warp
 // ballots.  Integer arithmetic throughout, so the result is exactly the oracle's.
 #include "tq_common.cuh"
@@ -62,72 +62,63 @@ __device__ __forceinline__ uint32_t enc_dist(uint32_t s, int tq) {
 
 // One pass over the tile's positions.  b < 0: free start and end; else closed on b.
 // Writes the backpointer rows bp[p][m] (p = 0..254) and returns the best allowed final
-// window and its cost.
+// window and its cost.  Thread t handles the groups (2^K consecutive windows with the
+// same high bits) t, t + 1024, t + 2048, ...: a warp reads 32 consecutive groups'
+// minima from best[] and writes 32 consecutive results, free of bank conflicts.
 template <int K>
 __device__ void enc_pass(EncSmem<K> &sm, int b, uint8_t *__restrict__ bp, uint32_t &out_cost, int &out_last) {
     using S = EncShape<K>;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const uint32_t s0 = (uint32_t)tid * kEncPer;
     unsigned long long key = ~0ull;
     for (int p = 0; p < kEncPos; ++p) {
         const int tq = sm.tau[p] + 1020;
         const uint32_t *prev = sm.best[(p + 1) & 1];
         uint32_t *next = sm.best[p & 1];
-        const uint32_t m0 = s0 & S::kMask;
-        if (p < kEncPos - 1) {
-            const uint32_t gm = s0 / S::G;   // first group of this thread
-            uint8_t *row = bp + (size_t)p * S::M + gm;
+        uint8_t *row = bp + (size_t)p * S::M;
 #pragma unroll 1
-            for (int g0 = 0; g0 < S::kGroups; g0 += 4) {   // four groups at a time
-                uint32_t gb[4], ga = 0;
+        for (int j = 0; j < S::kGroups; ++j) {
+            const uint32_t gi = (uint32_t)j * kEncThreads + tid;   // group: windows gi*G + d
+            const uint32_t s = gi * S::G;
+            const uint32_t m0 = s & S::kMask;
+            uint32_t c[S::G];
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int g = g0 + h;
-                    uint32_t c[S::G];
-#pragma unroll
-                    for (int d = 0; d < S::G; d += 4) {   // the group's path costs
-                        const uint32_t s = s0 + g * S::G + d;
-                        uint4 base4;
-                        if (p == 0) {   // start: free, or window 0's low bits equal to b
-                            base4.x = (b < 0 || ((s + 0) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
-                            base4.y = (b < 0 || ((s + 1) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
-                            base4.z = (b < 0 || ((s + 2) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
-                            base4.w = (b < 0 || ((s + 3) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
-                        } else {
-                            base4 = *reinterpret_cast<const uint4 *>(prev + m0 + g * S::G + d);
-                        }
-                        c[d] = base4.x + enc_dist(s, tq);
-                        c[d + 1] = base4.y + enc_dist(s + 1, tq);
-                        c[d + 2] = base4.z + enc_dist(s + 2, tq);
-                        c[d + 3] = base4.w + enc_dist(s + 3, tq);
-                    }
-                    // pairwise minimum, the left (smaller d) kept on a tie
-                    uint32_t a[S::G];
-#pragma unroll
-                    for (int d = 0; d < S::G; ++d) a[d] = d;
-#pragma unroll
-                    for (int w = 1; w < S::G; w <<= 1)
-#pragma unroll
-                        for (int d = 0; d < S::G; d += 2 * w)
-                            if (c[d + w] < c[d]) {
-                                c[d] = c[d + w];
-                                a[d] = a[d + w];
-                            }
-                    gb[h] = c[0];
-                    ga |= a[0] << (8 * h);
+            for (int d = 0; d < S::G; d += 4) {
+                uint4 base4;
+                if (p == 0) {   // start: free, or window 0's low bits equal to b
+                    base4.x = (b < 0 || ((s + d + 0) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
+                    base4.y = (b < 0 || ((s + d + 1) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
+                    base4.z = (b < 0 || ((s + d + 2) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
+                    base4.w = (b < 0 || ((s + d + 3) & S::kMask) == (uint32_t)b) ? 0u : kEncBig;
+                } else {
+                    base4 = *reinterpret_cast<const uint4 *>(prev + m0 + d);
                 }
-                *reinterpret_cast<uint4 *>(next + gm + g0) = make_uint4(gb[0], gb[1], gb[2], gb[3]);
-                *reinterpret_cast<uint32_t *>(row + g0) = ga;
+                c[d] = base4.x + enc_dist(s + d, tq);
+                c[d + 1] = base4.y + enc_dist(s + d + 1, tq);
+                c[d + 2] = base4.z + enc_dist(s + d + 2, tq);
+                c[d + 3] = base4.w + enc_dist(s + d + 3, tq);
             }
-        } else {
-#pragma unroll 4
-            for (int i = 0; i < kEncPer; ++i) {
-                const uint32_t s = s0 + i;
-                if (b >= 0 && (int)(s >> K) != b) continue;
-                const uint32_t base = prev[m0 + i];
-                const uint32_t c = base + enc_dist(s, tq);
-                const unsigned long long k = ((unsigned long long)c << 16) | s;
-                key = k < key ? k : key;
+            if (p < kEncPos - 1) {
+                // pairwise minimum, the left (smaller d) kept on a tie
+                uint32_t a[S::G];
+#pragma unroll
+                for (int d = 0; d < S::G; ++d) a[d] = d;
+#pragma unroll
+                for (int w = 1; w < S::G; w <<= 1)
+#pragma unroll
+                    for (int d = 0; d < S::G; d += 2 * w)
+                        if (c[d + w] < c[d]) {
+                            c[d] = c[d + w];
+                            a[d] = a[d + w];
+                        }
+                next[gi] = c[0];
+                row[gi] = (uint8_t)a[0];
+            } else {
+#pragma unroll
+                for (int d = 0; d < S::G; ++d) {
+                    if (b >= 0 && (int)((s + d) >> K) != b) continue;
+                    const unsigned long long k = ((unsigned long long)c[d] << 16) | (s + d);
+                    key = k < key ? k : key;
+                }
             }
         }
         __syncthreads();
