@@ -71,3 +71,25 @@ def test_encode_rejects_bad_arguments(api):
         api.trellis_encode(x, 5)
     with pytest.raises(api.TQError, match="WORKSPACE"):
         api.trellis_encode(x, 2, ws=torch.empty(16, dtype=torch.uint8, device="cuda"))
+
+
+def test_encode_full_projection_sampled_tiles(api):
+    # the benchmark's size: one 1024x4096 projection (16,384 tiles) at K = 2; sampled tiles
+    # are re-encoded by the oracle one by one, and every tile's stream must decode to a
+    # cost equal to the one the kernel reports
+    K, rows, cols = 2, 1024, 4096
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2002)
+    x = torch.randn((rows, cols), generator=g, device="cuda") * 100.0
+    bits, cost = api.trellis_encode(x, K)
+    codes = api.trellis_decode(bits, K, rows, cols).double()       # exact integer sums in fp64
+    tau = torch.clamp(torch.round(4.0 * x), -1276, 1276).double()
+    err = ((tau - 4.0 * codes) ** 2).reshape(rows // 16, 16, cols // 16, 16).sum(dim=(1, 3))
+    np.testing.assert_array_equal(err.cpu().numpy().astype(np.int64),
+                                  cost.cpu().numpy().view(np.uint32).astype(np.int64))
+    xs = x.cpu().numpy()
+    got = bits.cpu().numpy().view(np.uint32)
+    for t in (0, 5000, 16383):
+        i, j = divmod(t, cols // 16)
+        words, c, _ = OE.encode_tile(xs[16 * i:16 * i + 16, 16 * j:16 * j + 16], K)
+        np.testing.assert_array_equal(got[i, j], words)
