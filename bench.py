@@ -419,17 +419,18 @@ def run_ours(args, rank, world, local_rank):
                     "peak_source": peak_src + " (dense bf16 GEMM, sustained; fp16 dense rate is the same)",
                     "flops_per_launch": unit_work, "avg_launch_ms": g_avg_ms, "traffic": traffic}
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: api.MoeGraph, one per
+    # layer copy, replays the pinned-host -> device copies of x and the logits, the layer
+    # and the device -> pinned-host copy of the output as one graph launch
     pin_x = [torch.from_numpy(x).to(torch.bfloat16).pin_memory() for x, _ in xs]
     pin_l = [torch.from_numpy(lg).pin_memory() for _, lg in xs]
     pin_out = torch.empty((T, D), dtype=torch.float32).pin_memory()
+    e2e_graphs = [api.MoeGraph(layers[c], pin_x[c], pin_l[c], k, path=wl["path"], out_host=pin_out)
+                  for c in range(NL)]
+    torch.cuda.synchronize()
 
     def e2e_step(i):
-        c = i % NL
-        x_dev[c].copy_(pin_x[c], non_blocking=True)
-        l_dev[c].copy_(pin_l[c], non_blocking=True)
-        out = api.moe_layer(layers[c], x_dev[c], l_dev[c], k, bufs=bufs[c], path=wl["path"])
-        pin_out.copy_(out, non_blocking=True)
+        e2e_graphs[i % NL].replay()
 
     for i in range(args.warmup):
         e2e_step(i)

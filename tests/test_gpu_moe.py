@@ -151,6 +151,33 @@ def test_graph_replay_with_changing_routes(api):
         check_against_oracle(eager, OL.moe_layer(layer, xv, lv, k))
 
 
+@pytest.mark.parametrize("path,T", [("gemv", 8), ("gemm", 40)])
+def test_moe_graph_with_host_buffers(api, path, T):
+    # api.MoeGraph: pinned host inputs -> device, the layer, device -> pinned host output,
+    # replayed as one graph; new inputs written into the same host buffers each step
+    layer = inputs.small_layer(92, E=12, D=256, F=128)
+    k = 4
+    dl = api.DeviceLayer.from_synthetic(layer)
+    x_host = torch.empty((T, 256), dtype=torch.bfloat16).pin_memory()
+    l_host = torch.empty((T, 12), dtype=torch.float32).pin_memory()
+    rng = np.random.default_rng(93)
+    x_host.copy_(torch.from_numpy(inputs.random_activations(rng, (T, 256), "bf16")).to(torch.bfloat16))
+    l_host.copy_(torch.from_numpy(inputs.normal_logits(rng, T, 12)))
+    mg = api.MoeGraph(dl, x_host, l_host, k, path=path)
+    for trial in range(3):
+        xv = inputs.random_activations(rng, (T, 256), "bf16")
+        lv = inputs.normal_logits(rng, T, 12)
+        x_host.copy_(torch.from_numpy(xv).to(torch.bfloat16))
+        l_host.copy_(torch.from_numpy(lv))
+        out = mg.replay()
+        mg.stream.synchronize()
+        eager, _, _ = run_layer(api, layer, xv, lv, k, path=path, dl=dl)
+        np.testing.assert_array_equal(out.numpy().astype(np.float64), eager)
+        check_against_oracle(eager, OL.moe_layer(layer, xv, lv, k))
+    with pytest.raises(ValueError):
+        api.MoeGraph(dl, x_host.cuda(), l_host, k)
+
+
 def test_full_size_decode_layer_sampled_tokens(api):
     # The 384-expert mixed-width decode layer (D = 4096, F = 1024, 16 tokens, top-8) in
     # the launch configuration the benchmark times; the oracle computes 2 tokens.

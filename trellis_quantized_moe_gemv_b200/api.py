@@ -484,3 +484,50 @@ def moe_layer(layer: DeviceLayer, x: torch.Tensor, logits: torch.Tensor, k: int,
     else:
         route_unpermute(bufs.y_perm, bufs.routing.inv, bufs.w, bufs.out, stream)
     return bufs.out
+
+
+class MoeGraph:
+    """One MoE layer call captured as a CUDA graph together with its host transfers.
+
+    replay() copies x_host [T, D] (bf16/fp16) and logits_host [T, E] (fp32), both pinned,
+    to the device, runs moe_layer (routing, rotation, expert path, combine) and copies the
+    result into out_host [T, D] fp32 (pinned), all as one graph launch on `stream`.  The
+    same host buffers are read and written on every replay: write the next step's inputs
+    into x_host / logits_host, replay, read out_host after synchronising the stream.
+    The first calls run eagerly (the library configures its kernels on first use, which
+    must happen outside a capture)."""
+
+    def __init__(self, layer: DeviceLayer, x_host: torch.Tensor, logits_host: torch.Tensor, k: int,
+                 path: str = "auto", out_host: Optional[torch.Tensor] = None, stream=None, warmup: int = 2):
+        for t, name in ((x_host, "x_host"), (logits_host, "logits_host")):
+            if t.is_cuda or not t.is_pinned():
+                raise ValueError("MoeGraph: %s must be pinned host memory" % name)
+        T = x_host.shape[0]
+        self.layer, self.k, self.path = layer, k, path
+        self.x_host, self.logits_host = x_host, logits_host
+        self.out_host = out_host if out_host is not None else \
+            torch.empty((T, layer.D), dtype=torch.float32).pin_memory()
+        self.x = torch.empty(x_host.shape, dtype=x_host.dtype, device="cuda")
+        self.logits = torch.empty(logits_host.shape, dtype=logits_host.dtype, device="cuda")
+        self.bufs = MoeBuffers(layer, T, k)
+        self.stream = stream if stream is not None else torch.cuda.Stream()
+        self.stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(self.stream):
+            for _ in range(warmup):
+                self._body()
+            self.stream.synchronize()
+            self.graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph, stream=self.stream):
+                self._body()
+
+    def _body(self):
+        self.x.copy_(self.x_host, non_blocking=True)
+        self.logits.copy_(self.logits_host, non_blocking=True)
+        out = moe_layer(self.layer, self.x, self.logits, self.k, bufs=self.bufs, path=self.path)
+        self.out_host.copy_(out, non_blocking=True)
+
+    def replay(self) -> torch.Tensor:
+        """Enqueue one layer call on the graph's stream; returns out_host (valid once the
+        stream has been synchronised)."""
+        self.graph.replay()
+        return self.out_host
