@@ -459,7 +459,7 @@ class MoeBuffers:
                               device=dev)
 
 
-GEMM_MIN_TOKENS = 352   # measured crossover of the two paths on the 384-expert decode layer
+GEMM_MIN_TOKENS = 392   # measured crossover of the two paths on the 384-expert decode layer
 
 
 def moe_layer(layer: DeviceLayer, x: torch.Tensor, logits: torch.Tensor, k: int,

@@ -437,7 +437,8 @@ __device__ __forceinline__ bool expert_ref(const tq_moe_layer &L, int e, ExpertR
 }
 
 // MoE GEMV work item = one CTA of kItemWarps warps: (active expert, 8 strips of 16
-// rows, column range, passes of 4 of the expert's routes).  The warps split the item's
+// rows, column range, passes of 4 * NB of the expert's routes: NB blocks of 4 routes
+// share every decoded weight).  The warps split the item's
 // column tiles into contiguous ranges; each streams its range of the 8 strips through
 // its own ring, and the warps' integer partial sums are added in shared memory at the
 // end of a pass.
@@ -452,17 +453,18 @@ __device__ __forceinline__ bool expert_ref(const tq_moe_layer &L, int e, ExpertR
 // !GATEUP: item = (active expert, 128 output rows); activations = quantised h'
 //          (indexed by route); out = y [routes][D] fp32.
 constexpr int kGateUpSplits = 1;
+constexpr int kNb2MinRoutes = 5;
 
-template <bool GATEUP>
-__global__ void __launch_bounds__(kItemThreads, 5)
+template <bool GATEUP, int NB>
+__global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
     moe_gemv_items_kernel(const tq_moe_layer L, const uint16_t *__restrict__ xq, const int2 *__restrict__ xmeta,
                           const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm,
                           const int32_t *__restrict__ active_ids, const int32_t *__restrict__ n_active_p,
                           int k, int n_routes, float *__restrict__ out) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     ItemSmem &sm_items = *reinterpret_cast<ItemSmem *>(smem_raw);
-    ItemRed<1> &red = *reinterpret_cast<ItemRed<1> *>(smem_raw);
-    __shared__ int s_row[4];
+    ItemRed<NB> &red = *reinterpret_cast<ItemRed<NB> *>(smem_raw);
+    __shared__ int s_row[4 * NB];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2;
     constexpr int splits = GATEUP ? kGateUpSplits : 1;
     const int per_expert = (GATEUP ? L.F / 64 : L.D / 128) * splits;
@@ -494,9 +496,9 @@ __global__ void __launch_bounds__(kItemThreads, 5)
     else
         strip_lane = ex.down + (size_t)(sub * 8 + cs) * tiles * (8 * ex.K);
 
-    for (int tb = 0; tb < ne; tb += 4) {
+    for (int tb = 0; tb < ne; tb += 4 * NB) {
         // activation row of each route of the pass (-1: none)
-        if (threadIdx.x < 4) {
+        if (threadIdx.x < 4 * NB) {
             const int tt = tb + threadIdx.x;
             int row = -1;            // -1: no route; -2: route with an invalid index
             if (tt < ne) {
@@ -510,18 +512,22 @@ __global__ void __launch_bounds__(kItemThreads, 5)
             s_row[threadIdx.x] = row;
         }
         __syncthreads();
-        const int my_row = s_row[gq >> 1];
-        const uint16_t *xw[1] = {my_row >= 0 ? xq + (size_t)my_row * 2 * cols + (gq & 1) * cols : nullptr};
-        AccI<1> acc;
+        const uint16_t *xw[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            const int my_row = s_row[4 * b + (gq >> 1)];
+            xw[b] = my_row >= 0 ? xq + (size_t)my_row * 2 * cols + (gq & 1) * cols : nullptr;
+        }
+        AccI<NB> acc;
         zero(acc);
-        bool ok = stream_any<1>(ex.K, ring, parity, jb, je, strip_lane, xw, acc);
+        bool ok = stream_any<NB>(ex.K, ring, parity, jb, je, strip_lane, xw, acc);
         ok = __syncthreads_and(ok);
         if (!ok) return;   // every warp drained its copies; the item is left unwritten
         store_partials(acc, red);   // the rings are idle now
         __syncthreads();
         if (GATEUP) {
-            for (int i = threadIdx.x; i < 4 * 16 * 4; i += kItemThreads) {
-                const int rt = i & 3, row = (i >> 2) & 15, st = i >> 6;
+            for (int i = threadIdx.x; i < 4 * 16 * 4 * NB; i += kItemThreads) {
+                const int rt = i % (4 * NB), row = (i / (4 * NB)) & 15, st = i / (64 * NB);
                 const int xrow = s_row[rt];
                 if (xrow == -1) continue;
                 const int f = (sub * 4 + st) * 16 + row;
@@ -538,8 +544,8 @@ __global__ void __launch_bounds__(kItemThreads, 5)
                 o[L.F] = uv;
             }
         } else {
-            for (int i = threadIdx.x; i < 8 * 16 * 4; i += kItemThreads) {
-                const int rt = i & 3, row = (i >> 2) & 15, st = i >> 6;
+            for (int i = threadIdx.x; i < 8 * 16 * 4 * NB; i += kItemThreads) {
+                const int rt = i % (4 * NB), row = (i / (4 * NB)) & 15, st = i / (64 * NB);
                 const int xrow = s_row[rt];
                 if (xrow < 0) continue;
                 const int2 y = red_sum(red, st, row, rt);
@@ -731,7 +737,8 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     const size_t smem = sizeof(ItemSmem);
     static bool configured = false;
     if (!configured) {
-        if (set_smem(moe_gemv_items_kernel<true>, smem) || set_smem(moe_gemv_items_kernel<false>, smem))
+        if (set_smem(moe_gemv_items_kernel<true, 1>, smem) || set_smem(moe_gemv_items_kernel<false, 1>, smem) ||
+            set_smem(moe_gemv_items_kernel<true, 2>, smem) || set_smem(moe_gemv_items_kernel<false, 2>, smem))
             return TQ_ERR_CUDA;
         configured = true;
     }
@@ -742,10 +749,17 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     const int dn_items = max_active * (L->D / 128);
     int st = launch_quantize_rows<false>(RowSrc<__half>{x_rot, L->D}, T, L->D, w.xq, w.xmeta, s, kStageGemvQuant);
     if (st) return st;
+    // 8 routes per pass once a batch averages kNb2MinRoutes or more routes per expert
+    // (each decoded weight then feeds twice the MMAs instead of being decoded twice)
+    const bool nb2 = routes >= kNb2MinRoutes * min(L->E, routes);
     {
         LaunchScope ls(s, kStageGemvGateUp);
-        moe_gemv_items_kernel<true><<<gu_items, kItemThreads, smem, s>>>(*L, w.xq, w.xmeta, offsets, perm, active_ids,
-                                                                          n_active, k, routes, w.gu);
+        if (nb2)
+            moe_gemv_items_kernel<true, 2><<<gu_items, kItemThreads, smem, s>>>(
+                *L, w.xq, w.xmeta, offsets, perm, active_ids, n_active, k, routes, w.gu);
+        else
+            moe_gemv_items_kernel<true, 1><<<gu_items, kItemThreads, smem, s>>>(
+                *L, w.xq, w.xmeta, offsets, perm, active_ids, n_active, k, routes, w.gu);
     }
     st = launch_status();
     if (st) return st;
@@ -753,8 +767,12 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
                                     kStageRotateH, L->sign_h);
     if (st) return st;
     LaunchScope ls(s, kStageGemvDown);
-    moe_gemv_items_kernel<false><<<dn_items, kItemThreads, smem, s>>>(*L, w.hq, w.hmeta, offsets, perm, active_ids,
-                                                                       n_active, k, routes, y_perm);
+    if (nb2)
+        moe_gemv_items_kernel<false, 2><<<dn_items, kItemThreads, smem, s>>>(*L, w.hq, w.hmeta, offsets, perm,
+                                                                              active_ids, n_active, k, routes, y_perm);
+    else
+        moe_gemv_items_kernel<false, 1><<<dn_items, kItemThreads, smem, s>>>(*L, w.hq, w.hmeta, offsets, perm,
+                                                                              active_ids, n_active, k, routes, y_perm);
     return launch_status();
 }
 
