@@ -254,7 +254,7 @@ def gateup_flops(layer, T, k):
 
 WORKLOADS = {
     "moe_decode_t16": dict(T=16, path="gemv", stage="gemv_gateup",
-                           kernel="moe_gemv_items_kernel<1> (gate/up GEMV, int8 tensor cores)",
+                           kernel="moe_gemv_items_kernel<1, 1> (gate/up GEMV, int8 tensor cores, 4 routes per pass)",
                            widths="368/15/1 experts at K=2/3/4", routing="top-8 of N(0,1) logits"),
     "moe_prefill_t8192": dict(T=8192, path="gemm", stage="gemm_gateup",
                               kernel="moe_gemm_kernel<1> (gate/up tcgen05 GEMM + SiLU)",
