@@ -190,6 +190,17 @@ def test_full_size_decode_layer_sampled_tokens(api):
     assert api.device_status() == 0
 
 
+def test_full_size_decode_layer_eight_routes_per_pass(api):
+    # The same layer at 320 tokens (6.7 routes per active expert): the GEMV runs 8 routes
+    # per pass; sampled tokens against the oracle
+    w = inputs.moe_sweep_tokens(320, layer=inputs.moe_decode_t16()["layer"])
+    got, bufs, _ = run_layer(api, w["layer"], w["x"], w["logits"], 8, path="gemv")
+    assert np.isfinite(got).all()
+    res = OL.moe_tokens(w["layer"], w["x"], w["logits"], 8, token_ids=[3, 319])
+    check_against_oracle(got, res, tokens=[3, 319])
+    assert api.device_status() == 0
+
+
 def test_workspace_too_small_is_an_error(api):
     layer = inputs.small_layer(5, E=12, D=256, F=128)
     dl = api.DeviceLayer.from_synthetic(layer)
