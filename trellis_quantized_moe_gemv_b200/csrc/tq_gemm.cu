@@ -430,18 +430,23 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     uint32_t v[16];
                     tmem_ld16(tmem_d + ((uint32_t)(32 * q) << 16) + (uint32_t)(tt * kGBN + c0), v);
                     if (GATEUP) {
+                        // lane l < 16 holds the gate row of output f, lane l + 16 the up row;
+                        // one exchange per column pair gives lane l both values of column c
+                        // and lane l + 16 both values of column c + 1
                         const int f = (mtile * 4 + q) * 16 + (lane & 15);
-                        const float sg = __half2float(ex.s_gate[f]), su = __half2float(ex.s_up[f]);
+                        const int hi = lane >> 4;
+                        const float sg = __half2float(ex.s_gate[f]) * kKappa, su = __half2float(ex.s_up[f]) * kKappa;
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const float dv = __uint_as_float(v[c]);
-                            const float du = __shfl_xor_sync(0xffffffffu, dv, 16);
-                            const int col = c0 + c;
-                            if (lane < 16 && col < n) {
+                        for (int c = 0; c < 16; c += 2) {
+                            const float mine0 = __uint_as_float(v[c]), mine1 = __uint_as_float(v[c + 1]);
+                            const float other = __shfl_xor_sync(0xffffffffu, hi ? mine0 : mine1, 16);
+                            const float graw = hi ? other : mine0, uraw = hi ? mine1 : other;
+                            const int col = c0 + c + hi;
+                            if (col < n) {
                                 const int route = r0 + n0 + col;
                                 const float sx = args.rowsum[route];
-                                const float g = sg * kKappa * fmaf(16777216.0f, dv, -255.0f * sx);
-                                const float u = su * kKappa * fmaf(16777216.0f, du, -255.0f * sx);
+                                const float g = sg * fmaf(16777216.0f, graw, -255.0f * sx);
+                                const float u = su * fmaf(16777216.0f, uraw, -255.0f * sx);
                                 if (args.raw_gu) {
                                     args.out[(size_t)route * 2 * L.F + f] = g;
                                     args.out[((size_t)route * 2 + 1) * L.F + f] = u;
