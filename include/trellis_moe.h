@@ -98,7 +98,8 @@ int tq_device_status(int32_t *flags_out, int clear);
  *   0 route_topk, 1 route_permute, 2 hadamard128 of the input, 3 GEMV gate/up+SiLU,
  *   4 rotation of h, 5 GEMV down, 6 route_unpermute, 7 trellis_decode, 8 trellis_gemv,
  *   9 GEMM gate/up+SiLU, 10 GEMM down, 11 GEMM preparation (tile list, route-ordered
- *   activation rows), 12 GEMV activation quantisation (x' rows to 16-bit fixed point).
+ *   activation rows), 12 GEMV activation quantisation (x' rows to 16-bit fixed point),
+ *   13 trellis_encode, 14 route_gather_rows.
  * tq_profile_enable creates 2*max_launches events (host-side CUDA resources; call it
  * outside graph capture); launches beyond max_launches are not recorded.  A launch made
  * during stream capture records its events as external event-record nodes of the graph,
@@ -202,6 +203,21 @@ int route_topk(const float *logits, int T, int E, int k, int32_t *topk_ids, floa
 int route_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *counts,
                   int32_t *offsets, int32_t *perm, int32_t *inv, int32_t *active_ids,
                   int32_t *n_active, tq_stream stream);
+
+/*
+ * route_gather_rows -- out[j][:] = src[index[j] / divisor][:] for j < rows: the row moves
+ * of expert parallelism (no counterpart on the pages, which run on one GPU).  With
+ * index = perm and divisor = k it lays the tokens' rotated rows out in expert-grouped
+ * route order (the rows one rank sends to the owners of its routes' experts); with
+ * index = inv and divisor = 1 it puts expert-grouped results back into arrival order.
+ *   src   : [src_rows][cols] of dtype (TQ_DTYPE_F16 / BF16 / F32), 16-byte aligned.
+ *   index : [rows] int32 (device).  out : [rows][cols], 16-byte aligned, caller-owned.
+ *   cols * element size must be a multiple of 16 bytes (TQ_ERR_INVALID_ARG otherwise).
+ *   An index outside [0, src_rows * divisor) raises device flag bit 0 and yields a zero
+ *   row.  The rows are copied bit for bit.
+ */
+int route_gather_rows(const void *src, int dtype, long long src_rows, int cols, const int32_t *index,
+                      int divisor, long long rows, void *out, tq_stream stream);
 
 /*
  * route_unpermute -- combine: out[t][d] = sum_{s=0..k-1} topk_w[t][s] * y_perm[inv[t*k+s]][d],

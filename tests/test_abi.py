@@ -35,7 +35,8 @@ def test_header_declares_the_boundary():
     for required in ("trellis_decode", "hadamard128", "trellis_gemv", "route_topk", "route_permute",
                      "route_unpermute", "moe_trellis_gemv", "moe_trellis_gemm",
                      "moe_trellis_workspace_size", "tq_status_string", "tq_abi_version",
-                     "tq_device_status", "trellis_encode", "trellis_encode_workspace_size"):
+                     "tq_device_status", "trellis_encode", "trellis_encode_workspace_size",
+                     "route_gather_rows"):
         assert required in names
 
 
@@ -87,6 +88,13 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.route_permute(FAKE, 4, 8, 2000, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
     assert lib.route_unpermute(FAKE, FAKE, FAKE, 4, 8, 6, FAKE, None) == 1
     assert lib.route_unpermute(MISALIGNED, FAKE, FAKE, 4, 8, 8, FAKE, None) == 3
+    # route_gather_rows(src, dtype, src_rows, cols, index, divisor, rows, out, stream)
+    assert lib.route_gather_rows(FAKE, 3, 4, 8, FAKE, 1, 4, FAKE, None) == 1         # dtype
+    assert lib.route_gather_rows(FAKE, 0, 4, 4, FAKE, 1, 4, FAKE, None) == 1         # 8-byte rows
+    assert lib.route_gather_rows(FAKE, 2, 4, 4, FAKE, 0, 4, FAKE, None) == 1         # divisor
+    assert lib.route_gather_rows(FAKE, 2, 4, 4, None, 1, 4, FAKE, None) == 1
+    assert lib.route_gather_rows(MISALIGNED, 2, 4, 4, FAKE, 1, 4, FAKE, None) == 3
+    assert lib.route_gather_rows(FAKE, 1, 4, 8, FAKE, 1, 0, FAKE, None) == 0         # empty: no-op
 
 
 def _layer_struct(K=2, E=16, D=256, F=128, n_groups=1):

@@ -67,6 +67,7 @@ SIGNATURES = {
     "route_topk": ([_VP, _I, _I, _I, _VP, _VP, _VP], _I),
     "route_permute": ([_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "route_unpermute": ([_VP, _VP, _VP, _I, _I, _I, _VP, _VP], _I),
+    "route_gather_rows": ([_VP, _I, _I64, _I, _VP, _I, _I64, _VP, _VP], _I),
     "route_unpermute_signed": ([_VP, _VP, _VP, _I, _I, _I, _VP, _VP, _VP], _I),
     "moe_trellis_workspace_size": ([ctypes.POINTER(TqMoeLayer), _I, _I], _SZ),
     "moe_trellis_gemv": ([ctypes.POINTER(TqMoeLayer), _VP, _VP, _VP, _VP, _VP, _I, _I, _VP, _VP,
@@ -146,7 +147,7 @@ def device_status(clear: bool = False) -> int:
 
 STAGES = ("route_topk", "route_permute", "rotate_x", "gemv_gateup", "rotate_h", "gemv_down",
           "route_unpermute", "trellis_decode", "trellis_gemv", "gemm_gateup", "gemm_down", "gemm_prep",
-          "gemv_quant", "trellis_encode")
+          "gemv_quant", "trellis_encode", "route_gather")
 
 
 def launch_count() -> int:
@@ -302,6 +303,22 @@ def route_permute(topk_ids: torch.Tensor, E: int, out: Optional[Routing] = None,
                                 _p(r.inv), _p(r.active_ids), _p(r.n_active), _stream(stream)),
            "route_permute")
     return r
+
+
+def route_gather_rows(src: torch.Tensor, index: torch.Tensor, divisor: int = 1,
+                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[j] = src[index[j] // divisor] (rows copied bit for bit; fp16, bf16 or fp32)."""
+    if src.dtype not in TQ_DTYPE:
+        raise TypeError("route_gather_rows: src must be fp16, bf16 or fp32")
+    _require(src, src.dtype, "src")
+    _require(index, torch.int32, "index")
+    rows = index.numel()
+    if out is None:
+        out = torch.empty((rows, src.shape[1]), dtype=src.dtype, device=src.device)
+    _require(out, src.dtype, "out")
+    _check(_fn("route_gather_rows")(_p(src), TQ_DTYPE[src.dtype], src.shape[0], src.shape[1], _p(index), divisor,
+                                    rows, _p(out), _stream(stream)), "route_gather_rows")
+    return out
 
 
 def route_unpermute(y_perm: torch.Tensor, inv: torch.Tensor, topk_w: torch.Tensor,

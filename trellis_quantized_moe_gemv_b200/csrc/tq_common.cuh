@@ -35,7 +35,7 @@ enum Stage {
     kStageTopk = 0, kStagePermute = 1, kStageRotateX = 2, kStageGemvGateUp = 3,
     kStageRotateH = 4, kStageGemvDown = 5, kStageUnpermute = 6, kStageDecode = 7,
     kStageGemv = 8, kStageGemmGateUp = 9, kStageGemmDown = 10, kStageGemmPrep = 11,
-    kStageGemvQuant = 12, kStageEncode = 13, kNumStages = 14
+    kStageGemvQuant = 12, kStageEncode = 13, kStageGather = 14, kNumStages = 15
 };
 
 // Brackets one kernel launch: counts it and, while profiling is on, records a start

@@ -446,6 +446,46 @@ TQ_API int route_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *
     return launch_status();
 }
 
+// Row gather for moving routed rows between layouts (expert-parallel dispatch and
+// return): out[j] = src[index[j] / divisor], one 16-byte vector per thread.  An index
+// outside [0, src_rows * divisor) raises device flag bit 0 and writes a zero row.
+__global__ void __launch_bounds__(256) route_gather_rows_kernel(const uint4 *__restrict__ src, long long src_rows,
+                                                                int row_vecs, const int32_t *__restrict__ index,
+                                                                int divisor, long long rows,
+                                                                uint4 *__restrict__ out) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= rows * row_vecs) return;
+    const long long j = idx / row_vecs;
+    const int c = (int)(idx % row_vecs);
+    const int ix = index[j];
+    const long long r = ix >= 0 ? ix / divisor : -1;
+    if (r < 0 || r >= src_rows) {
+        if (c == 0) raise_flag(1);
+        out[idx] = make_uint4(0u, 0u, 0u, 0u);
+        return;
+    }
+    out[idx] = src[r * row_vecs + c];
+}
+
+TQ_API int route_gather_rows(const void *src, int dtype, long long src_rows, int cols, const int32_t *index,
+                             int divisor, long long rows, void *out, tq_stream stream) {
+    if (dtype < TQ_DTYPE_F16 || dtype > TQ_DTYPE_F32 || src_rows < 0 || cols < 1 || divisor < 1 || rows < 0)
+        return TQ_ERR_INVALID_ARG;
+    const int esize = dtype == TQ_DTYPE_F32 ? 4 : 2;
+    if (((long long)cols * esize) % 16) return TQ_ERR_INVALID_ARG;
+    if (rows == 0) return TQ_OK;
+    if (!src || !index || !out) return TQ_ERR_INVALID_ARG;
+    if (!aligned16(src) || !aligned16(out)) return TQ_ERR_ALIGNMENT;
+    const int row_vecs = (int)((long long)cols * esize / 16);
+    const long long n = rows * row_vecs;
+    if ((n + 255) / 256 > 0x7fffffffll) return TQ_ERR_UNSUPPORTED;
+    cudaStream_t s = (cudaStream_t)stream;
+    LaunchScope ls(s, kStageGather);
+    route_gather_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const uint4 *>(src), src_rows, row_vecs, index, divisor, rows, reinterpret_cast<uint4 *>(out));
+    return launch_status();
+}
+
 TQ_API int route_unpermute(const float *y_perm, const int32_t *inv, const float *topk_w, int T,
                            int k, int D, float *out, tq_stream stream) {
     if (T < 0 || k < 1 || D < 4 || D % 4) return TQ_ERR_INVALID_ARG;
