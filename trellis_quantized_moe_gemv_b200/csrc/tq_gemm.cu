@@ -65,6 +65,7 @@ struct __align__(1024) GemmSmem {
     uint64_t kb_done[kGKbRing];
     uint64_t acc_full;                         // MMA -> epilogue
     uint64_t mma_done;                         // MMA drain on early exit
+    float rs[kGDecodeWarps][kGBN / 2];         // epilogue: each decode warp's route row sums
     uint32_t tmem_base;
     int32_t abort;                             // a role gave up
 };
@@ -416,26 +417,42 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
         // ------------------------------------------------------------ epilogue
         // group dg reads half (dg >> 1) of the columns of weight tile dg & 1, one warp
-        // per tensor-memory lane quarter
+        // per tensor-memory lane quarter.  The warp's route row sums (into its own
+        // shared-memory row) and its rows' scales are loaded before the accumulator
+        // wait, so that no global load sits in the store loop.
         {
             const int tt = tile;
             const int q = warp & 3;
+            const int row = 32 * q + lane;  // weight row of tile tt = tensor-memory lane
+            const int mtile = mt * kGTiles + tt;
+            const int half_cols = ((nmma / 16 + 1) / 2) * 16;
+            const int cb = slot * half_cols, ce = min(nmma, cb + half_cols);
+            float *rsw = sm.rs[warp - kGFirstDecodeWarp];
+            for (int i = lane; i < ce - cb; i += 32) {
+                const int col = cb + i;
+                rsw[i] = col < n ? args.rowsum[r0 + n0 + col] : 0.f;
+            }
+            const int f = (mtile * 4 + q) * 16 + (lane & 15);
+            const int hi = lane >> 4;
+            float sk0, sk1 = 0.f;            // the lane's row scales times 2^-12
+            if (GATEUP) {
+                sk0 = __half2float(ex.s_gate[f]) * kKappa;
+                sk1 = __half2float(ex.s_up[f]) * kKappa;
+            } else {
+                sk0 = __half2float(ex.s_down[mtile * kGBM + row]) * kKappa;
+            }
+            __syncwarp();
             if (wait(&sm.acc_full, 0)) {
                 tc_fence_after();
-                const int row = 32 * q + lane;  // weight row of tile tt = tensor-memory lane
-                const int mtile = mt * kGTiles + tt;
-                const int half_cols = ((nmma / 16 + 1) / 2) * 16;
-                const int cb = slot * half_cols, ce = min(nmma, cb + half_cols);
+                const uint32_t taddr = tmem_d + ((uint32_t)(32 * q) << 16) + (uint32_t)(tt * kGBN);
                 for (int c0 = cb; c0 < ce; c0 += 16) {
                     uint32_t v[16];
-                    tmem_ld16(tmem_d + ((uint32_t)(32 * q) << 16) + (uint32_t)(tt * kGBN + c0), v);
+                    tmem_ld16(taddr + c0, v);
+                    const float *rsc = rsw + (c0 - cb);
                     if (GATEUP) {
                         // lane l < 16 holds the gate row of output f, lane l + 16 the up row;
                         // one exchange per column pair gives lane l both values of column c
                         // and lane l + 16 both values of column c + 1
-                        const int f = (mtile * 4 + q) * 16 + (lane & 15);
-                        const int hi = lane >> 4;
-                        const float sg = __half2float(ex.s_gate[f]) * kKappa, su = __half2float(ex.s_up[f]) * kKappa;
 #pragma unroll
                         for (int c = 0; c < 16; c += 2) {
                             const float mine0 = __uint_as_float(v[c]), mine1 = __uint_as_float(v[c + 1]);
@@ -444,9 +461,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
                             const int col = c0 + c + hi;
                             if (col < n) {
                                 const int route = r0 + n0 + col;
-                                const float sx = args.rowsum[route];
-                                const float g = sg * fmaf(16777216.0f, graw, -255.0f * sx);
-                                const float u = su * fmaf(16777216.0f, uraw, -255.0f * sx);
+                                const float sx = rsc[c + hi];
+                                const float g = sk0 * fmaf(16777216.0f, graw, -255.0f * sx);
+                                const float u = sk1 * fmaf(16777216.0f, uraw, -255.0f * sx);
                                 if (args.raw_gu) {
                                     args.out[(size_t)route * 2 * L.F + f] = g;
                                     args.out[((size_t)route * 2 + 1) * L.F + f] = u;
@@ -457,16 +474,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         }
                     } else {
                         const int d = mtile * kGBM + row;
-                        const float sd = __half2float(ex.s_down[d]);
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
                             const int col = c0 + c;
-                            if (col < n) {
-                                const int route = r0 + n0 + col;
-                                const float sx = args.rowsum[route];
-                                args.out[(size_t)route * L.D + d] =
-                                    sd * kKappa * fmaf(16777216.0f, __uint_as_float(v[c]), -255.0f * sx);
-                            }
+                            if (col < n)
+                                args.out[(size_t)(r0 + n0 + col) * L.D + d] =
+                                    sk0 * fmaf(16777216.0f, __uint_as_float(v[c]), -255.0f * rsc[c]);
                         }
                     }
                 }
