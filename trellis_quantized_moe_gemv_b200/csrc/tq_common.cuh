@@ -5,6 +5,7 @@
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <utility>
 
 #include "trellis_moe.h"
 
@@ -50,6 +51,33 @@ struct LaunchScope {
 // Text of the most recent CUDA failure seen by the library (tq_last_error_string).
 int record_error(const char *what);
 int record_cuda_error(const char *what);
+
+// Chained launches (programmatic dependent launch).  A kernel started by
+// launch_chained may begin while the previous kernel on its stream is still finishing;
+// its first statement is chain_entry(), which waits for that kernel to complete and
+// its writes to be visible (so nothing another kernel wrote is read earlier than with a
+// plain launch) and lets the next chained kernel be launched.  Both instructions do
+// nothing in a kernel launched the ordinary way.
+__device__ __forceinline__ void chain_entry() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                  Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 inline int launch_status() {
     cudaError_t e = cudaGetLastError();

@@ -328,6 +328,7 @@ struct SwigluSrc {
 template <typename Src, bool ROTATE>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int cols, const int8_t *__restrict__ signs,
                                                             uint16_t *__restrict__ xq, int2 *__restrict__ meta) {
+    chain_entry();
     __shared__ float s_max[8];
     __shared__ int s_sum[8];
     const int row = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -402,7 +403,7 @@ int launch_quantize_rows(const Src &src, long long rows, int cols, uint16_t *xq,
     if (rows <= 0) return TQ_OK;
     if (rows > 0x7fffffffll) return TQ_ERR_UNSUPPORTED;
     LaunchScope ls(s, stage);
-    quantize_rows_kernel<Src, ROTATE><<<(unsigned)rows, 256, 0, s>>>(src, cols, signs, xq, meta);
+    launch_chained(quantize_rows_kernel<Src, ROTATE>, (unsigned)rows, 256, 0, s, src, cols, signs, xq, meta);
     return launch_status();
 }
 
@@ -461,6 +462,7 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
                           const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm,
                           const int32_t *__restrict__ active_ids, const int32_t *__restrict__ n_active_p,
                           int k, int n_routes, float *__restrict__ out) {
+    chain_entry();
     extern __shared__ __align__(128) unsigned char smem_raw[];
     ItemSmem &sm_items = *reinterpret_cast<ItemSmem *>(smem_raw);
     ItemRed<NB> &red = *reinterpret_cast<ItemRed<NB> *>(smem_raw);
@@ -755,11 +757,11 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     {
         LaunchScope ls(s, kStageGemvGateUp);
         if (nb2)
-            moe_gemv_items_kernel<true, 2><<<gu_items, kItemThreads, smem, s>>>(
-                *L, w.xq, w.xmeta, offsets, perm, active_ids, n_active, k, routes, w.gu);
+            launch_chained(moe_gemv_items_kernel<true, 2>, gu_items, kItemThreads, smem, s, *L, w.xq, w.xmeta, offsets,
+                           perm, active_ids, n_active, k, routes, w.gu);
         else
-            moe_gemv_items_kernel<true, 1><<<gu_items, kItemThreads, smem, s>>>(
-                *L, w.xq, w.xmeta, offsets, perm, active_ids, n_active, k, routes, w.gu);
+            launch_chained(moe_gemv_items_kernel<true, 1>, gu_items, kItemThreads, smem, s, *L, w.xq, w.xmeta, offsets,
+                           perm, active_ids, n_active, k, routes, w.gu);
     }
     st = launch_status();
     if (st) return st;
@@ -768,11 +770,11 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     if (st) return st;
     LaunchScope ls(s, kStageGemvDown);
     if (nb2)
-        moe_gemv_items_kernel<false, 2><<<dn_items, kItemThreads, smem, s>>>(*L, w.hq, w.hmeta, offsets, perm,
-                                                                              active_ids, n_active, k, routes, y_perm);
+        launch_chained(moe_gemv_items_kernel<false, 2>, dn_items, kItemThreads, smem, s, *L, w.hq, w.hmeta, offsets,
+                       perm, active_ids, n_active, k, routes, y_perm);
     else
-        moe_gemv_items_kernel<false, 1><<<dn_items, kItemThreads, smem, s>>>(*L, w.hq, w.hmeta, offsets, perm,
-                                                                              active_ids, n_active, k, routes, y_perm);
+        launch_chained(moe_gemv_items_kernel<false, 1>, dn_items, kItemThreads, smem, s, *L, w.hq, w.hmeta, offsets,
+                       perm, active_ids, n_active, k, routes, y_perm);
     return launch_status();
 }
 

@@ -60,6 +60,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) hadamard128_kernel(const T *__restrict__ x, long long n_chunks,
                                                           const int8_t *__restrict__ signs, int chunks_per_row,
                                                           __half *__restrict__ out) {
+    chain_entry();
     const long long chunk = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (chunk >= n_chunks) return;
@@ -91,16 +92,16 @@ int launch_hadamard128(const void *x, int x_dtype, long long rows, long long col
     LaunchScope ls(s, stage);
     switch (x_dtype) {
         case TQ_DTYPE_F16:
-            hadamard128_kernel<__half><<<(unsigned)blocks, threads, 0, s>>>((const __half *)x, n_chunks, signs,
-                                                                            (int)(cols / 128), out);
+            launch_chained(hadamard128_kernel<__half>, (unsigned)blocks, threads, 0, s, (const __half *)x, n_chunks,
+                           signs, (int)(cols / 128), out);
             break;
         case TQ_DTYPE_BF16:
-            hadamard128_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, s>>>(
-                (const __nv_bfloat16 *)x, n_chunks, signs, (int)(cols / 128), out);
+            launch_chained(hadamard128_kernel<__nv_bfloat16>, (unsigned)blocks, threads, 0, s,
+                           (const __nv_bfloat16 *)x, n_chunks, signs, (int)(cols / 128), out);
             break;
         case TQ_DTYPE_F32:
-            hadamard128_kernel<float><<<(unsigned)blocks, threads, 0, s>>>((const float *)x, n_chunks, signs,
-                                                                           (int)(cols / 128), out);
+            launch_chained(hadamard128_kernel<float>, (unsigned)blocks, threads, 0, s, (const float *)x, n_chunks,
+                           signs, (int)(cols / 128), out);
             break;
         default:
             return TQ_ERR_INVALID_ARG;
@@ -115,6 +116,7 @@ int launch_hadamard128(const void *x, int x_dtype, long long rows, long long col
 __global__ void __launch_bounds__(256) route_unpermute_signed_kernel(
     const float *__restrict__ y_perm, const int32_t *__restrict__ inv, const float *__restrict__ w, int T, int k,
     int D, int n_routes, const int8_t *__restrict__ signs, float *__restrict__ out) {
+    chain_entry();
     const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     const int chunks = D / 128;
@@ -154,8 +156,8 @@ TQ_API int route_unpermute_signed(const float *y_perm, const int32_t *inv, const
     const long long blocks = (warps * 32 + 255) / 256;
     if (blocks > 0x7fffffffll) return TQ_ERR_UNSUPPORTED;
     tq::LaunchScope ls(s, tq::kStageUnpermute);
-    tq::route_unpermute_signed_kernel<<<(unsigned)blocks, 256, 0, s>>>(y_perm, inv, topk_w, T, k, D, T * k, signs_y,
-                                                                        out);
+    tq::launch_chained(tq::route_unpermute_signed_kernel, (unsigned)blocks, 256, 0, s, y_perm, inv, topk_w, T, k, D,
+                       T * k, signs_y, out);
     return tq::launch_status();
 }
 

@@ -14,6 +14,7 @@ template <int PER_LANE>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T,
                                                          int E, int k, int32_t *__restrict__ ids,
                                                          float *__restrict__ w) {
+    chain_entry();
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= T) return;
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
     const int32_t *__restrict__ topk_ids, int n_routes, int E, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv,
     int32_t *__restrict__ active_ids, int32_t *__restrict__ n_active) {
+    chain_entry();
     extern __shared__ int32_t smem[];
     int32_t *cursor = smem;                 // [E] histogram, then routes placed so far
     int32_t *base = cursor + E;             // [E] exclusive offsets
@@ -377,6 +379,7 @@ __global__ void __launch_bounds__(256) route_unpermute_kernel(const float *__res
                                                               const float *__restrict__ w, int T,
                                                               int k, int D, int n_routes,
                                                               float *__restrict__ out) {
+    chain_entry();
     const int d4 = D >> 2;
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long long)T * d4) return;
@@ -414,11 +417,11 @@ TQ_API int route_topk(const float *logits, int T, int E, int k, int32_t *topk_id
     const int per = (E + 31) / 32;
     LaunchScope ls(s, kStageTopk);
     if (per <= 4)
-        route_topk_kernel<4><<<blocks, threads, 0, s>>>(logits, T, E, k, topk_ids, topk_w);
+        launch_chained(route_topk_kernel<4>, blocks, threads, 0, s, logits, T, E, k, topk_ids, topk_w);
     else if (per <= 12)
-        route_topk_kernel<12><<<blocks, threads, 0, s>>>(logits, T, E, k, topk_ids, topk_w);
+        launch_chained(route_topk_kernel<12>, blocks, threads, 0, s, logits, T, E, k, topk_ids, topk_w);
     else
-        route_topk_kernel<32><<<blocks, threads, 0, s>>>(logits, T, E, k, topk_ids, topk_w);
+        launch_chained(route_topk_kernel<32>, blocks, threads, 0, s, logits, T, E, k, topk_ids, topk_w);
     return launch_status();
 }
 
@@ -441,8 +444,8 @@ TQ_API int route_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *
         configured = true;
     }
     LaunchScope ls(s, kStagePermute);
-    route_permute_kernel<<<1, kPermThreads, smem, s>>>(topk_ids, T * k, E, counts, offsets, perm,
-                                                       inv, active_ids, n_active);
+    launch_chained(route_permute_kernel, 1, kPermThreads, smem, s, topk_ids, T * k, E, counts, offsets, perm, inv,
+                   active_ids, n_active);
     return launch_status();
 }
 
@@ -496,7 +499,7 @@ TQ_API int route_unpermute(const float *y_perm, const int32_t *inv, const float 
     const long long n = (long long)T * (D / 4);
     const int threads = 256;
     LaunchScope ls(s, kStageUnpermute);
-    route_unpermute_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, s>>>(
-        y_perm, inv, topk_w, T, k, D, T * k, out);
+    launch_chained(route_unpermute_kernel, (unsigned)((n + threads - 1) / threads), threads, 0, s, y_perm, inv,
+                   topk_w, T, k, D, T * k, out);
     return launch_status();
 }
