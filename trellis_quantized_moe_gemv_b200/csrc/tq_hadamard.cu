@@ -5,6 +5,7 @@
 //
 // One warp per 128-chunk.  Lane l holds elements 4l..4l+3: index bits 0 and 1 are
 // butterflies inside the lane, bits 2..6 pair lane l with lane l ^ (1 << (b-2)).
+#include "tq_combine.cuh"
 #include "tq_common.cuh"
 
 namespace tq {
@@ -123,20 +124,8 @@ __global__ void __launch_bounds__(256) route_unpermute_signed_kernel(
     if (wid >= (long long)T * chunks) return;
     const int t = (int)(wid / chunks), c = (int)(wid % chunks);
     const int col = c * 128 + 4 * lane;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < k; ++s) {
-        const int r = inv[t * k + s];
-        const float ws = w[t * k + s];
-        if (r < 0 || r >= n_routes) {
-            if (lane == 0) raise_flag(1);
-            continue;
-        }
-        const float4 y = *reinterpret_cast<const float4 *>(y_perm + (size_t)r * D + col);
-        v[0] = fmaf(ws, y.x, v[0]);
-        v[1] = fmaf(ws, y.y, v[1]);
-        v[2] = fmaf(ws, y.z, v[2]);
-        v[3] = fmaf(ws, y.w, v[3]);
-    }
+    const float4 a = combine_slots(y_perm, inv, w, t, k, D, n_routes, col, lane == 0);
+    float v[4] = {a.x, a.y, a.z, a.w};
     fwht128_warp(v, lane);
     const char4 sg = *reinterpret_cast<const char4 *>(signs + col);
     *reinterpret_cast<float4 *>(out + (size_t)t * D + col) = make_float4(v[0] * sg.x, v[1] * sg.y, v[2] * sg.z, v[3] * sg.w);

@@ -2,6 +2,7 @@
 //
 // "top-8 softmax routing" of the routed experts; per-width groups with ascending
 // global expert ids ("DeepSeek-V4.1-Flash-1017 TrellisMX K2 Mix", "What is stored").
+#include "tq_combine.cuh"
 #include "tq_common.cuh"
 
 namespace tq {
@@ -385,21 +386,7 @@ __global__ void __launch_bounds__(256) route_unpermute_kernel(const float *__res
     if (idx >= (long long)T * d4) return;
     const int t = (int)(idx / d4);
     const int c = (int)(idx % d4);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < k; ++s) {
-        int r = inv[t * k + s];
-        float ws = w[t * k + s];
-        if (r < 0 || r >= n_routes) {
-            raise_flag(1);
-            continue;
-        }
-        float4 y = reinterpret_cast<const float4 *>(y_perm + (size_t)r * D)[c];
-        acc.x = fmaf(ws, y.x, acc.x);
-        acc.y = fmaf(ws, y.y, acc.y);
-        acc.z = fmaf(ws, y.z, acc.z);
-        acc.w = fmaf(ws, y.w, acc.w);
-    }
-    reinterpret_cast<float4 *>(out + (size_t)t * D)[c] = acc;
+    reinterpret_cast<float4 *>(out + (size_t)t * D)[c] = combine_slots(y_perm, inv, w, t, k, D, n_routes, 4 * c, true);
 }
 
 }  // namespace tq
