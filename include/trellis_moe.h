@@ -220,6 +220,18 @@ int route_gather_rows(const void *src, int dtype, long long src_rows, int cols, 
                       int divisor, long long rows, void *out, tq_stream stream);
 
 /*
+ * route_topk_permute -- route_topk followed by route_permute, with the same arguments
+ * and results (topk_ids / topk_w as route_topk writes them, the grouping arrays as
+ * route_permute writes them).  Up to T*k = 4096 routes it is one single-CTA launch (the
+ * CTA's warps take the tokens' top-k in turn, then the CTA groups the routes from a
+ * shared-memory copy of the ids), recorded under profiling stage 0; larger batches run
+ * the two calls.  1 <= k <= 32, k <= E <= 1024.
+ */
+int route_topk_permute(const float *logits, int T, int E, int k, int32_t *topk_ids, float *topk_w,
+                       int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv,
+                       int32_t *active_ids, int32_t *n_active, tq_stream stream);
+
+/*
  * route_unpermute -- combine: out[t][d] = sum_{s=0..k-1} topk_w[t][s] * y_perm[inv[t*k+s]][d],
  * summed in slot order in fp32 (deterministic, no atomics).
  *   y_perm : [T*k][D] fp32 in expert-grouped order.  inv, topk_w : [T*k].

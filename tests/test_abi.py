@@ -36,7 +36,7 @@ def test_header_declares_the_boundary():
                      "route_unpermute", "moe_trellis_gemv", "moe_trellis_gemm",
                      "moe_trellis_workspace_size", "tq_status_string", "tq_abi_version",
                      "tq_device_status", "trellis_encode", "trellis_encode_workspace_size",
-                     "route_gather_rows"):
+                     "route_gather_rows", "route_topk_permute"):
         assert required in names
 
 
@@ -88,6 +88,10 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.route_permute(FAKE, 4, 8, 2000, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
     assert lib.route_unpermute(FAKE, FAKE, FAKE, 4, 8, 6, FAKE, None) == 1
     assert lib.route_unpermute(MISALIGNED, FAKE, FAKE, 4, 8, 8, FAKE, None) == 3
+    # route_topk_permute(logits, T, E, k, ids, w, counts, offsets, perm, inv, active, n_active, stream)
+    assert lib.route_topk_permute(FAKE, 4, 384, 0, *[FAKE] * 8, None) == 1          # k
+    assert lib.route_topk_permute(FAKE, 4, 2000, 8, *[FAKE] * 8, None) == 1         # E
+    assert lib.route_topk_permute(FAKE, 4, 384, 8, FAKE, FAKE, None, *[FAKE] * 5, None) == 1
     # route_gather_rows(src, dtype, src_rows, cols, index, divisor, rows, out, stream)
     assert lib.route_gather_rows(FAKE, 3, 4, 8, FAKE, 1, 4, FAKE, None) == 1         # dtype
     assert lib.route_gather_rows(FAKE, 0, 4, 4, FAKE, 1, 4, FAKE, None) == 1         # 8-byte rows

@@ -183,6 +183,29 @@ def test_route_permute_exact(api, T, E, k):
     np.testing.assert_array_equal(r.active_ids.cpu().numpy()[:n_act], active)
 
 
+@pytest.mark.parametrize("T,E,k", [(1, 384, 8), (16, 384, 8), (37, 40, 8), (7, 1024, 32), (512, 384, 8),
+                                   (513, 384, 8), (3, 5, 2), (128, 12, 4)])
+def test_route_topk_permute_fused_equals_the_two_calls(api, T, E, k):
+    # up to 4096 routes one launch (shared-memory ids), beyond it the two calls; either
+    # way the same arrays as route_topk + route_permute, and the oracle's grouping
+    rng = np.random.default_rng(900 + T + E + k)
+    logits = torch.from_numpy(inputs.normal_logits(rng, T, E)).cuda()
+    ids, w, r = api.route_topk_permute(logits, k, E)
+    ids2, w2 = api.route_topk(logits, k)
+    r2 = api.route_permute(ids2, E)
+    torch.cuda.synchronize()
+    assert torch.equal(ids, ids2) and torch.equal(w, w2)
+    for name in ("counts", "offsets", "perm", "inv"):
+        assert torch.equal(getattr(r, name), getattr(r2, name)), name
+    n_act = int(r.n_active.item())
+    assert n_act == int(r2.n_active.item())
+    assert torch.equal(r.active_ids[:n_act], r2.active_ids[:n_act])
+    counts, offsets, perm, inv = OL.route_permute(ids.cpu().numpy(), E)
+    np.testing.assert_array_equal(r.perm.cpu().numpy(), perm)
+    np.testing.assert_array_equal(r.inv.cpu().numpy(), inv)
+    assert api.device_status() == 0
+
+
 @pytest.mark.parametrize("T,k,E", [(2048, 8, 384), (2500, 8, 1024), (2051, 8, 7), (40000, 8, 384)])
 def test_route_permute_multi_block_exact(api, T, k, E):
     # T*k >= 16384 takes the multi-CTA grouping (4096-route blocks, ragged last block);

@@ -68,6 +68,7 @@ SIGNATURES = {
     "route_permute": ([_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "route_unpermute": ([_VP, _VP, _VP, _I, _I, _I, _VP, _VP], _I),
     "route_gather_rows": ([_VP, _I, _I64, _I, _VP, _I, _I64, _VP, _VP], _I),
+    "route_topk_permute": ([_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "route_unpermute_signed": ([_VP, _VP, _VP, _I, _I, _I, _VP, _VP, _VP], _I),
     "moe_trellis_workspace_size": ([ctypes.POINTER(TqMoeLayer), _I, _I], _SZ),
     "moe_trellis_gemv": ([ctypes.POINTER(TqMoeLayer), _VP, _VP, _VP, _VP, _VP, _I, _I, _VP, _VP,
@@ -305,6 +306,22 @@ def route_permute(topk_ids: torch.Tensor, E: int, out: Optional[Routing] = None,
     return r
 
 
+def route_topk_permute(logits: torch.Tensor, k: int, E: int, ids: Optional[torch.Tensor] = None,
+                       w: Optional[torch.Tensor] = None, out: Optional["Routing"] = None, stream=None):
+    """route_topk then route_permute (one launch for up to 4096 routes): (ids, w, routing)."""
+    _require(logits, torch.float32, "logits")
+    T = logits.shape[0]
+    if ids is None:
+        ids = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if w is None:
+        w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    r = out if out is not None else Routing.empty(T, k, E, logits.device)
+    _check(_fn("route_topk_permute")(_p(logits), T, E, k, _p(ids), _p(w), _p(r.counts), _p(r.offsets),
+                                     _p(r.perm), _p(r.inv), _p(r.active_ids), _p(r.n_active), _stream(stream)),
+           "route_topk_permute")
+    return ids, w, r
+
+
 def route_gather_rows(src: torch.Tensor, index: torch.Tensor, divisor: int = 1,
                       out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """out[j] = src[index[j] // divisor] (rows copied bit for bit; fp16, bf16 or fp32)."""
@@ -486,8 +503,7 @@ def moe_layer(layer: DeviceLayer, x: torch.Tensor, logits: torch.Tensor, k: int,
     x: [T, D] bf16/fp16; logits: [T, E] fp32.  Returns out [T, D] fp32."""
     T = x.shape[0]
     bufs = bufs or MoeBuffers(layer, T, k)
-    route_topk(logits, k, bufs.ids, bufs.w, stream)
-    route_permute(bufs.ids, layer.E, bufs.routing, stream)
+    route_topk_permute(logits, k, layer.E, bufs.ids, bufs.w, bufs.routing, stream)
     if layer.signs is not None:
         hadamard128_signed(x, layer.signs["x"], bufs.x_rot, stream)
     else:

@@ -11,14 +11,12 @@ constexpr int kTopkMaxPerLane = 32;   // E <= 32 * 32
 
 // One warp per token.  Each lane owns logits e = lane + 32*j.  k rounds of a warp-wide
 // arg-max (larger logit first, ties to the lower id) select the experts in order.
+// The token's ids also go to ids_copy[lane] (lanes < k) when ids_copy is not null.
 template <int PER_LANE>
-__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T,
-                                                         int E, int k, int32_t *__restrict__ ids,
-                                                         float *__restrict__ w) {
-    chain_entry();
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (warp >= T) return;
+__device__ __forceinline__ void topk_token(const float *__restrict__ logits, int token, int E, int k,
+                                           int32_t *__restrict__ ids, float *__restrict__ w, int lane,
+                                           int32_t *ids_copy) {
+    const int warp = token;
     const float *row = logits + (size_t)warp * E;
     float v[PER_LANE];
 #pragma unroll
@@ -68,7 +66,19 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
     if (lane < k) {
         ids[(size_t)warp * k + lane] = sel_e;
         w[(size_t)warp * k + lane] = ex / sum;
+        if (ids_copy) ids_copy[lane] = sel_e;
     }
+}
+
+template <int PER_LANE>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T,
+                                                         int E, int k, int32_t *__restrict__ ids,
+                                                         float *__restrict__ w) {
+    chain_entry();
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= T) return;
+    topk_token<PER_LANE>(logits, warp, E, k, ids, w, lane, nullptr);
 }
 
 // Stable grouping of routes by expert in one CTA of 1024 threads.  Routes are taken
@@ -79,16 +89,17 @@ constexpr int kPermThreads = 1024;
 constexpr int kPermWarps = kPermThreads / 32;
 constexpr int kPermMaxE = 1024;
 
-inline size_t permute_smem_bytes(int E) {
+__host__ __device__ inline size_t permute_smem_bytes(int E) {
     return sizeof(int32_t) * ((size_t)(3 + kPermWarps) * E);
 }
 
-__global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
-    const int32_t *__restrict__ topk_ids, int n_routes, int E, int32_t *__restrict__ counts,
-    int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv,
-    int32_t *__restrict__ active_ids, int32_t *__restrict__ n_active) {
-    chain_entry();
-    extern __shared__ int32_t smem[];
+// The grouping by one CTA of kPermThreads threads; smem holds permute_smem_bytes(E).
+// topk_ids may point to global or shared memory.
+__device__ __forceinline__ void permute_cta(const int32_t *topk_ids, int n_routes, int E,
+                                            int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                                            int32_t *__restrict__ perm, int32_t *__restrict__ inv,
+                                            int32_t *__restrict__ active_ids, int32_t *__restrict__ n_active,
+                                            int32_t *smem) {
     int32_t *cursor = smem;                 // [E] histogram, then routes placed so far
     int32_t *base = cursor + E;             // [E] exclusive offsets
     int32_t *total = base + E;              // [E] routes of the current chunk
@@ -190,6 +201,34 @@ __global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
         for (int x = tid; x < kPermWarps * E; x += kPermThreads) wcnt[x] = 0;
         __syncthreads();
     }
+}
+
+__global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
+    const int32_t *__restrict__ topk_ids, int n_routes, int E, int32_t *__restrict__ counts,
+    int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv,
+    int32_t *__restrict__ active_ids, int32_t *__restrict__ n_active) {
+    chain_entry();
+    extern __shared__ int32_t smem[];
+    permute_cta(topk_ids, n_routes, E, counts, offsets, perm, inv, active_ids, n_active, smem);
+}
+
+// Routing of a small batch in one launch: the 32 warps take the tokens' top-k in turn
+// (writing ids and weights, and the ids into shared memory), then the CTA groups the
+// routes from the shared copy -- the same results as route_topk then route_permute.
+constexpr int kFusedRouteMax = 4096;    // routes (T*k) of one fused launch
+
+template <int PER_LANE>
+__global__ void __launch_bounds__(kPermThreads) route_topk_permute_kernel(
+    const float *__restrict__ logits, int T, int E, int k, int32_t *__restrict__ ids, float *__restrict__ w,
+    int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+    int32_t *__restrict__ inv, int32_t *__restrict__ active_ids, int32_t *__restrict__ n_active) {
+    chain_entry();
+    extern __shared__ int32_t smem[];
+    int32_t *ids_s = smem + (permute_smem_bytes(E) / sizeof(int32_t));   // [T*k]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int t = warp; t < T; t += kPermWarps) topk_token<PER_LANE>(logits, t, E, k, ids, w, lane, ids_s + t * k);
+    __syncthreads();
+    permute_cta(ids_s, T * k, E, counts, offsets, perm, inv, active_ids, n_active, smem);
 }
 
 // ---------------------------------------------------------------- multi-CTA grouping
@@ -433,6 +472,47 @@ TQ_API int route_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *
     LaunchScope ls(s, kStagePermute);
     launch_chained(route_permute_kernel, 1, kPermThreads, smem, s, topk_ids, T * k, E, counts, offsets, perm, inv,
                    active_ids, n_active);
+    return launch_status();
+}
+
+TQ_API int route_topk_permute(const float *logits, int T, int E, int k, int32_t *topk_ids, float *topk_w,
+                              int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv,
+                              int32_t *active_ids, int32_t *n_active, tq_stream stream) {
+    if (T < 0 || k < 1 || k > 32 || E < k || E > kPermMaxE) return TQ_ERR_INVALID_ARG;
+    if ((long long)T * k > (1ll << 30)) return TQ_ERR_UNSUPPORTED;
+    if (!counts || !offsets || !active_ids || !n_active) return TQ_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !topk_ids || !topk_w || !perm || !inv)) return TQ_ERR_INVALID_ARG;
+    if ((long long)T * k > kFusedRouteMax || T == 0) {
+        // large batches (and the empty one): the two launches
+        int st = T > 0 ? route_topk(logits, T, E, k, topk_ids, topk_w, stream) : TQ_OK;
+        if (st) return st;
+        return route_permute(topk_ids, T, k, E, counts, offsets, perm, inv, active_ids, n_active, stream);
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t smem = permute_smem_bytes(E) + sizeof(int32_t) * (size_t)T * k;
+    static bool configured = false;
+    if (!configured) {
+        const int most = (int)(permute_smem_bytes(kPermMaxE) + sizeof(int32_t) * kFusedRouteMax);
+        if (cudaFuncSetAttribute(route_topk_permute_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(route_topk_permute_kernel<12>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(route_topk_permute_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) !=
+                cudaSuccess)
+            return TQ_ERR_CUDA;
+        configured = true;
+    }
+    const int per = (E + 31) / 32;
+    LaunchScope ls(s, kStageTopk);
+    if (per <= 4)
+        launch_chained(route_topk_permute_kernel<4>, 1, kPermThreads, smem, s, logits, T, E, k, topk_ids, topk_w,
+                       counts, offsets, perm, inv, active_ids, n_active);
+    else if (per <= 12)
+        launch_chained(route_topk_permute_kernel<12>, 1, kPermThreads, smem, s, logits, T, E, k, topk_ids, topk_w,
+                       counts, offsets, perm, inv, active_ids, n_active);
+    else
+        launch_chained(route_topk_permute_kernel<32>, 1, kPermThreads, smem, s, logits, T, E, k, topk_ids, topk_w,
+                       counts, offsets, perm, inv, active_ids, n_active);
     return launch_status();
 }
 
