@@ -58,13 +58,13 @@ class OracleOps:
         return torch.from_numpy(self.OL.combine(y_perm.numpy(), inv.numpy(), w.numpy()))
 
 
-def _case(rank, hot):
+def _case(rank, hot, empty_rank=-1):
     from trellis_quantized_moe_gemv_b200 import inputs
     layer = inputs.small_layer(321, E=6, D=256, F=128, split={2: 4, 3: 1, 4: 1})
     if hot:
         layer = inputs.with_signs(layer, 322)
     rng = np.random.default_rng(400 + rank)
-    T = 3 + 2 * rank                                  # ranks hold different token counts
+    T = 0 if rank == empty_rank else 3 + 2 * rank     # ranks hold different token counts
     x = inputs.random_activations(rng, (T, layer.D), "bf16")
     logits = inputs.normal_logits(rng, T, layer.E)
     if hot:
@@ -72,7 +72,7 @@ def _case(rank, hot):
     return layer, x, logits
 
 
-def _worker(rank, world, port, hot, out):
+def _worker(rank, world, port, hot, out, empty_rank=-1):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     from oracle import layer as OL
@@ -80,15 +80,16 @@ def _worker(rank, world, port, hot, out):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
-    layer, x, logits = _case(rank, hot)
+    layer, x, logits = _case(rank, hot, empty_rank)
     k = 2
     b = EP.expert_bounds(layer.E, world)
     ops = OracleOps(layer, b[rank], b[rank + 1])
     moe = EP.ExpertParallelMoE(layer, k, ops=ops)
     got = moe.forward(torch.from_numpy(np.asarray(x, dtype=np.float64)), torch.from_numpy(logits))
-    ref = OL.moe_layer(layer, x, logits, k)["out"]
-    out[rank] = (float(np.abs(got.numpy() - ref).max()), float(np.abs(ref).max()), ops.expert_rows,
-                 int(x.shape[0]) * k)
+    ref = OL.moe_layer(layer, x, logits, k)["out"] if x.shape[0] else np.zeros((0, layer.D))
+    assert got.shape == ref.shape
+    out[rank] = (float(np.abs(got.numpy() - ref).max(initial=0.0)), float(np.abs(ref).max(initial=0.0)),
+                 ops.expert_rows, int(x.shape[0]) * k)
     dist.barrier()
     dist.destroy_process_group()
 
@@ -137,3 +138,15 @@ def test_owned_groups_keep_ids_and_arrays_together():
                 np.testing.assert_array_equal(g["s_down"][i], src.s_down[j])
                 seen.append(int(e))
     assert sorted(seen) == list(range(12))
+
+
+def test_rank_without_tokens_still_serves_its_experts():
+    # rank 0 holds no tokens this step but owns experts that rank 1's tokens use
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.spawn(_worker, args=(2, _free_port(), False, out, 0), nprocs=2, join=True)
+    assert out[0][3] == 0 and out[0][2] > 0          # no routes of its own, rows served
+    for rank in range(2):
+        err, scale, rows, routes = out[rank]
+        assert err <= 1e-12 * max(scale, 1.0), (rank, err, scale)
+    assert out[0][2] + out[1][2] == out[1][3]
