@@ -247,19 +247,46 @@ def expert_forward(weights: ExpertWeights, e: int, x_rot, down_rows=None, signs=
                 bound_y=abs_bound(Wd, h_rot), Wd=Wd)
 
 
-def _rot_abs(v) -> np.ndarray:
-    """Elementwise bound on |rotate(dv)| given |dv| <= v: per 128-chunk, sum / sqrt(128)."""
+def rot_abs_bound(v) -> np.ndarray:
+    """Elementwise bound on |rotate(dv)| given |dv| <= v elementwise: every output of a
+    128-chunk's orthonormal rotation is a +-1/sqrt(128) combination of that chunk's
+    inputs, so |rotate(dv)_j| <= (sum of v over j's chunk) / sqrt(128).  The bound is
+    attained at j by dv = v * (sign pattern of H_128's row j within the chunk)."""
     v = np.asarray(v, dtype=np.float64)
     n = v.shape[-1]
     chunk = v.reshape(v.shape[:-1] + (n // HADAMARD_N, HADAMARD_N)).sum(-1)
     return np.repeat(chunk, HADAMARD_N, axis=-1) / np.sqrt(float(HADAMARD_N))
 
 
+_rot_abs = rot_abs_bound
+
+
+SILU_D2_MAX = 0.5    # max |silu''(z)| (attained at z = 0)
+
+
+def swiglu_error_bound(g, u, dg, du) -> np.ndarray:
+    """Elementwise bound on |silu(g + a) * (u + b) - silu(g) * u| for |a| <= dg, |b| <= du.
+
+    silu(g + a) * (u + b) - silu(g) * u = (silu(g + a) - silu(g)) * (u + b) + silu(g) * b, and
+    by Taylor's theorem |silu(g + a) - silu(g)| <= |silu'(g)| dg + (max|silu''| / 2) dg^2, so
+    the change is at most (|silu'(g)| dg + 0.25 dg^2) (|u| + du) + |silu(g)| du."""
+    g, u = np.asarray(g, dtype=np.float64), np.asarray(u, dtype=np.float64)
+    dsilu = np.abs(silu_prime(g)) * dg + 0.5 * SILU_D2_MAX * dg * dg
+    return dsilu * (np.abs(u) + du) + np.abs(silu(g)) * du
+
+
 def e2e_error_bound(stage, eps_proj: float, w_abs):
-    """First-order bound on |out_gpu - out| of one route's contribution, given that each
-    projection meets |dy| <= eps_proj * (|W| . |input|) (h' rounding included); with
-    the two-sided transform the raw projections' errors are spread by their output
-    rotations (per 128-chunk: sum / sqrt(128)).
+    """First-order-exact bound on |out_gpu - out| of one route's contribution, given that
+    each projection meets |dy| <= eps_proj * (|W| . |input|) (h' rounding included).
+
+    The projection errors are carried through the layer stage by stage:
+      * gate/up: dg = eps * (|W_g| . |x'|), du likewise; with the two-sided transform the
+        raw projections' errors are spread by their output rotations (rot_abs_bound);
+      * SwiGLU: dh = swiglu_error_bound(g, u, dg, du);
+      * rotation of h: |d h'| <= rot_abs_bound(dh);
+      * down: its own budget applies to the perturbed input, eps * (|W_d| . (|h'| + |dh'|)), so
+        |dy| <= (1 + eps) |W_d| . rot_abs_bound(dh) + eps * (|W_d| . |h'|), spread by the down
+        projection's output rotation when two-sided.
 
     stage: the dict of ``expert_forward`` for that route's rows; w_abs: |route weight|.
     Returns the bound for the route's y scaled by its weight.
@@ -269,17 +296,12 @@ def e2e_error_bound(stage, eps_proj: float, w_abs):
     du = eps_proj * stage["bound_u"]
     if stage.get("two_sided"):
         # errors of the raw projections spread by their output rotation
-        dg, du = _rot_abs(dg), _rot_abs(du)
-    # |silu(g+dg)*(u+du) - silu(g)*u| <= |silu'(g)| dg |u| + (|silu(g)| + 1.1 dg) du
-    #                                    + 0.25 dg^2 |u|          (|silu''| <= 0.5)
-    dh = (np.abs(silu_prime(g)) * dg * np.abs(u)
-          + (np.abs(silu(g)) + 1.1 * dg) * du + 0.25 * dg * dg * np.abs(u))
-    n = dh.shape[-1]
-    chunk = dh.reshape(dh.shape[:-1] + (n // HADAMARD_N, HADAMARD_N)).sum(-1)
-    dh_rot = np.repeat(chunk, HADAMARD_N, axis=-1) / np.sqrt(float(HADAMARD_N))
-    dy = np.abs(dh_rot) @ np.abs(stage["Wd"]).T + eps_proj * stage["bound_y"]
+        dg, du = rot_abs_bound(dg), rot_abs_bound(du)
+    dh = swiglu_error_bound(g, u, dg, du)
+    dh_rot = rot_abs_bound(dh)
+    dy = (1.0 + eps_proj) * (dh_rot @ np.abs(stage["Wd"]).T) + eps_proj * stage["bound_y"]
     if stage.get("two_sided"):
-        dy = _rot_abs(dy)
+        dy = rot_abs_bound(dy)
         if stage.get("down_rows") is not None:
             pos = {int(r): i for i, r in enumerate(stage["rows"])}
             dy = dy[:, [pos[int(r)] for r in stage["down_rows"]]]
