@@ -352,12 +352,16 @@ int moe_trellis_gemv(const tq_moe_layer *layer, const uint16_t *x_rot, const int
  *   bytes plus 8 bytes per row (T <= 36 at k = 8, D = 4096, F = 1024), must fit in it;
  *   larger calls return TQ_ERR_WORKSPACE without doing anything.
  *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   Arguments are checked first, with the same statuses as moe_trellis_gemv; then a call
+ *   whose workspace would not fit returns TQ_ERR_WORKSPACE.
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- *   once per device, with that device current); make that first call before any stream
- *   capture.  Every call on a device shares the one array and it keeps the last call's
- *   contents; each call writes every workspace byte it reads before reading it, so
- *   nothing needs clearing, but calls that overlap on the GPU (other streams, other
- *   threads) race on the array and must be serialised by the caller.
+ *   once per device, with that device current) and keeps it for the life of the
+ *   context: make that first call before any stream capture, and reload the library
+ *   after a cudaDeviceReset.  Every call on a device shares the one array and it keeps
+ *   the last call's contents; each call writes every workspace byte it reads before
+ *   reading it, so nothing needs clearing, but calls that overlap on the GPU (other
+ *   streams, other threads) race on the array and must be serialised by the caller.
+ *   The results are those of moe_trellis_gemv bit for bit.
  */
 int moe_trellis_gemv_noalloc(const tq_moe_layer *layer, const uint16_t *x_rot,
                              const int32_t *offsets, const int32_t *perm, const int32_t *active_ids,

@@ -3,10 +3,13 @@ memory at call time (fixed-pool runtimes, plugin or sandboxed engines, allocatio
 latency paths) -- against moe_trellis_gemv with a caller-provided workspace.
 
 Two calls in a row on different tokens and routes: the second call runs on scratch
-still holding the first call's contents.  Each result must agree with the existing
-entry point's within the tolerance the MoE parity tests use (the oracle's error bound
-of the composed layer), and the host-side size check must reject calls beyond the
-compiled-in scratch.  Collected last so that a stop at the first failure has already
+still holding the first call's contents.  Both entry points run the same kernels on the
+same inputs, so each result must equal the workspace entry point's bit for bit (a stale
+scratch read would show up here even when it stays within the error bound); each is also
+checked against the oracle within the tolerance the MoE parity tests use (the oracle's
+error bound of the composed layer).  The host-side checks must reject calls beyond the
+compiled-in scratch, and report bad arguments with the same status as the workspace
+entry point.  Collected last so that a stop at the first failure has already
 run every other test; self-contained so it also passes alone in a fresh process.
 """
 import numpy as np
@@ -59,10 +62,10 @@ def test_noalloc_matches_workspace_entry_point_twice(api):
         res = OL.moe_layer(layer, x, logits, k)
         tol = res["bound"] + 1e-6 * np.abs(res["out"]) + 1e-12
         assert np.isfinite(got).all(), "call %d" % call
-        err = np.abs(got - ref_gpu)
+        np.testing.assert_array_equal(got, ref_gpu, err_msg="call %d" % call)
+        # and against the oracle itself
+        err = np.abs(got - res["out"])
         assert np.all(err <= tol), "call %d: max err/tol %.3e" % (call, (err / tol).max())
-        # and both against the oracle itself
-        assert np.all(np.abs(got - res["out"]) <= tol), "call %d" % call
     assert api.device_status() == 0
 
 
@@ -75,3 +78,19 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(api):
     y = torch.empty((T * k, 256), dtype=torch.float32, device="cuda")
     with pytest.raises(api.TQError, match="WORKSPACE"):
         api.moe_trellis_gemv_noalloc(dl, x_rot, routing, T, k, y)
+
+
+def test_noalloc_reports_bad_arguments_like_the_workspace_entry_point(api):
+    # k > E is an invalid argument for both entry points, even when the call would also
+    # be too large for the scratch
+    layer = inputs.small_layer(5, E=12, D=256, F=128)
+    dl = api.DeviceLayer.from_synthetic(layer)
+    T, k = 6000, 13
+    x_rot = torch.zeros((T, 256), dtype=torch.float16, device="cuda")
+    routing = api.Routing.empty(T, k, 12, "cuda")
+    y = torch.empty((T * k, 256), dtype=torch.float32, device="cuda")
+    with pytest.raises(api.TQError, match="INVALID_ARG"):
+        api.moe_trellis_gemv_noalloc(dl, x_rot, routing, T, k, y)
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(api.TQError, match="INVALID_ARG"):
+        api.moe_trellis_gemv(dl, x_rot, routing, T, k, y, ws)

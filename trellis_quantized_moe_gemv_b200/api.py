@@ -461,9 +461,13 @@ def moe_trellis_gemv(layer, x_rot, routing, T, k, y_perm=None, ws=None, stream=N
 
 def moe_trellis_gemv_noalloc(layer: DeviceLayer, x_rot: torch.Tensor, routing: Routing, T: int, k: int,
                              y_perm: torch.Tensor, stream=None) -> torch.Tensor:
-    """moe_trellis_gemv with the library's own fixed scratch array instead of a workspace,
-    for callers that cannot allocate device memory at call time.  y_perm ([T*k, D] fp32)
-    must be provided; the call itself allocates nothing.  At most T*k*F = 699,050."""
+    """moe_trellis_gemv with the library's own fixed 4 MiB scratch array instead of a
+    workspace, for callers that cannot allocate device memory at call time.  y_perm
+    ([T*k, D] fp32) must be provided; the call itself allocates nothing.  The call must
+    fit the scratch: the GEMV workspace, moe_trellis_gemv's share of
+    moe_trellis_workspace_size (12*T*k*F + 4*T*D bytes plus 8 per row, each part rounded
+    up to 256 bytes), at most 4 MiB -- T <= 36 at k = 8, D = 4096, F = 1024.  Larger calls
+    raise TQError (TQ_ERR_WORKSPACE)."""
     _require(x_rot, torch.float16, "x_rot")
     _require(y_perm, torch.float32, "y_perm")
     _check(_fn("moe_trellis_gemv_noalloc")(ctypes.byref(layer.struct), _p(x_rot), _p(routing.offsets),

@@ -816,9 +816,10 @@ TQ_API size_t moe_trellis_workspace_size(const tq_moe_layer *layer, int T, int k
     return gemv > gemm ? gemv : gemm;
 }
 
-int moe_validate_call(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
+// Every argument of a MoE call except the workspace.
+int moe_validate_args(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
                       const int32_t *perm, const int32_t *active_ids, const int32_t *n_active, int T,
-                      int k, float *y_perm, void *ws, size_t ws_bytes) {
+                      int k, float *y_perm) {
     int st = validate_layer(layer);
     if (st) return st;
     if (T < 0 || k < 1 || k > layer->E) return TQ_ERR_INVALID_ARG;
@@ -826,6 +827,14 @@ int moe_validate_call(const tq_moe_layer *layer, const uint16_t *x_rot, const in
     if (T == 0) return TQ_OK;
     if (!x_rot || !offsets || !perm || !active_ids || !n_active || !y_perm) return TQ_ERR_INVALID_ARG;
     if (!aligned16(x_rot) || !aligned16(y_perm)) return TQ_ERR_ALIGNMENT;
+    return TQ_OK;
+}
+
+int moe_validate_call(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
+                      const int32_t *perm, const int32_t *active_ids, const int32_t *n_active, int T,
+                      int k, float *y_perm, void *ws, size_t ws_bytes) {
+    int st = moe_validate_args(layer, x_rot, offsets, perm, active_ids, n_active, T, k, y_perm);
+    if (st || T == 0) return st;
     if (!ws || ws_bytes < workspace_bytes(layer, T, k)) return TQ_ERR_WORKSPACE;
     if (!aligned16(ws)) return TQ_ERR_ALIGNMENT;
     return TQ_OK;

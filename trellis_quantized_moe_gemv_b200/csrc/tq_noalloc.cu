@@ -9,6 +9,8 @@
 // workspace from a fixed array compiled into the library instead.
 #include "tq_common.cuh"
 
+#include <atomic>
+
 namespace tq {
 
 // Scratch for the GEMV's workspace (gate/up partial sums, quantised h' and x'): at most
@@ -19,20 +21,25 @@ constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kNoAllocMaxDevices = 64;
-static void *g_noalloc_ptr[kNoAllocMaxDevices];
+static std::atomic<void *> g_noalloc_ptr[kNoAllocMaxDevices];
 
-// Device address of the scratch array on the current device; looked up once per
-// device (the array's name is only a host-side stand-in in host code).
+// Device address of the scratch array on the current device (in host code the array's
+// name is only a host-side stand-in, never a device address).  Looked up once per
+// device, by the first call with that device current, and kept for the life of the
+// process's context on that device: after cudaDeviceReset the library must be
+// reloaded before this entry point is called again.  Threads that race on the first
+// lookup all store the same address.
 static int noalloc_scratch(void **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess) return record_cuda_error("cudaGetDevice");
     if (dev < 0 || dev >= kNoAllocMaxDevices) return TQ_ERR_UNSUPPORTED;
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return TQ_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+    void *p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+            return record_cuda_error("cudaGetSymbolAddress");
+        g_noalloc_ptr[dev].store(p, std::memory_order_release);
     }
-    *out = g_noalloc_ptr[dev];
+    *out = p;
     return TQ_OK;
 }
 
@@ -42,24 +49,20 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
 
 }  // namespace tq
 
-int moe_validate_call(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
+int moe_validate_args(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
                       const int32_t *perm, const int32_t *active_ids, const int32_t *n_active, int T,
-                      int k, float *y_perm, void *ws, size_t ws_bytes);
+                      int k, float *y_perm);
 
 TQ_API int moe_trellis_gemv_noalloc(const tq_moe_layer *layer, const uint16_t *x_rot,
                                     const int32_t *offsets, const int32_t *perm,
                                     const int32_t *active_ids, const int32_t *n_active, int T, int k,
                                     float *y_perm, tq_stream stream) {
-    const int valid = tq::validate_layer(layer);
-    if (valid != TQ_OK) return valid;
-    if (T < 0 || k < 1) return TQ_ERR_INVALID_ARG;
-    if (T == 0) return TQ_OK;
+    // the same argument statuses as moe_trellis_gemv, then the size of the call
+    int st = moe_validate_args(layer, x_rot, offsets, perm, active_ids, n_active, T, k, y_perm);
+    if (st || T == 0) return st;
     if (tq::workspace_bytes(layer, T, k) > tq::kNoAllocScratchBytes) return TQ_ERR_WORKSPACE;
     void *scratch = nullptr;
-    int st = tq::noalloc_scratch(&scratch);
-    if (st) return st;
-    st = moe_validate_call(layer, x_rot, offsets, perm, active_ids, n_active, T, k, y_perm, scratch,
-                           tq::kNoAllocScratchBytes);
+    st = tq::noalloc_scratch(&scratch);
     if (st) return st;
     return tq::run_moe_gemv(layer, reinterpret_cast<const __half *>(x_rot), offsets, perm, active_ids,
                             n_active, T, k, y_perm, scratch, (cudaStream_t)stream);
