@@ -75,9 +75,10 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 32768, FAKE, 1, FAKE, FAKE, big, None) == 2  # cols
     assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 128, FAKE, 70000, FAKE, FAKE, big, None) == 2
     assert lib.trellis_gemv(FAKE, FAKE, 2, 16, 128, FAKE, 0, FAKE, None, 0, None) == 0
-    # workspace: quantised rows (two half-words per value), 8 bytes per row, 8 per output
+    # workspace: quantised rows (four half-word planes: the main word and the residual
+    # word, high and low bytes), 16 bytes of metadata per row, 16 bytes per output
     need = lib.trellis_gemv_workspace_size(32, 256, 3)
-    assert need == 3 * 2 * 256 * 2 + 256 + 32 * 3 * 8
+    assert need == 3 * 4 * 256 * 2 + 256 + 32 * 3 * 16
     assert lib.trellis_gemv(FAKE, FAKE, 2, 32, 256, FAKE, 3, FAKE, FAKE, ctypes.c_size_t(need - 1),
                             None) == 4
     assert lib.trellis_gemv(FAKE, FAKE, 2, 32, 256, FAKE, 3, FAKE, MISALIGNED, ctypes.c_size_t(need),
@@ -117,12 +118,13 @@ def _layer_struct(K=2, E=16, D=256, F=128, n_groups=1):
 def test_moe_workspace_and_layer_validation(lib):
     st = _layer_struct()
     need = lib.moe_trellis_workspace_size(ctypes.byref(st), 16, 8)
-    # GEMV: per-route gate and up results (fp32), h' and x' as 16-bit fixed point (two
-    # half-words per value) and their per-row (exponent, sum)
-    gemv_need = 128 * 2 * 128 * 4 + 128 * 2 * 128 * 2 + 128 * 8 + 16 * 2 * 256 * 2 + 256
-    # the GEMM path also holds route-ordered activations (fp16), their row sums, h, h'
-    # and its tile list
-    gemm_need = 128 * 256 * 2 + 512 + 128 * 128 * 4 + 128 * 128 * 2 + 512 + 256
+    # GEMV: per-route gate and up results (fp32; this layer's 16 experts x 2 items get 2
+    # column splits: min(8, ceil(3 * SMs / 32), D / 128)), h' and x' as fixed point (four
+    # half-word planes per value: main and residual word) and 16 bytes of metadata per row
+    gemv_need = 128 * 2 * 2 * 128 * 4 + 128 * 4 * 128 * 2 + 128 * 16 + 16 * 4 * 256 * 2 + 256
+    # the GEMM path also holds route-ordered activations (fp16), their row sums, h, h',
+    # its row sums and power-of-two row scales, and the tile list
+    gemm_need = 128 * 256 * 2 + 512 + 128 * 128 * 4 + 128 * 128 * 2 + 512 + 512 + 256
     assert need == max(gemv_need, gemm_need)
     bad = _layer_struct(K=5)
     assert lib.moe_trellis_workspace_size(ctypes.byref(bad), 16, 8) == 0

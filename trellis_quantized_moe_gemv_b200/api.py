@@ -465,9 +465,9 @@ def moe_trellis_gemv_noalloc(layer: DeviceLayer, x_rot: torch.Tensor, routing: R
     workspace, for callers that cannot allocate device memory at call time.  y_perm
     ([T*k, D] fp32) must be provided; the call itself allocates nothing.  The call must
     fit the scratch: the GEMV workspace, moe_trellis_gemv's share of
-    moe_trellis_workspace_size (12*T*k*F + 4*T*D bytes plus 8 per row, each part rounded
-    up to 256 bytes), at most 4 MiB -- T <= 36 at k = 8, D = 4096, F = 1024.  Larger calls
-    raise TQError (TQ_ERR_WORKSPACE)."""
+    moe_trellis_workspace_size (include/trellis_moe.h gives the byte formula), at most
+    4 MiB -- T <= 25 at k = 8, D = 4096, F = 1024.  Larger calls raise TQError
+    (TQ_ERR_WORKSPACE)."""
     _require(x_rot, torch.float16, "x_rot")
     _require(y_perm, torch.float32, "y_perm")
     _check(_fn("moe_trellis_gemv_noalloc")(ctypes.byref(layer.struct), _p(x_rot), _p(routing.offsets),
@@ -497,7 +497,7 @@ class MoeBuffers:
                               device=dev)
 
 
-GEMM_MIN_TOKENS = 392   # measured crossover of the two paths on the 384-expert decode layer
+GEMM_MIN_TOKENS = 360   # measured crossover of the two paths on the 384-expert decode layer
 
 
 def moe_layer(layer: DeviceLayer, x: torch.Tensor, logits: torch.Tensor, k: int,

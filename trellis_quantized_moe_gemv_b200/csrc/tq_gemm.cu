@@ -19,7 +19,10 @@
 //       - one thread issues 4 tcgen05.mma (M=128, N<=256, K=16, fp32 accumulator in
 //         tensor memory) and commits them to the stage's "empty" barrier.
 //   * Epilogue (4 warps, one per tensor-memory lane quarter): tcgen05.ld of the
-//     accumulator, D -> s * 2^-12 * (2^24 D - 255 * rowsum), then
+//     accumulator, D -> s * 2^-12 * (2^24 D - 255 * rowsum), times the route row's
+//     power-of-two scale for the down projection (h' rows are stored as fp16 h' / 2^e,
+//     largest magnitude in [2^14, 2^15), so any finite fp32 h keeps fp16's relative
+//     precision and never overflows), then
 //       gate/up: strips are interleaved gate/up per 16 rows, so lane l and l^16 hold g
 //                and u of the same intermediate row: h = silu(g) * u (fp32);
 //       down:    y_perm (fp32).
@@ -65,10 +68,14 @@ struct __align__(1024) GemmSmem {
     uint64_t kb_done[kGKbRing];
     uint64_t acc_full;                         // MMA -> epilogue
     uint64_t mma_done;                         // MMA drain on early exit
-    float rs[kGDecodeWarps][kGBN / 2];         // epilogue: each decode warp's route row sums
+    float2 rs[kGDecodeWarps][kGBN / 2];        // epilogue: each decode warp's route (row sum, scale)
     uint32_t tmem_base;
     int32_t abort;                             // a role gave up
 };
+
+// dynamic shared memory of one CTA (plus 1 KB for the 1024-byte alignment) must fit the
+// 227 KB a CTA may use on sm_100
+static_assert(sizeof(GemmSmem) + 1024 <= 227 * 1024, "GEMM shared memory exceeds the per-CTA limit");
 
 struct GemmMaps {
     CUtensorMap b[kGBoxes];               // route-ordered activations, box rows 32..256
@@ -254,6 +261,7 @@ struct GemmArgs {
     const int32_t *offsets;
     const int32_t *tiles;        // [0] = count, then (expert, first route) pairs
     const float *rowsum;         // [T*k] sum of each route's activation row
+    const float *rowscale;       // [T*k] power-of-two scale of each route's row, or null (1)
     float *out;                  // gate/up: h [T*k][F] (raw_gu: g, u [T*k][2][F]); down: y [T*k][D]
     int kdim;                    // D (gate/up) or F (down)
     int raw_gu;                  // gate/up of the two-sided transform: store g and u, not h
@@ -427,10 +435,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int mtile = mt * kGTiles + tt;
             const int half_cols = ((nmma / 16 + 1) / 2) * 16;
             const int cb = slot * half_cols, ce = min(nmma, cb + half_cols);
-            float *rsw = sm.rs[warp - kGFirstDecodeWarp];
+            float2 *rsw = sm.rs[warp - kGFirstDecodeWarp];
             for (int i = lane; i < ce - cb; i += 32) {
                 const int col = cb + i;
-                rsw[i] = col < n ? args.rowsum[r0 + n0 + col] : 0.f;
+                float2 v = make_float2(0.f, 1.f);
+                if (col < n) {
+                    v.x = args.rowsum[r0 + n0 + col];
+                    if (args.rowscale) v.y = args.rowscale[r0 + n0 + col];
+                }
+                rsw[i] = v;
             }
             const int f = (mtile * 4 + q) * 16 + (lane & 15);
             const int hi = lane >> 4;
@@ -448,7 +461,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 for (int c0 = cb; c0 < ce; c0 += 16) {
                     uint32_t v[16];
                     tmem_ld16(taddr + c0, v);
-                    const float *rsc = rsw + (c0 - cb);
+                    const float2 *rsc = rsw + (c0 - cb);
                     if (GATEUP) {
                         // lane l < 16 holds the gate row of output f, lane l + 16 the up row;
                         // one exchange per column pair gives lane l both values of column c
@@ -461,7 +474,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                             const int col = c0 + c + hi;
                             if (col < n) {
                                 const int route = r0 + n0 + col;
-                                const float sx = rsc[c + hi];
+                                const float sx = rsc[c + hi].x;
                                 const float g = sk0 * fmaf(16777216.0f, graw, -255.0f * sx);
                                 const float u = sk1 * fmaf(16777216.0f, uraw, -255.0f * sx);
                                 if (args.raw_gu) {
@@ -479,7 +492,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                             const int col = c0 + c;
                             if (col < n)
                                 args.out[(size_t)(r0 + n0 + col) * L.D + d] =
-                                    sk0 * fmaf(16777216.0f, __uint_as_float(v[c]), -255.0f * rsc[c]);
+                                    (sk0 * rsc[c].y) * fmaf(16777216.0f, __uint_as_float(v[c]), -255.0f * rsc[c].x);
                         }
                     }
                 }
@@ -499,27 +512,49 @@ __global__ void __launch_bounds__(kGThreads, 1)
 // Route-ordered fp16 activation rows, one warp per destination row j: the source row is
 // perm[j] / k (the token of grouped route j) or j itself when perm is null; ROTATE
 // applies the 128-wide rotation on the way.  rowsum[j] = fp32 sum of the stored fp16
-// values.  An out-of-range source raises device flag bit 0 and stores zeros.
+// values.  With rowscale (the rotated h rows of the down projection) the row is stored
+// as v / 2^e, 2^e = rowscale[j] chosen so that its largest magnitude lies in
+// [2^14, 2^15) (2^e = 1 for a zero row, 2^e >= 2^-112); the row is read twice.  An out-of-range source
+// raises device flag bit 0 and stores zeros.
 template <typename T, bool ROTATE>
 __global__ void __launch_bounds__(256) route_rows_kernel(const T *__restrict__ x, int dst_rows, int cols,
                                                          const int32_t *__restrict__ perm, int k, int src_rows,
-                                                         __half *__restrict__ dst, float *__restrict__ rowsum) {
+                                                         __half *__restrict__ dst, float *__restrict__ rowsum,
+                                                         float *__restrict__ rowscale) {
     const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (j >= dst_rows) return;
     const int src = perm ? perm[j] / k : j;
     const bool valid = src >= 0 && src < src_rows && (!perm || perm[j] >= 0);
     if (!valid && lane == 0) raise_flag(1);
-    float sum = 0.f;
-    for (int c = 0; c < cols; c += 128) {
-        float v[4] = {0.f, 0.f, 0.f, 0.f};
+    auto load = [&](int c, float (&v)[4]) {
+        v[0] = v[1] = v[2] = v[3] = 0.f;
         if (valid) {
             float4 f = load4<T>(x + (size_t)src * cols + c + 4 * lane);
             v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
             if (ROTATE) fwht128_warp(v, lane);
         }
-        __half2 lo = __floats2half2_rn(v[0], v[1]);
-        __half2 hi = __floats2half2_rn(v[2], v[3]);
+    };
+    float inv_scale = 1.f;
+    if (rowscale) {
+        float m = 0.f;
+        for (int c = 0; c < cols; c += 128) {
+            float v[4];
+            load(c, v);
+            m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fmaxf(fabsf(v[2]), fabsf(v[3])), m));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const int e = m > 0.f ? max(ilogbf(m) - 14, -112) : 0;   // 2^e and 2^-e stay normal
+        inv_scale = ldexpf(1.f, -e);
+        if (lane == 0) rowscale[j] = ldexpf(1.f, e);
+    }
+    float sum = 0.f;
+    for (int c = 0; c < cols; c += 128) {
+        float v[4];
+        load(c, v);
+        __half2 lo = __floats2half2_rn(v[0] * inv_scale, v[1] * inv_scale);
+        __half2 hi = __floats2half2_rn(v[2] * inv_scale, v[3] * inv_scale);
         const float2 lf = __half22float2(lo), hf = __half22float2(hi);
         sum += (lf.x + lf.y) + (hf.x + hf.y);
         uint2 u;
@@ -534,19 +569,20 @@ __global__ void __launch_bounds__(256) route_rows_kernel(const T *__restrict__ x
 
 // The two-sided transform between the gate/up and down GEMMs, one warp per route row j:
 // g = sign_gu * rotate(g), u likewise (the output side of gate and up), h = silu(g) * u,
-// h' = rotate(sign_h * h) (the input side of down), stored fp16 with its fp32 row sum.
+// h' = rotate(sign_h * h) (the input side of down), stored fp16 as h' / rowscale[j] (the
+// power of two that puts the row's largest magnitude in [2^14, 2^15)) with the fp32 sum
+// of the stored values.  The row is computed twice (its maximum first).
 __global__ void __launch_bounds__(256) swiglu_rows_kernel(const float *__restrict__ gu, int rows, int F,
                                                           const int8_t *__restrict__ sign_gu,
                                                           const int8_t *__restrict__ sign_h, __half *__restrict__ dst,
-                                                          float *__restrict__ rowsum) {
+                                                          float *__restrict__ rowsum, float *__restrict__ rowscale) {
     const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (j >= rows) return;
-    float sum = 0.f;
-    for (int c = 0; c < F; c += 128) {
+    auto row_chunk = [&](int c, float (&h)[4]) {
         const float4 g4 = load4<float>(gu + (size_t)j * 2 * F + c + 4 * lane);
         const float4 u4 = load4<float>(gu + ((size_t)j * 2 + 1) * F + c + 4 * lane);
-        float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w}, h[4];
+        float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w};
         fwht128_warp(g, lane);
         fwht128_warp(u, lane);
         const char4 so = *reinterpret_cast<const char4 *>(sign_gu + c + 4 * lane);
@@ -556,8 +592,24 @@ __global__ void __launch_bounds__(256) swiglu_rows_kernel(const float *__restric
 #pragma unroll
         for (int i = 0; i < 4; ++i) h[i] = silu_f32(g[i] * o[i]) * (u[i] * o[i]) * in[i];
         fwht128_warp(h, lane);
-        __half2 lo = __floats2half2_rn(h[0], h[1]);
-        __half2 hi = __floats2half2_rn(h[2], h[3]);
+    };
+    float m = 0.f;
+    for (int c = 0; c < F; c += 128) {
+        float h[4];
+        row_chunk(c, h);
+        m = fmaxf(fmaxf(fabsf(h[0]), fabsf(h[1])), fmaxf(fmaxf(fabsf(h[2]), fabsf(h[3])), m));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int e = m > 0.f ? max(ilogbf(m) - 14, -112) : 0;   // 2^e and 2^-e stay normal
+    const float inv_scale = ldexpf(1.f, -e);
+    if (lane == 0) rowscale[j] = ldexpf(1.f, e);
+    float sum = 0.f;
+    for (int c = 0; c < F; c += 128) {
+        float h[4];
+        row_chunk(c, h);
+        __half2 lo = __floats2half2_rn(h[0] * inv_scale, h[1] * inv_scale);
+        __half2 hi = __floats2half2_rn(h[2] * inv_scale, h[3] * inv_scale);
         const float2 lf = __half22float2(lo), hf = __half22float2(hi);
         sum += (lf.x + lf.y) + (hf.x + hf.y);
         uint2 w;
@@ -690,7 +742,8 @@ size_t gemm_workspace_bytes(const tq_moe_layer *L, int T, int k) {
     const size_t hcols = L->sign_gu ? 2 : 1;   // two-sided: g and u, else h
     return align256_g(R * L->D * sizeof(__half)) + align256_g(R * sizeof(float)) +
            align256_g(R * hcols * L->F * sizeof(float)) + align256_g(R * L->F * sizeof(__half)) +
-           align256_g(R * sizeof(float)) + align256_g((1 + 2 * (size_t)gemm_max_tiles(T, k, L->E)) * sizeof(int32_t));
+           align256_g(R * sizeof(float)) + align256_g(R * sizeof(float)) +
+           align256_g((1 + 2 * (size_t)gemm_max_tiles(T, k, L->E)) * sizeof(int32_t));
 }
 
 int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offsets, const int32_t *perm,
@@ -719,6 +772,8 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     w += align256_g((size_t)R * L->F * sizeof(__half));
     float *shr = reinterpret_cast<float *>(w);
     w += align256_g((size_t)R * sizeof(float));
+    float *scr = reinterpret_cast<float *>(w);   // power-of-two scale of each h' row
+    w += align256_g((size_t)R * sizeof(float));
     int32_t *tiles = reinterpret_cast<int32_t *>(w);
     const int max_tiles = gemm_max_tiles(T, k, L->E);
 
@@ -742,12 +797,13 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     {
         // x_rot is already rotated: copy its rows to their route rows (+ row sums)
         LaunchScope ls(s, kStageGemmPrep);
-        route_rows_kernel<__half, false><<<(R * 32 + 255) / 256, 256, 0, s>>>(x_rot, R, L->D, perm, k, T, xp, sxp);
+        route_rows_kernel<__half, false><<<(R * 32 + 255) / 256, 256, 0, s>>>(x_rot, R, L->D, perm, k, T, xp, sxp,
+                                                                             nullptr);
     }
     st = launch_status();
     if (st) return st;
     {
-        GemmArgs a{*L, offsets, tiles, sxp, h, L->D, two};
+        GemmArgs a{*L, offsets, tiles, sxp, nullptr, h, L->D, two};
         LaunchScope ls(s, kStageGemmGateUp);
         moe_gemm_kernel<true><<<dim3(L->F / (64 * kGTiles), max_tiles), kGThreads, smem, s>>>(maps_x, a);
     }
@@ -756,14 +812,15 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     {
         LaunchScope ls(s, kStageRotateH);
         if (two)
-            swiglu_rows_kernel<<<(R * 32 + 255) / 256, 256, 0, s>>>(h, R, L->F, L->sign_gu, L->sign_h, hr, shr);
+            swiglu_rows_kernel<<<(R * 32 + 255) / 256, 256, 0, s>>>(h, R, L->F, L->sign_gu, L->sign_h, hr, shr, scr);
         else
-            route_rows_kernel<float, true><<<(R * 32 + 255) / 256, 256, 0, s>>>(h, R, L->F, nullptr, 1, R, hr, shr);
+            route_rows_kernel<float, true><<<(R * 32 + 255) / 256, 256, 0, s>>>(h, R, L->F, nullptr, 1, R, hr, shr,
+                                                                                scr);
     }
     st = launch_status();
     if (st) return st;
     {
-        GemmArgs a{*L, offsets, tiles, shr, y_perm, L->F, 0};
+        GemmArgs a{*L, offsets, tiles, shr, scr, y_perm, L->F, 0};
         LaunchScope ls(s, kStageGemmDown);
         moe_gemm_kernel<false><<<dim3(L->D / (kGBM * kGTiles), max_tiles), kGThreads, smem, s>>>(maps_h, a);
     }

@@ -12,7 +12,10 @@
 //     x_q = round(x / 2^e), |x_q| <= 32639, split into two signed bytes
 //     x_q = 256 xh + xl (xl in [-128, 127]).  quantize_rows_kernel writes each byte
 //     twice into a half-word (one row of xh half-words, one of xl half-words) and e
-//     and sum_j x_q of every row.
+//     and sum_j x_q of every row.  A row whose rounding step is coarse for its mass
+//     (2^(e-1) * cols > 2^-12 * sum_j |x_j|: a few elements dominate) also gets a second
+//     word, the residual x - x_q 2^e as 16-bit fixed point at 2^(e-15), so such a row is
+//     32-bit fixed point; its two words take two MMA column pairs ("slots").
 //   * A warp walks 8 strips (16 output rows each): lane group g = lane/4 owns strip g
 //     and lane t = lane%4 owns columns 4t..4t+3 of each tile, so every lane decodes the
 //     same tile-relative bit offsets (compile-time shifts).
@@ -21,10 +24,12 @@
 //     lo/hi the two bytes of (window * 0x3A2F) mod 2^16.  One A register is one weight
 //     spread over 4 k-slots; its two zero slots meet whatever the activation word holds
 //     there, so the MMA adds (lo + hi) * x = t * x with no byte shuffling.
-//   * The MMA's 8 columns are 4 routes x 2 limbs (column 2r: route r's xh, 2r+1: its
-//     xl).  |partial sums| <= 510 * 128 * cols < 2^31 for cols <= 16384.
+//   * The MMA's 8 columns are 4 slots x 2 limbs (column 2r: slot r's xh, 2r+1: its
+//     xl); a slot holds one word of one route.  |partial sums| <= 510 * 128 * cols <
+//     2^31 for cols <= 16384.
 //   * Epilogue, in double: y = s * 2^-12 * 2^e * (256 H + L - 255 sum_j x_q), H and L
-//     the two limb sums; sum_j c_j x_j = sum_j t_j x_j - 255 sum_j x_j.
+//     the two limb sums (sum_j c_j x_j = sum_j t_j x_j - 255 sum_j x_j), plus
+//     2^(e-15) * (256 H' + L' - 255 sum_j r_q) from the residual slot of a two-word row.
 //   * Bit streams reach shared memory by bulk copies into a per-warp ring of stages
 //     (one mbarrier per stage, bounded waits); activations come from L2, one tile
 //     ahead.
@@ -34,6 +39,17 @@ namespace tq {
 
 constexpr int kMaxCols = 16384;        // keeps every int32 partial sum in range
 constexpr int kQMax = 32639;           // 127 * 256 + 127: both bytes stay signed
+constexpr int kResShift = 15;          // residual word scale: 2^(e - 15)
+constexpr int kResBudgetLog2 = 12;     // second word when 2^(e-1) * cols > 2^-12 * sum |x|
+
+// Fixed-point activation row: x ~ x_q 2^e (+ r_q 2^(e - kResShift) when res != 0).
+// Planes of a row in memory: [0] xh half-words, [1] xl, [2] rh, [3] rl (cols each).
+struct __align__(16) RowQ {
+    int e;        // power of two of the main word
+    int sum;      // sum_j x_q
+    int res;      // 1: the row carries the residual word
+    int rsum;     // sum_j r_q
+};
 constexpr int kItemWarps = 4;
 constexpr int kItemThreads = kItemWarps * 32;
 constexpr int kStages = 2;
@@ -257,10 +273,18 @@ __device__ __forceinline__ int2 red_sum(const ItemRed<NB> &red, int strip, int r
     return make_int2(h, l);
 }
 
-// y = s * 2^-12 * 2^e * (256 H + L - 255 sum x_q), formed in double.
-__device__ __forceinline__ float finish_q(int H, int L, int2 meta, float scale) {
-    const double a = 256.0 * (double)H + (double)L - 255.0 * (double)meta.y;
-    return (float)(a * ldexp((double)scale * (double)kKappa, meta.x));
+// y = s * 2^-12 * 2^e * (256 H + L - 255 sum x_q), formed in double (the integer part
+// and the scale are exact doubles, so the result is rounded once to double and once to
+// float).  A two-word row adds its residual sums (H2, L2) at 2^-15 of the main word's
+// scale: 2^15 a + a2 stays below 2^53 for cols <= 16384, so it is exact too.
+__device__ __forceinline__ float finish_q(int H, int L, const RowQ &q, float scale, int H2 = 0, int L2 = 0) {
+    double a = 256.0 * (double)H + (double)L - 255.0 * (double)q.sum;
+    int e = q.e;
+    if (q.res) {
+        a = a * (double)(1 << kResShift) + (256.0 * (double)H2 + (double)L2 - 255.0 * (double)q.rsum);
+        e -= kResShift;
+    }
+    return (float)(a * ldexp((double)scale * (double)kKappa, e));
 }
 
 __device__ __forceinline__ void split_range(int n, int part, int parts, int &b, int &e) {
@@ -273,12 +297,14 @@ __device__ __forceinline__ void split_range(int n, int part, int parts, int &b, 
 //
 // One CTA of 8 warps per row of `cols` values (a multiple of 128): take the row from
 // its source (optionally rotating every 128-chunk with fwht128_warp, the hadamard128
-// transform), take max |v| over the row, pick e with max / 2^e <= 32639
+// transform), take max |v| and sum |v| over the row, pick e with max / 2^e <= 32639
 // (e = ilogb(max) - 14, one more if the mantissa is too large), and write
 // x_q = rint(v / 2^e) as its two signed bytes, each held twice in a half-word:
-// xq[row][0][col] = xh * 0x0101, xq[row][1][col] = xl * 0x0101.
-// meta[row] = (e, sum_j x_q).  The row is read again in the second pass instead of
-// being kept in registers, so any row length works.
+// xq[row][0][col] = xh * 0x0101, xq[row][1][col] = xl * 0x0101.  When
+// 2^(e-1) * cols > 2^-12 * sum |v| the row also gets its residual word
+// r_q = rint((v - x_q 2^e) / 2^(e-15)) (|r_q| <= 2^14; v - x_q 2^e is exact in fp32) in
+// planes 2 and 3.  meta[row] = (e, sum x_q, residual flag, sum r_q).  The row is read
+// again in the second pass instead of being kept in registers, so any row length works.
 
 // Plain rows x[row][cols].
 template <typename T>
@@ -327,15 +353,13 @@ struct SwigluSrc {
 
 template <typename Src, bool ROTATE>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int cols, const int8_t *__restrict__ signs,
-                                                            uint16_t *__restrict__ xq, int2 *__restrict__ meta) {
+                                                            uint16_t *__restrict__ xq, RowQ *__restrict__ meta) {
     chain_entry();
-    __shared__ float s_max[8];
-    __shared__ int s_sum[8];
+    __shared__ float s_max[8], s_l1[8];
+    __shared__ int s_sum[8], s_rsum[8];
     const int row = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int chunks = cols / 128;
-    float m = 0.f;
-    for (int c = warp; c < chunks; c += 8) {
-        float v[4];
+    auto load = [&](int c, float (&v)[4]) {
         src.load(row, c, lane, v);
         if constexpr (ROTATE) {
             if (signs) {   // input side of the two-sided transform: rotate(signs * v)
@@ -344,34 +368,47 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int c
             }
             fwht128_warp(v, lane);
         }
+    };
+    float m = 0.f, l1 = 0.f;
+    for (int c = warp; c < chunks; c += 8) {
+        float v[4];
+        load(c, v);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) m = fmaxf(m, fabsf(v[i]));
+        for (int i = 0; i < 4; ++i) {
+            m = fmaxf(m, fabsf(v[i]));
+            l1 += fabsf(v[i]);
+        }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) s_max[warp] = m;
+    for (int o = 16; o > 0; o >>= 1) {
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    if (lane == 0) {
+        s_max[warp] = m;
+        s_l1[warp] = l1;
+    }
     __syncthreads();
     m = s_max[0];
+    l1 = s_l1[0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) m = fmaxf(m, s_max[w]);
+    for (int w = 1; w < 8; ++w) {
+        m = fmaxf(m, s_max[w]);
+        l1 += s_l1[w];
+    }
     int e = 0;
     if (m > 0.f) {                   // a NaN or infinite max is not supported
         e = ilogbf(m) - 14;
         if (ldexpf(m, -e) > (float)kQMax) ++e;
     }
-    uint16_t *qh = xq + (size_t)row * 2 * cols, *ql = qh + cols;
-    int sum = 0;
+    // second word when the rounding step, summed over the row, exceeds 2^-12 of its mass
+    const bool res = m > 0.f && ldexpf((float)cols, e - 1) > ldexpf(l1, -kResBudgetLog2);
+    uint16_t *qh = xq + (size_t)row * 4 * cols, *ql = qh + cols, *rh = ql + cols, *rl = rh + cols;
+    int sum = 0, rsum = 0;
     for (int c = warp; c < chunks; c += 8) {
         float v[4];
-        src.load(row, c, lane, v);
-        if constexpr (ROTATE) {
-            if (signs) {   // input side of the two-sided transform: rotate(signs * v)
-                const char4 sg = *reinterpret_cast<const char4 *>(signs + c * 128 + 4 * lane);
-                v[0] *= sg.x; v[1] *= sg.y; v[2] *= sg.z; v[3] *= sg.w;
-            }
-            fwht128_warp(v, lane);
-        }
-        uint32_t wh[4], wl[4];
+        load(c, v);
+        uint32_t wh[4], wl[4], vh[4], vl[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             int q = __float2int_rn(ldexpf(v[i], -e));
@@ -381,24 +418,47 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int c
             const int hi = (q - lo) >> 8;
             wh[i] = (uint32_t)(hi & 255) * 0x0101u;
             wl[i] = (uint32_t)(lo & 255) * 0x0101u;
+            if (res) {
+                const float r = __fsub_rn(v[i], ldexpf((float)q, e));   // exact
+                int rq = __float2int_rn(ldexpf(r, kResShift - e));
+                rq = max(-kQMax, min(kQMax, rq));
+                rsum += rq;
+                const int rlo = ((rq + 128) & 255) - 128;
+                const int rhi = (rq - rlo) >> 8;
+                vh[i] = (uint32_t)(rhi & 255) * 0x0101u;
+                vl[i] = (uint32_t)(rlo & 255) * 0x0101u;
+            }
         }
         const size_t off = (size_t)c * 128 + 4 * lane;
         *reinterpret_cast<uint2 *>(qh + off) = make_uint2(wh[0] | (wh[1] << 16), wh[2] | (wh[3] << 16));
         *reinterpret_cast<uint2 *>(ql + off) = make_uint2(wl[0] | (wl[1] << 16), wl[2] | (wl[3] << 16));
+        if (res) {
+            *reinterpret_cast<uint2 *>(rh + off) = make_uint2(vh[0] | (vh[1] << 16), vh[2] | (vh[3] << 16));
+            *reinterpret_cast<uint2 *>(rl + off) = make_uint2(vl[0] | (vl[1] << 16), vl[2] | (vl[3] << 16));
+        }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) s_sum[warp] = sum;
+    for (int o = 16; o > 0; o >>= 1) {
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        rsum += __shfl_xor_sync(0xffffffffu, rsum, o);
+    }
+    if (lane == 0) {
+        s_sum[warp] = sum;
+        s_rsum[warp] = rsum;
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
-        int total = 0;
-        for (int w = 0; w < 8; ++w) total += s_sum[w];
-        meta[row] = make_int2(e, total);
+        int total = 0, rtotal = 0;
+        for (int w = 0; w < 8; ++w) {
+            total += s_sum[w];
+            rtotal += s_rsum[w];
+        }
+        meta[row] = RowQ{e, total, res ? 1 : 0, rtotal};
     }
 }
 
 template <bool ROTATE, typename Src>
-int launch_quantize_rows(const Src &src, long long rows, int cols, uint16_t *xq, int2 *meta, cudaStream_t s,
+int launch_quantize_rows(const Src &src, long long rows, int cols, uint16_t *xq, RowQ *meta, cudaStream_t s,
                          int stage, const int8_t *signs = nullptr) {
     if (rows <= 0) return TQ_OK;
     if (rows > 0x7fffffffll) return TQ_ERR_UNSUPPORTED;
@@ -445,30 +505,53 @@ __device__ __forceinline__ bool expert_ref(const tq_moe_layer &L, int e, ExpertR
 // end of a pass.
 //
 // GATEUP: item = (active expert, 64 intermediate rows: strips 0..3 of gate, 0..3 of
-//         up, column split sp of kGateUpSplits); activations = the tokens' quantised
+//         up, column split sp of gu_splits); activations = the tokens' quantised
 //         rotated rows (xq, xmeta indexed by token); out = gu [routes][split][2][F]
-//         fp32, the split's share of gate x' and up x' (the SwiGLU is applied when h
-//         is rotated and quantised).  More than one split multiplies the CTAs of a
-//         small batch; measured on the 16-token decode layer it gains nothing, so the
-//         columns are not split.
+//         fp32, the split's share of gate x' and up x' (the SwiGLU pass that rotates
+//         and quantises h adds the splits in order).  Splits multiply the CTAs of a
+//         small batch (gate_up_splits): a 1-token step has 8 active experts, i.e. 128
+//         unsplit items for 148 SMs.
 // !GATEUP: item = (active expert, 128 output rows); activations = quantised h'
 //          (indexed by route); out = y [routes][D] fp32.
-constexpr int kGateUpSplits = 1;
 constexpr int kNb2MinRoutes = 5;
+constexpr int kMaxGateUpSplits = 8;
+
+// Column splits of the gate/up items: enough CTAs for ~3 per SM at the batch's largest
+// possible number of active experts (min(E, T k)); 1 from a few tokens on.
+inline int gate_up_splits(const tq_moe_layer *L, int T, int k) {
+    const long long max_active = min((long long)L->E, (long long)T * k);
+    const long long items = max_active * (L->F / 64);
+    if (items <= 0) return 1;
+    const long long want = (3ll * num_sms() + items - 1) / items;
+    return (int)max(1ll, min((long long)kMaxGateUpSplits, min(want, (long long)(L->D / 128))));
+}
+
+// Slots of one pass: the routes [tb, next) of the item's expert, one slot per word of
+// each route's activation row (a two-word row takes two adjacent slots).
+template <int NB>
+struct PassSlots {
+    int row[4 * NB];      // activation row of the slot (-1: empty, -2: route with an invalid index)
+    int word[4 * NB];     // 0: main word, 1: residual word
+    int route[4 * NB];    // route offset within the expert (main-word slots)
+    int cand[4 * NB];     // candidate routes' rows, then words needed
+    int need[4 * NB];
+    int next;
+};
 
 template <bool GATEUP, int NB>
 __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
-    moe_gemv_items_kernel(const tq_moe_layer L, const uint16_t *__restrict__ xq, const int2 *__restrict__ xmeta,
+    moe_gemv_items_kernel(const tq_moe_layer L, const uint16_t *__restrict__ xq, const RowQ *__restrict__ xmeta,
                           const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm,
                           const int32_t *__restrict__ active_ids, const int32_t *__restrict__ n_active_p,
-                          int k, int n_routes, float *__restrict__ out) {
+                          int k, int n_routes, int gu_splits, float *__restrict__ out) {
     chain_entry();
     extern __shared__ __align__(128) unsigned char smem_raw[];
     ItemSmem &sm_items = *reinterpret_cast<ItemSmem *>(smem_raw);
     ItemRed<NB> &red = *reinterpret_cast<ItemRed<NB> *>(smem_raw);
-    __shared__ int s_row[4 * NB];
+    __shared__ PassSlots<NB> ps;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2;
-    constexpr int splits = GATEUP ? kGateUpSplits : 1;
+    const int splits = GATEUP ? gu_splits : 1;
+    constexpr int NS = 4 * NB;
     const int per_expert = (GATEUP ? L.F / 64 : L.D / 128) * splits;
     const int item = blockIdx.x;
     if (item >= *n_active_p * per_expert) return;
@@ -498,11 +581,11 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
     else
         strip_lane = ex.down + (size_t)(sub * 8 + cs) * tiles * (8 * ex.K);
 
-    for (int tb = 0; tb < ne; tb += 4 * NB) {
-        // activation row of each route of the pass (-1: none)
-        if (threadIdx.x < 4 * NB) {
+    for (int tb = 0; tb < ne;) {
+        // the next NS routes' activation rows and the words each needs
+        if (threadIdx.x < NS) {
             const int tt = tb + threadIdx.x;
-            int row = -1;            // -1: no route; -2: route with an invalid index
+            int row = -1, need = 0;
             if (tt < ne) {
                 if (GATEUP) {
                     const int pr = perm[r0 + tt];
@@ -510,15 +593,37 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
                 } else {
                     row = r0 + tt;
                 }
+                need = (row >= 0 && xmeta[row].res) ? 2 : 1;
             }
-            s_row[threadIdx.x] = row;
+            ps.cand[threadIdx.x] = row;
+            ps.need[threadIdx.x] = need;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            // as many whole routes as fit in the pass's slots (the first always fits)
+            int slot = 0, i = 0;
+            while (i < NS && ps.need[i] > 0 && slot + ps.need[i] <= NS) {
+                for (int w = 0; w < ps.need[i]; ++w, ++slot) {
+                    ps.row[slot] = ps.cand[i];
+                    ps.word[slot] = w;
+                    ps.route[slot] = tb + i;
+                }
+                ++i;
+            }
+            for (; slot < NS; ++slot) {
+                ps.row[slot] = -1;
+                ps.word[slot] = 0;
+                ps.route[slot] = -1;
+            }
+            ps.next = tb + i;
         }
         __syncthreads();
         const uint16_t *xw[NB];
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-            const int my_row = s_row[4 * b + (gq >> 1)];
-            xw[b] = my_row >= 0 ? xq + (size_t)my_row * 2 * cols + (gq & 1) * cols : nullptr;
+            const int slot = 4 * b + (gq >> 1);
+            const int my_row = ps.row[slot];
+            xw[b] = my_row >= 0 ? xq + (size_t)my_row * 4 * cols + (2 * ps.word[slot] + (gq & 1)) * cols : nullptr;
         }
         AccI<NB> acc;
         zero(acc);
@@ -528,51 +633,95 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
         store_partials(acc, red);   // the rings are idle now
         __syncthreads();
         if (GATEUP) {
-            for (int i = threadIdx.x; i < 4 * 16 * 4 * NB; i += kItemThreads) {
-                const int rt = i % (4 * NB), row = (i / (4 * NB)) & 15, st = i / (64 * NB);
-                const int xrow = s_row[rt];
-                if (xrow == -1) continue;
+            for (int i = threadIdx.x; i < 4 * 16 * NS; i += kItemThreads) {
+                const int rt = i % NS, row = (i / NS) & 15, st = i / (16 * NS);
+                const int xrow = ps.row[rt];
+                if (xrow == -1 || ps.word[rt] != 0) continue;
                 const int f = (sub * 4 + st) * 16 + row;
                 float gv = 0.f, uv = 0.f;    // a route with an invalid index: h = 0
                 if (xrow >= 0) {
-                    int2 m = xmeta[xrow];
-                    if (sp) m.y = 0;         // the -255 sum x term is added once, by split 0
+                    RowQ m = xmeta[xrow];
+                    if (sp) m.sum = m.rsum = 0;   // the -255 sum x term is added once, by split 0
                     const int2 g = red_sum(red, st, row, rt), u = red_sum(red, st + 4, row, rt);
-                    gv = finish_q(g.x, g.y, m, __half2float(ex.s_gate[f]));
-                    uv = finish_q(u.x, u.y, m, __half2float(ex.s_up[f]));
+                    int2 g2 = make_int2(0, 0), u2 = make_int2(0, 0);
+                    if (m.res) {
+                        g2 = red_sum(red, st, row, rt + 1);
+                        u2 = red_sum(red, st + 4, row, rt + 1);
+                    }
+                    gv = finish_q(g.x, g.y, m, __half2float(ex.s_gate[f]), g2.x, g2.y);
+                    uv = finish_q(u.x, u.y, m, __half2float(ex.s_up[f]), u2.x, u2.y);
                 }
-                float *o = out + ((size_t)(r0 + tb + rt) * splits + sp) * 2 * L.F + f;
+                float *o = out + ((size_t)(r0 + ps.route[rt]) * splits + sp) * 2 * L.F + f;
                 o[0] = gv;
                 o[L.F] = uv;
             }
         } else {
-            for (int i = threadIdx.x; i < 8 * 16 * 4 * NB; i += kItemThreads) {
-                const int rt = i % (4 * NB), row = (i / (4 * NB)) & 15, st = i / (64 * NB);
-                const int xrow = s_row[rt];
-                if (xrow < 0) continue;
+            for (int i = threadIdx.x; i < 8 * 16 * NS; i += kItemThreads) {
+                const int rt = i % NS, row = (i / NS) & 15, st = i / (16 * NS);
+                const int xrow = ps.row[rt];
+                if (xrow < 0 || ps.word[rt] != 0) continue;
+                const RowQ m = xmeta[xrow];
                 const int2 y = red_sum(red, st, row, rt);
+                const int2 y2 = m.res ? red_sum(red, st, row, rt + 1) : make_int2(0, 0);
                 const int d = (sub * 8 + st) * 16 + row;
-                out[(size_t)xrow * L.D + d] = finish_q(y.x, y.y, xmeta[xrow], __half2float(ex.s_down[d]));
+                out[(size_t)xrow * L.D + d] = finish_q(y.x, y.y, m, __half2float(ex.s_down[d]), y2.x, y2.y);
             }
         }
-        __syncthreads();   // the rings and s_row are reused by the next pass
+        tb = ps.next;
+        __syncthreads();   // the rings and the pass slots are reused by the next pass
     }
 }
 
 // ------------------------------------------------------------------------ single GEMV
 //
-// CTA = (group of 8 strips = 128 rows, column split, pass of 4*NB tokens); the 4 warps
-// split the CTA's column tiles.  The integer partial sums of all CTAs of a row group
-// are added into acc [batch][rows][2] with atomics (exact, so order-independent), and
-// gemv_finish_kernel applies the scales.
+// CTA = (group of 8 strips = 128 rows, column split, pass of 4*NB slots); the 4 warps
+// split the CTA's column tiles.  Slots number the words of the batch's rows in order:
+// token t's main word is slot t + R(t), R(t) the two-word rows before t, its residual
+// word the next slot.  The integer partial sums of all CTAs of a row group are added
+// into acc [batch][rows][4] (main H, L, residual H, L) with atomics (exact, so
+// order-independent), and gemv_finish_kernel applies the scales.
 template <int NB>
 __global__ void __launch_bounds__(kItemThreads, 4)
     trellis_gemv_kernel(const uint32_t *__restrict__ bits, int K, int rows, int cols, const uint16_t *__restrict__ xq,
-                        int batch, int col_splits, int *__restrict__ acc_out) {
+                        const RowQ *__restrict__ meta, int batch, int col_splits, int *__restrict__ acc_out) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     ItemSmem &sm_items = *reinterpret_cast<ItemSmem *>(smem_raw);
     ItemRed<NB> &red = *reinterpret_cast<ItemRed<NB> *>(smem_raw);
+    constexpr int NS = 4 * NB;
+    __shared__ int s_tok[NS], s_word[NS];
+    __shared__ int s_warp[kItemWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2;
+    // this pass's slots: token ranges per thread, residual-row counts scanned over the CTA
+    const int slot0 = blockIdx.z * NS;
+    if (threadIdx.x < NS) {
+        s_tok[threadIdx.x] = -1;
+        s_word[threadIdx.x] = 0;
+    }
+    const int per = (batch + kItemThreads - 1) / kItemThreads;
+    const int t_begin = min(batch, (int)threadIdx.x * per), t_end = min(batch, t_begin + per);
+    int mine = 0;
+    for (int t = t_begin; t < t_end; ++t) mine += meta[t].res;
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int before = incl - mine;
+    for (int w = 0; w < warp; ++w) before += s_warp[w];
+    for (int t = t_begin, slot = t_begin + before; t < t_end; ++t) {
+        const int words = 1 + meta[t].res;
+        for (int w = 0; w < words; ++w, ++slot)
+            if (slot >= slot0 && slot < slot0 + NS) {
+                s_tok[slot - slot0] = t;
+                s_word[slot - slot0] = w;
+            }
+    }
+    __syncthreads();
+    if (s_tok[0] < 0) return;   // beyond the batch's last slot (the grid covers two words per row)
+
     const int n_strips = rows / 16, tiles = cols / 16;
     const WarpRing ring{sm_items.buf[warp], sm_items.bar[warp]};
     ring_init(ring);
@@ -584,12 +733,12 @@ __global__ void __launch_bounds__(kItemThreads, 4)
     je += cb;
     const int strip = min((int)blockIdx.x * 8 + (lane & 7), n_strips - 1);   // rows beyond are dropped
     const uint32_t *strip_lane = bits + (size_t)strip * tiles * (8 * K);
-    const int tok0 = blockIdx.z * 4 * NB;
     const uint16_t *xw[NB];
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-        const int t = tok0 + 4 * b + (gq >> 1);
-        xw[b] = t < batch ? xq + (size_t)t * 2 * cols + (gq & 1) * cols : nullptr;
+        const int slot = 4 * b + (gq >> 1);
+        const int t = s_tok[slot];
+        xw[b] = t >= 0 ? xq + (size_t)t * 4 * cols + (2 * s_word[slot] + (gq & 1)) * cols : nullptr;
     }
     AccI<NB> acc;
     zero(acc);
@@ -598,24 +747,24 @@ __global__ void __launch_bounds__(kItemThreads, 4)
     if (!ok) return;
     store_partials(acc, red);
     __syncthreads();
-    for (int i = threadIdx.x; i < 8 * 16 * 4 * NB; i += kItemThreads) {
-        const int rt = i % (4 * NB), row = (i / (4 * NB)) & 15, st = i / (64 * NB);
-        const int t = tok0 + rt, r = (blockIdx.x * 8 + st) * 16 + row;
-        if (t >= batch || r >= rows) continue;
+    for (int i = threadIdx.x; i < 8 * 16 * NS; i += kItemThreads) {
+        const int rt = i % NS, row = (i / NS) & 15, st = i / (16 * NS);
+        const int t = s_tok[rt], r = (blockIdx.x * 8 + st) * 16 + row;
+        if (t < 0 || r >= rows) continue;
         const int2 v = red_sum(red, st, row, rt);
-        int *dst = acc_out + ((size_t)t * rows + r) * 2;
+        int *dst = acc_out + ((size_t)t * rows + r) * 4 + 2 * s_word[rt];
         atomicAdd(dst, v.x);
         atomicAdd(dst + 1, v.y);
     }
 }
 
-__global__ void gemv_finish_kernel(const int *__restrict__ acc, const int2 *__restrict__ meta,
+__global__ void gemv_finish_kernel(const int *__restrict__ acc, const RowQ *__restrict__ meta,
                                    const __half *__restrict__ scales, int rows, int batch, float *__restrict__ y) {
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (size_t)rows * batch) return;
     const int t = (int)(i / rows), r = (int)(i % rows);
-    const int2 hl = reinterpret_cast<const int2 *>(acc)[i];
-    y[i] = finish_q(hl.x, hl.y, meta[t], __half2float(scales[r]));
+    const int4 hl = reinterpret_cast<const int4 *>(acc)[i];
+    y[i] = finish_q(hl.x, hl.y, meta[t], __half2float(scales[r]), hl.z, hl.w);
 }
 
 template <typename Kern>
@@ -628,24 +777,25 @@ inline int set_smem(Kern kern, size_t bytes) {
 
 inline size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
-// Workspace of the single GEMV: quantised rows, their (e, sum), integer sums.
+// Workspace of the single GEMV: quantised rows (4 planes), their RowQ, integer sums.
 struct GemvWs {
     uint16_t *xq;
-    int2 *meta;
+    RowQ *meta;
     int *acc;
 };
 
 size_t gemv_ws_bytes(int rows, int cols, int batch) {
-    return align256((size_t)batch * 2 * cols * 2) + align256((size_t)batch * 8) + align256((size_t)rows * batch * 8);
+    return align256((size_t)batch * 4 * cols * 2) + align256((size_t)batch * sizeof(RowQ)) +
+           align256((size_t)rows * batch * 16);
 }
 
 GemvWs gemv_ws(void *ws, int rows, int cols, int batch) {
     char *p = reinterpret_cast<char *>(ws);
     GemvWs w;
     w.xq = reinterpret_cast<uint16_t *>(p);
-    p += align256((size_t)batch * 2 * cols * 2);
-    w.meta = reinterpret_cast<int2 *>(p);
-    p += align256((size_t)batch * 8);
+    p += align256((size_t)batch * 4 * cols * 2);
+    w.meta = reinterpret_cast<RowQ *>(p);
+    p += align256((size_t)batch * sizeof(RowQ));
     w.acc = reinterpret_cast<int *>(p);
     return w;
 }
@@ -661,14 +811,17 @@ int run_gemv(const uint32_t *bits, const __half *scales, int K, int rows, int co
     }
     int st = launch_quantize_rows<false>(RowSrc<__half>{x, cols}, batch, cols, w.xq, w.meta, s, kStageGemvQuant);
     if (st) return st;
-    if (cudaMemsetAsync(w.acc, 0, (size_t)rows * batch * 8, s) != cudaSuccess) return record_cuda_error("cudaMemsetAsync");
+    if (cudaMemsetAsync(w.acc, 0, (size_t)rows * batch * 16, s) != cudaSuccess) return record_cuda_error("cudaMemsetAsync");
+    // the split count is chosen for one word per row; the grid covers up to two words per
+    // row, and the CTAs of passes beyond the batch's last slot return at once
     const int groups = (rows / 16 + 7) / 8, passes = (batch + 4 * NB - 1) / (4 * NB), tiles = cols / 16;
     const int want = (4 * num_sms() + groups * passes - 1) / (groups * passes);
     const int splits = max(1, min(want, tiles / (2 * kItemWarps)));
+    const int slot_passes = (2 * batch + 4 * NB - 1) / (4 * NB);
     {
         LaunchScope ls(s, kStageGemv);
-        trellis_gemv_kernel<NB><<<dim3(groups, splits, passes), kItemThreads, smem, s>>>(bits, K, rows, cols, w.xq,
-                                                                                         batch, splits, w.acc);
+        trellis_gemv_kernel<NB><<<dim3(groups, splits, slot_passes), kItemThreads, smem, s>>>(
+            bits, K, rows, cols, w.xq, w.meta, batch, splits, w.acc);
     }
     st = launch_status();
     if (st) return st;
@@ -701,20 +854,20 @@ int validate_layer(const tq_moe_layer *L) {
 }
 
 // Workspace of the MoE GEMV: gate/up partial sums gu [routes][splits][2][F] fp32,
-// quantised h' [routes][2][F] half-words and its (e, sum) per route, quantised x'
-// [T][2][D] half-words and its (e, sum) per token.
+// quantised h' [routes][4][F] half-words (main and residual word planes) and its RowQ
+// per route, quantised x' [T][4][D] half-words and its RowQ per token.
 struct MoeGemvWs {
     float *gu;
     uint16_t *hq;
-    int2 *hmeta;
+    RowQ *hmeta;
     uint16_t *xq;
-    int2 *xmeta;
+    RowQ *xmeta;
 };
 
 size_t workspace_bytes(const tq_moe_layer *L, int T, int k) {
     const size_t routes = (size_t)T * k;
-    return align256(routes * kGateUpSplits * 2 * L->F * 4) + align256(routes * 2 * L->F * 2) + align256(routes * 8) +
-           align256((size_t)T * 2 * L->D * 2) + align256((size_t)T * 8);
+    return align256(routes * gate_up_splits(L, T, k) * 2 * L->F * 4) + align256(routes * 4 * L->F * 2) +
+           align256(routes * sizeof(RowQ)) + align256((size_t)T * 4 * L->D * 2) + align256((size_t)T * sizeof(RowQ));
 }
 
 MoeGemvWs moe_gemv_ws(const tq_moe_layer *L, int T, int k, void *ws) {
@@ -722,14 +875,14 @@ MoeGemvWs moe_gemv_ws(const tq_moe_layer *L, int T, int k, void *ws) {
     char *p = reinterpret_cast<char *>(ws);
     MoeGemvWs w;
     w.gu = reinterpret_cast<float *>(p);
-    p += align256(routes * kGateUpSplits * 2 * L->F * 4);
+    p += align256(routes * gate_up_splits(L, T, k) * 2 * L->F * 4);
     w.hq = reinterpret_cast<uint16_t *>(p);
-    p += align256(routes * 2 * L->F * 2);
-    w.hmeta = reinterpret_cast<int2 *>(p);
-    p += align256(routes * 8);
+    p += align256(routes * 4 * L->F * 2);
+    w.hmeta = reinterpret_cast<RowQ *>(p);
+    p += align256(routes * sizeof(RowQ));
     w.xq = reinterpret_cast<uint16_t *>(p);
-    p += align256((size_t)T * 2 * L->D * 2);
-    w.xmeta = reinterpret_cast<int2 *>(p);
+    p += align256((size_t)T * 4 * L->D * 2);
+    w.xmeta = reinterpret_cast<RowQ *>(p);
     return w;
 }
 
@@ -747,7 +900,8 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     const int routes = T * k;
     const MoeGemvWs w = moe_gemv_ws(L, T, k, ws);
     const int max_active = min(L->E, routes);
-    const int gu_items = max_active * (L->F / 64) * kGateUpSplits;
+    const int splits = gate_up_splits(L, T, k);
+    const int gu_items = max_active * (L->F / 64) * splits;
     const int dn_items = max_active * (L->D / 128);
     int st = launch_quantize_rows<false>(RowSrc<__half>{x_rot, L->D}, T, L->D, w.xq, w.xmeta, s, kStageGemvQuant);
     if (st) return st;
@@ -758,23 +912,23 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
         LaunchScope ls(s, kStageGemvGateUp);
         if (nb2)
             launch_chained(moe_gemv_items_kernel<true, 2>, gu_items, kItemThreads, smem, s, *L, w.xq, w.xmeta, offsets,
-                           perm, active_ids, n_active, k, routes, w.gu);
+                           perm, active_ids, n_active, k, routes, splits, w.gu);
         else
             launch_chained(moe_gemv_items_kernel<true, 1>, gu_items, kItemThreads, smem, s, *L, w.xq, w.xmeta, offsets,
-                           perm, active_ids, n_active, k, routes, w.gu);
+                           perm, active_ids, n_active, k, routes, splits, w.gu);
     }
     st = launch_status();
     if (st) return st;
-    st = launch_quantize_rows<true>(SwigluSrc{w.gu, L->F, kGateUpSplits, L->sign_gu}, routes, L->F, w.hq, w.hmeta, s,
+    st = launch_quantize_rows<true>(SwigluSrc{w.gu, L->F, splits, L->sign_gu}, routes, L->F, w.hq, w.hmeta, s,
                                     kStageRotateH, L->sign_h);
     if (st) return st;
     LaunchScope ls(s, kStageGemvDown);
     if (nb2)
         launch_chained(moe_gemv_items_kernel<false, 2>, dn_items, kItemThreads, smem, s, *L, w.hq, w.hmeta, offsets,
-                       perm, active_ids, n_active, k, routes, y_perm);
+                       perm, active_ids, n_active, k, routes, 1, y_perm);
     else
         launch_chained(moe_gemv_items_kernel<false, 1>, dn_items, kItemThreads, smem, s, *L, w.hq, w.hmeta, offsets,
-                       perm, active_ids, n_active, k, routes, y_perm);
+                       perm, active_ids, n_active, k, routes, 1, y_perm);
     return launch_status();
 }
 

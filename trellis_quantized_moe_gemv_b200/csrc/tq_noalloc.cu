@@ -13,10 +13,9 @@
 
 namespace tq {
 
-// Scratch for the GEMV's workspace (gate/up partial sums, quantised h' and x'): at most
-// 4 MiB, i.e. 12 * T * k * F + 4 * T * D bytes plus 8 per row (T <= 36 tokens at k = 8,
-// D = 4096, F = 1024).  Every GPU that loads the library holds this array until the
-// process exits.
+// Scratch for the GEMV's workspace (gate/up partial sums, fixed-point h' and x'): at most
+// 4 MiB (T <= 25 tokens at k = 8, D = 4096, F = 1024).  Every GPU that loads the library
+// holds this array until the process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
