@@ -28,6 +28,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "routed-expert tok/s per MoE layer; GEMV HBM GB/s and GEMM tensor-pipe % of peak"
+# what each expert path contracts (weights are exact integer codes on both)
+DTYPE_LABEL = {
+    "gemv": "gemv: activations as 16-bit fixed point (two words for rows with outliers), "
+            "u8 x s8 IMMA, int32 sums; gemm: f16 operands, f32 accumulate",
+    "gemm": "gemm: f16 operands (decoded codes exact), f32 accumulate in tensor memory",
+}
 N_LAYER_COPIES = 4   # default of --layers
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
@@ -38,6 +44,16 @@ def parse_args():
     p.add_argument("--steps", type=int, default=None,
                    help="timed steps (default: 500 decode, 50 prefill: about 0.15-0.2 s timed)")
     p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--repeats", type=int, default=5,
+                   help="the timed loop of --steps steps runs this many times; the median repeat is reported")
+    p.add_argument("--no-prefill", action="store_true",
+                   help="skip the prefill-layer (tensor-core GEMM) measurement of the default run")
+    p.add_argument("--batch1", action="store_true",
+                   help="decode GEMV at 1 and 16 tokens on single-width layers (K = 2, 3, 4), L2 flushed before "
+                        "every step; kernel GB/s from the library's events")
+    p.add_argument("--gemv-single", action="store_true",
+                   help="trellis_gemv on 1024x4096 projections at batch 1 (K = 2, 3, 4), L2 flushed before "
+                        "every call")
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="moe_decode_t16", choices=["moe_decode_t16", "moe_prefill_t8192"])
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -159,12 +175,15 @@ class ClockSampler:
             self._stop.set()
             self._t.join()
 
-    def summary(self, t0, t1):
+    def summary(self, windows):
+        """Median SM clock and the clock-event reasons seen in the timed windows
+        [(t0, t1), ...] (the repeats of the timed loop)."""
         if not self.ok:
             return None
-        inside = [s for s in self.samples if t0 <= s[0] <= t1]
-        window = "timed"
+        inside = [s for s in self.samples if any(t0 <= s[0] <= t1 for t0, t1 in windows)]
+        window = "timed (%d repeats)" % len(windows)
         if not inside:
+            t0, t1 = windows[0][0], windows[-1][1]
             inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
             window = "nearest to the timed region (region shorter than the sampling period)"
         if not inside:
@@ -342,25 +361,29 @@ def run_ours(args, rank, world, local_rank):
         else:
             graphs[i % NL].replay()
 
-    # ---- device-timed region
+    # ---- device-timed region: R repeats of K steps, each bracketed by a barrier and a
+    # synchronize on both sides; the median repeat is the result
     sampler = ClockSampler(local_rank)
     sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
     launches0 = api.launch_count()
-    t_wall0 = time.time()
+    windows, rep_ms = [], []
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for i in range(args.steps):
-        step(i)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    t_wall1 = time.time()
-    if world > 1:
-        dist.barrier()
-    launches = (api.launch_count() - launches0) if args.eager else launches_per_step * args.steps
+    for r in range(args.repeats):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_wall0 = time.time()
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        windows.append((t_wall0, time.time()))
+        if world > 1:
+            dist.barrier()
+        rep_ms.append(ev0.elapsed_time(ev1))
+    launches = (api.launch_count() - launches0) // args.repeats if args.eager else launches_per_step * args.steps
     stages = api.profile_collect()
     sampler.stop()
     # per-stage breakdown, outside the timed region
@@ -374,7 +397,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     stage_breakdown = api.profile_collect()
     api.profile_disable()
-    ms_total = ev0.elapsed_time(ev1)
+    ms_total = statistics.median(rep_ms)
     flags = api.device_status()
     if flags:
         raise RuntimeError("device anomaly flags %d during the timed region" % flags)
@@ -409,14 +432,15 @@ def run_ours(args, rank, world, local_rank):
         unit_work = gateup_flops(layers[0], T, k)
         E = layers[0].E
         achieved = unit_work / (g_avg_ms * 1e-3) / 1e12
-        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        peak = float(peaks["bf16_tflops"])     # burst: the timed region is sub-second
         prof = profile_traffic("moe_gemm_gateup_prefill_t8192")
         traffic = None
         if prof is not None:
             traffic = float(prof["dram_bytes_per_unit"]) * float(prof.get("units", 1))
         roofline = {"kernel": wl["kernel"], "bound": "tensor", "achieved": achieved, "peak": peak,
                     "unit": "TFLOP/s", "frac": achieved / peak,
-                    "peak_source": peak_src + " (dense bf16 GEMM, sustained; fp16 dense rate is the same)",
+                    "peak_source": peak_src + " (dense bf16 GEMM, burst: the timed region is sub-second; "
+                                              "fp16 dense rate is the same)",
                     "flops_per_launch": unit_work, "avg_launch_ms": g_avg_ms, "traffic": traffic}
 
     # ---- end to end through the public API with host buffers: api.MoeGraph, one per
@@ -435,22 +459,31 @@ def run_ours(args, rank, world, local_rank):
     for i in range(args.warmup):
         e2e_step(i)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms, e2e_value = aggregate_ranks(e0.elapsed_time(e1), T * args.steps, world, device)
+    e2e_rep = []
+    for r in range(args.repeats):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(args.steps):
+            e2e_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_rep.append(e0.elapsed_time(e1))
+    e2e_ms, e2e_value = aggregate_ranks(statistics.median(e2e_rep), T * args.steps, world, device)
     h2d = T * D * 2 + T * E * 4
     d2h = T * D * 4
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w0, routes=16, name=args.workload)
+
+    prefill = None
+    if args.workload == "moe_decode_t16" and not args.no_prefill and not args.two_sided:
+        del graphs, e2e_graphs
+        prefill = measure_prefill(args, api, inputs, torch, device, rank, world, stream)
 
     line = {
         "metric": METRIC,
@@ -463,7 +496,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16",
+        "dtype": DTYPE_LABEL[wl["path"]],
         "data": "synthetic",
         "config": {
             "workload": args.workload, "experts": E, "hidden": D, "intermediate": F,
@@ -482,14 +515,90 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches,
         "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "clocks": sampler.summary(t_wall0, t_wall1),
+        "clocks": sampler.summary(windows),
         "cpu_baseline": cpu,
+        "prefill": prefill,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_prefill(args, api, inputs, torch, device, rank, world, stream, steps=20):
+    """The prefill layer (384 experts all K = 3, 8192 Zipf-routed tokens, top-8) through the
+    tcgen05 GEMM path: R repeats of `steps` CUDA-graph replays (each reads all 1.8 GB of bit
+    streams, beyond L2), median repeat; the gate/up GEMM's average launch time from the
+    library's events in the timed graph; tensor roofline against the burst bf16 peak (the
+    timed region is well under a second)."""
+    import torch.distributed as dist
+    T, k = 8192, 8
+    w0, layers, xs = build_prefill_workload(api, inputs, device, rank, T=T)
+    L = layers[0]
+    bufs = api.MoeBuffers(L, T, k)
+    x = torch.from_numpy(xs[0][0]).to(torch.bfloat16).to(device)
+    lg = torch.from_numpy(xs[0][1]).to(device)
+    for _ in range(args.warmup):
+        api.moe_layer(L, x, lg, k, bufs=bufs, path="gemm")
+    torch.cuda.synchronize()
+    api.profile_enable(64)
+    api.profile_stages(["gemm_gateup", "gemm_down"])
+    api.profile_collect()      # the graph's event nodes are re-recorded at every replay
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            api.moe_layer(L, x, lg, k, bufs=bufs, path="gemm")
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    rep_ms, windows = [], []
+    for r in range(args.repeats):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.time()
+        e0.record(stream)
+        for i in range(steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        windows.append((t0, time.time()))
+        rep_ms.append(e0.elapsed_time(e1))
+    sampler.stop()
+    st = api.profile_collect()
+    api.profile_disable()
+    if api.device_status():
+        raise RuntimeError("device anomaly flags during the prefill measurement")
+    ms_max, tok_s = aggregate_ranks(statistics.median(rep_ms), T * steps, world, device)
+    gu_ms = st["gemm_gateup"][0] / max(st["gemm_gateup"][1], 1)
+    dn_ms = st["gemm_down"][0] / max(st["gemm_down"][1], 1)
+    peaks, src = load_peaks()
+    flops = gateup_flops(L, T, k)
+    achieved = flops / (gu_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    prof = profile_traffic("moe_gemm_gateup_prefill_t8192")
+    del g
+    return {
+        "workload": "moe_prefill_t8192", "tokens": T, "steps": steps, "repeats": args.repeats,
+        "ms_per_step": ms_max / steps, "value": tok_s, "unit": "tok/s", "dtype": DTYPE_LABEL["gemm"],
+        "roofline": {"kernel": WORKLOADS["moe_prefill_t8192"]["kernel"], "bound": "tensor", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": src + " (dense bf16 GEMM, burst: the region is sub-second; fp16 dense "
+                                          "rate is the same)",
+                     "flops_per_launch": flops, "avg_launch_ms": gu_ms,
+                     "traffic": (float(prof["dram_bytes_per_unit"]) * float(prof.get("units", 1)))
+                     if prof is not None else None},
+        "down_avg_launch_ms": dn_ms,
+        "clocks": sampler.summary(windows),
+    }
 
 
 def cpu_baseline(w0, routes, name="moe_decode_t16"):
@@ -569,6 +678,135 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def device_layer(api, torch, device, K, seed, E=384, D=4096, F=1024):
+    """A single-width layer (every expert at K bits per weight) with bit streams and
+    U[0.5, 1.5] scales drawn on the device from a seeded generator."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+
+    def rbits(n, rows, cols):
+        return torch.randint(-2 ** 31, 2 ** 31 - 1, (n, (rows // 16) * (cols // 16) * 8 * K), dtype=torch.int32,
+                             device=device, generator=gen)
+
+    def rscale(shape):
+        return (torch.rand(shape, device=device, generator=gen) + 0.5).to(torch.float16)
+    g = dict(K=K, ids=np.arange(E, dtype=np.int32), gate=rbits(E, F, D), up=rbits(E, F, D), down=rbits(E, D, F),
+             s_gate=rscale((E, F)), s_up=rscale((E, F)), s_down=rscale((E, D)))
+    return api.DeviceLayer(E, D, F, [g], device)
+
+
+def run_batch1(args, local_rank):
+    """The decode GEMV at 1 and 16 tokens on single-width 384-expert layers (K = 2, 3, 4),
+    top-8 of N(0,1) logits, a fresh token every step, L2 evicted (a 512 MB write) before
+    every step.  The library's events give each GEMV launch's device time; the gate/up
+    kernel's HBM rate is its algorithmic bytes (the touched experts' gate and up bit
+    streams and scales, activations in, results out) over that time.  One JSON line per
+    (K, tokens)."""
+    import torch
+    from trellis_quantized_moe_gemv_b200 import api, inputs
+    from trellis_quantized_moe_gemv_b200 import build as tqbuild
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    tqbuild.build()
+    api.lib()
+    E, D, F, k = 384, 4096, 1024, 8
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    peaks, src = load_peaks()
+    steps = max(args.steps, 8)
+    for K in (2, 3, 4):
+        L = device_layer(api, torch, device, K, 4000 + K)
+        for T in (1, 16):
+            rng = np.random.default_rng(4100 + 10 * K + T)
+            bufs = api.MoeBuffers(L, T, k)
+            data = [(torch.from_numpy(inputs.random_activations(rng, (T, D), "bf16")).to(torch.bfloat16).to(device),
+                     torch.from_numpy(inputs.normal_logits(rng, T, E)).to(device)) for _ in range(16)]
+            for i in range(args.warmup):
+                api.moe_layer(L, data[i % 16][0], data[i % 16][1], k, bufs=bufs, path="gemv")
+            torch.cuda.synchronize()
+            api.profile_enable(64 * steps)
+            api.profile_collect()
+            gu_bytes = dn_bytes = 0
+            for i in range(steps):
+                flush.zero_()
+                api.moe_layer(L, data[i % 16][0], data[i % 16][1], k, bufs=bufs, path="gemv")
+                counts = bufs.routing.counts.cpu().numpy()
+                n_exp = int((counts > 0).sum())
+                gu_bytes += n_exp * (2 * F * D * K // 8 + 2 * F * 2) + T * D * 2 + T * k * 2 * F * 4
+                dn_bytes += n_exp * (D * F * K // 8 + D * 2) + T * k * F * 2 + T * k * D * 4
+            torch.cuda.synchronize()
+            st = api.profile_collect()
+            api.profile_disable()
+            if api.device_status():
+                raise RuntimeError("device anomaly flags during the batch-1 measurement")
+            gu_ms = st["gemv_gateup"][0] / max(st["gemv_gateup"][1], 1)
+            dn_ms = st["gemv_down"][0] / max(st["gemv_down"][1], 1)
+            step_ms = sum(v[0] for v in st.values()) / steps
+            hbm = float(peaks["hbm_gbs"])
+            gu_gbs = gu_bytes / steps / (gu_ms * 1e-3) / 1e9
+            dn_gbs = dn_bytes / steps / (dn_ms * 1e-3) / 1e9
+            print(json.dumps({
+                "metric": "decode GEMV HBM GB/s on compressed bytes", "workload": "moe_gemv_single_width_K%d_t%d" % (K, T),
+                "K": K, "tokens": T, "top_k": k, "steps": steps, "l2": "512 MB written before every step",
+                "gateup": {"avg_launch_ms": gu_ms, "bytes_per_launch": gu_bytes / steps, "achieved_gbs": gu_gbs,
+                           "frac": gu_gbs / hbm},
+                "down": {"avg_launch_ms": dn_ms, "bytes_per_launch": dn_bytes / steps, "achieved_gbs": dn_gbs,
+                         "frac": dn_gbs / hbm},
+                "layer_device_ms": step_ms, "layer_tok_s": T / (step_ms * 1e-3),
+                "peak": hbm, "peak_source": src + " (copy bandwidth)"}), flush=True)
+            del bufs, data
+        del L
+        torch.cuda.empty_cache()
+
+
+def run_gemv_single(args, local_rank):
+    """trellis_gemv on one 1024x4096 projection at batch 1 (K = 2, 3, 4): 16 projections
+    drawn on the device, L2 evicted before every call, each call's device time (row
+    quantisation, the GEMV and its finishing kernel) from the library's events.  A 1-2 MB
+    projection is a few microseconds of HBM time, so this measures launch latency as much
+    as bandwidth."""
+    import torch
+    from trellis_quantized_moe_gemv_b200 import api, inputs
+    from trellis_quantized_moe_gemv_b200 import build as tqbuild
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    tqbuild.build()
+    api.lib()
+    rows, cols = 1024, 4096
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    peaks, src = load_peaks()
+    steps = max(args.steps, 8)
+    for K in (2, 3, 4):
+        gen = torch.Generator(device=device)
+        gen.manual_seed(4200 + K)
+        mats = [torch.randint(-2 ** 31, 2 ** 31 - 1, ((rows // 16) * (cols // 16) * 8 * K,), dtype=torch.int32,
+                              device=device, generator=gen) for _ in range(16)]
+        scales = (torch.rand(rows, device=device, generator=gen) + 0.5).to(torch.float16)
+        x = torch.randn((1, cols), device=device, generator=gen).to(torch.float16)
+        y = torch.empty((1, rows), dtype=torch.float32, device=device)
+        ws = torch.empty(api.trellis_gemv_workspace_size(rows, cols, 1), dtype=torch.uint8, device=device)
+        for i in range(args.warmup):
+            api.trellis_gemv(mats[i % 16], scales, K, rows, cols, x, y, ws)
+        torch.cuda.synchronize()
+        api.profile_enable(16 * steps)
+        api.profile_collect()
+        for i in range(steps):
+            flush.zero_()
+            api.trellis_gemv(mats[i % 16], scales, K, rows, cols, x, y, ws)
+        torch.cuda.synchronize()
+        st = api.profile_collect()
+        api.profile_disable()
+        call_ms = (st["trellis_gemv"][0] + st["gemv_quant"][0]) / steps
+        gemv_ms = st["trellis_gemv"][0] / steps
+        nbytes = rows * cols * K // 8 + rows * 2 + cols * 2 + rows * 4
+        gbs = nbytes / (gemv_ms * 1e-3) / 1e9
+        print(json.dumps({
+            "metric": "single-projection GEMV HBM GB/s on compressed bytes", "workload": "proj_1024x4096_K%d_b1" % K,
+            "K": K, "batch": 1, "steps": steps, "l2": "512 MB written before every call",
+            "bytes_per_call": nbytes, "gemv_ms": gemv_ms, "call_device_ms": call_ms, "achieved_gbs": gbs,
+            "frac": gbs / float(peaks["hbm_gbs"]), "peak_source": src + " (copy bandwidth)",
+            "note": "gemv_ms covers the GEMV and its finishing kernel (two launches)"}), flush=True)
+
+
 SWEEP_T = (1, 8, 64, 256, 384, 512, 1024, 2048, 16384)   # the configured sizes plus three near the crossover
 
 
@@ -583,7 +821,9 @@ def run_sweep(args, local_rank):
     device = torch.device("cuda", local_rank)
     tqbuild.build()
     api.lib()
-    w0, layers, _ = build_decode_workload(api, inputs, torch, device, 0, 4)
+    # 12 layer copies: at 1 token a step touches ~26 MB of bit streams, so 4 copies would
+    # stay in the 126 MB L2; from 8 tokens on, 4 copies are cycled
+    w0, all_layers, _ = build_decode_workload(api, inputs, torch, device, 0, 12)
     host_layer, k = w0["layer"], 8
     stream = torch.cuda.current_stream()
     results = []
@@ -591,7 +831,10 @@ def run_sweep(args, local_rank):
         w = inputs.moe_sweep_tokens(T, layer=host_layer)
         x = torch.from_numpy(w["x"]).to(torch.bfloat16).to(device)
         lg = torch.from_numpy(w["logits"]).to(device)
-        row = {"sweep": "moe_sweep_tokens", "tokens": T, "top_k": k, "routing": "top-8 of N(0,1) logits"}
+        layers = all_layers if T == 1 else all_layers[:4]
+        NC = len(layers)
+        row = {"sweep": "moe_sweep_tokens", "tokens": T, "top_k": k, "routing": "top-8 of N(0,1) logits",
+               "layer_copies_cycled": NC}
         for path in ("gemv", "gemm"):
             bufs = [api.MoeBuffers(L, T, k) for L in layers]
             for c, L in enumerate(layers):
@@ -608,14 +851,14 @@ def run_sweep(args, local_rank):
                     graphs.append(g)
             stream.wait_stream(side)
             for i in range(8):
-                graphs[i % 4].replay()
+                graphs[i % NC].replay()
             torch.cuda.synchronize()
             steps = max(8, min(400, int(4e5 / max(T, 1))))
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             for i in range(steps):
-                graphs[i % 4].replay()
+                graphs[i % NC].replay()
             e1.record(stream)
             torch.cuda.synchronize()
             ms = e0.elapsed_time(e1) / steps
@@ -691,6 +934,12 @@ def main():
     if args.encode:
         if rank == 0:
             run_encode(args, local_rank)
+    elif args.batch1:
+        if rank == 0:
+            run_batch1(args, local_rank)
+    elif args.gemv_single:
+        if rank == 0:
+            run_gemv_single(args, local_rank)
     elif args.sweep:
         if rank == 0:
             run_sweep(args, local_rank)
