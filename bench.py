@@ -33,6 +33,8 @@ DTYPE_LABEL = {
     "gemv": "gemv: activations as 16-bit fixed point (two words for rows with outliers), "
             "u8 x s8 IMMA, int32 sums; gemm: f16 operands, f32 accumulate",
     "gemm": "gemm: f16 operands (decoded codes exact), f32 accumulate in tensor memory",
+    "gemm_fp8": "gemm: e4m3 weights (pair-trellis codes exact) and e4m3 activations with power-of-two row "
+                "scales, f32 accumulate in tensor memory",
 }
 N_LAYER_COPIES = 4   # default of --layers
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
@@ -55,7 +57,8 @@ def parse_args():
                    help="trellis_gemv on 1024x4096 projections at batch 1 (K = 2, 3, 4), L2 flushed before "
                         "every call")
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="moe_decode_t16", choices=["moe_decode_t16", "moe_prefill_t8192"])
+    p.add_argument("--workload", default="moe_decode_t16",
+                   choices=["moe_decode_t16", "moe_prefill_t8192", "moe_prefill_t8192_fp8"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--layers", type=int, default=4,
                    help="synthetic layer copies cycled through (4 keep every step's weights out of L2)")
@@ -255,10 +258,14 @@ def gateup_algorithmic_bytes(layer, counts):
     return total
 
 
-def build_prefill_workload(api, inputs, device, rank, T=8192, E=384, two_sided=False):
+def build_prefill_workload(api, inputs, device, rank, T=8192, E=384, two_sided=False, fp8=False):
     """The all-K=3 384-expert layer with 8192 Zipf(1.1)-routed tokens: one step touches
-    every expert (1.8 GB of bit streams), far beyond L2, so one layer copy suffices."""
-    w0 = inputs.moe_prefill_t8192(seed=1004 + 100 * rank, T=T, E=E)
+    every expert (1.8 GB of bit streams), far beyond L2, so one layer copy suffices.
+    fp8: the same shape with pair-trellis (E4M3) streams."""
+    if fp8:
+        w0 = inputs.moe_prefill_t8192_fp8(seed=1006 + 100 * rank, T=T, E=E)
+    else:
+        w0 = inputs.moe_prefill_t8192(seed=1004 + 100 * rank, T=T, E=E)
     if two_sided:
         inputs.with_signs(w0["layer"], 8000 + 100 * rank)
     layers = [api.DeviceLayer.from_synthetic(w0["layer"], device)]
@@ -279,6 +286,11 @@ WORKLOADS = {
                               kernel="moe_gemm_kernel<1> (gate/up tcgen05 GEMM + SiLU)",
                               widths="all 384 experts at K=3",
                               routing="top-8 of log p + Gumbel, p ~ rank^-1.1 (Zipf)"),
+    "moe_prefill_t8192_fp8": dict(T=8192, path="gemm", stage="gemm_gateup",
+                                  kernel="moe_gemm_kernel<1, fp8> (gate/up tcgen05 kind::f8f6f4 GEMM + SiLU, "
+                                         "pair-trellis E4M3 weights and activations)",
+                                  widths="all 384 experts at K=3, pair-trellis (E4M3) codebook",
+                                  routing="top-8 of log p + Gumbel, p ~ rank^-1.1 (Zipf)"),
 }
 
 
@@ -308,7 +320,7 @@ def run_ours(args, rank, world, local_rank):
     else:
         NL = 1
         w0, layers, xs = build_prefill_workload(api, inputs, device, rank, T=T, E=args.experts or 384,
-                                                two_sided=args.two_sided)
+                                                two_sided=args.two_sided, fp8=args.workload.endswith("fp8"))
     E, D, F = layers[0].E, layers[0].D, layers[0].F
     bufs = [api.MoeBuffers(L, T, k) for L in layers]
     x_dev = [torch.from_numpy(x).to(torch.bfloat16).to(device) for x, _ in xs]
@@ -433,14 +445,18 @@ def run_ours(args, rank, world, local_rank):
         E = layers[0].E
         achieved = unit_work / (g_avg_ms * 1e-3) / 1e12
         peak = float(peaks["bf16_tflops"])     # burst: the timed region is sub-second
-        prof = profile_traffic("moe_gemm_gateup_prefill_t8192")
+        fp8 = args.workload.endswith("fp8")
+        if fp8:
+            peak *= 2.0                        # E4M3 dense rate: twice bf16 (4.5 vs 2.25 PF nominal)
+        prof = profile_traffic("moe_gemm_gateup_prefill_t8192_fp8" if fp8 else "moe_gemm_gateup_prefill_t8192")
         traffic = None
         if prof is not None:
             traffic = float(prof["dram_bytes_per_unit"]) * float(prof.get("units", 1))
         roofline = {"kernel": wl["kernel"], "bound": "tensor", "achieved": achieved, "peak": peak,
                     "unit": "TFLOP/s", "frac": achieved / peak,
-                    "peak_source": peak_src + " (dense bf16 GEMM, burst: the timed region is sub-second; "
-                                              "fp16 dense rate is the same)",
+                    "peak_source": peak_src + (" (dense bf16 GEMM burst x 2, the nominal E4M3 / bf16 ratio)"
+                                               if fp8 else " (dense bf16 GEMM, burst: the timed region is "
+                                                           "sub-second; fp16 dense rate is the same)"),
                     "flops_per_launch": unit_work, "avg_launch_ms": g_avg_ms, "traffic": traffic}
 
     # ---- end to end through the public API with host buffers: api.MoeGraph, one per
@@ -496,7 +512,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": DTYPE_LABEL[wl["path"]],
+        "dtype": DTYPE_LABEL["gemm_fp8" if args.workload.endswith("fp8") else wl["path"]],
         "data": "synthetic",
         "config": {
             "workload": args.workload, "experts": E, "hidden": D, "intermediate": F,
@@ -505,6 +521,7 @@ def run_ours(args, rank, world, local_rank):
             "l2": ("inputs larger than L2: each step reads ~0.35 GB of bit streams; %d layers "
                    "(%.1f GB) cycled" % (NL, 1.23 * NL)) if wl["path"] == "gemv" else
                   "inputs larger than L2: each step reads all 1.8 GB of bit streams",
+            "codebook": "pair_e4m3" if args.workload.endswith("fp8") else "t16",
             "path": wl["path"], "launch": "eager" if args.eager else "cuda-graph replay per step",
             "parallelism": "replicas" if world > 1 else "single-gpu",
             "transform": "two-sided (Hadamard on both sides, layer signs)" if args.two_sided

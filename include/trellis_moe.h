@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 2
+#define TQ_ABI_VERSION 3
 
 typedef enum {
     TQ_OK = 0,
@@ -67,6 +67,13 @@ typedef enum {
 } tq_status;
 
 typedef enum { TQ_DTYPE_F16 = 0, TQ_DTYPE_BF16 = 1, TQ_DTYPE_F32 = 2 } tq_dtype;
+
+/* Codebook of a layer's bit streams (every width group of a layer shares it: "All
+ * encodes of a layer share its signs and its codebook", exlr8 card, "Stores"). */
+typedef enum {
+    TQ_CODEBOOK_T16 = 0,        /* T16: one weight per 16-bit window (dsx T16 card)       */
+    TQ_CODEBOOK_PAIR_E4M3 = 1   /* pair trellis decoded to FP8 E4M3 (exlr8 card, pmcgx)   */
+} tq_codebook;
 
 typedef void *tq_stream; /* cudaStream_t */
 
@@ -137,6 +144,21 @@ int tq_profile_collect(double *stage_ms, int32_t *stage_launches, int n_stages);
  */
 int trellis_decode(const uint32_t *bits, int K, int rows, int cols, uint16_t *out,
                    tq_stream stream);
+
+/*
+ * trellis_decode_e4m3 -- standalone decode of a pair-trellis matrix to its FP8 E4M3 codes
+ * (the pmcgx codebook of the "deepseek-v4.1-flash-exlr8" card, "Stores": two weights share
+ * one 20-bit state; each is the sum of the two fp16 halves of the state's product with its
+ * multiplier, rounded to E4M3).  Readings: the stream layout is T16's (same tiles, words
+ * and bit order); pair q of a tile reads stream bits 2Kq .. 2Kq + 19 (tail-biting) and
+ * holds tile positions 2q (product with 0xCBAC1FED) and 2q + 1 (0xBCA14C51); bit 14 of each
+ * 16-bit half is cleared before it is read as binary16; the halves are added in binary16
+ * (nearest even) and the sum rounded to E4M3 (nearest even).  W[r][c] = s[r] * 2^-5 * w.
+ *   bits : [rows/16][cols/16][8K] uint32, 16-byte aligned.
+ *   out  : [rows][cols] E4M3 bytes, row-major, 16-byte aligned (scales not applied).
+ *   rows, cols: multiples of 16.  K in {2, 3, 4}.
+ */
+int trellis_decode_e4m3(const uint32_t *bits, int K, int rows, int cols, uint8_t *out, tq_stream stream);
 
 /*
  * hadamard128 -- x' = (1/sqrt(128)) * H_128 x on every contiguous 128-chunk of each
@@ -307,6 +329,7 @@ typedef struct {
     const int8_t *sign_gu;       /* device [F]                                         */
     const int8_t *sign_h;        /* device [F]                                         */
     const int8_t *sign_y;        /* device [D]                                         */
+    int codebook;                /* tq_codebook of every group (0: T16)                */
 } tq_moe_layer;
 
 /*
@@ -348,9 +371,11 @@ int moe_trellis_gemv(const tq_moe_layer *layer, const uint16_t *x_rot, const int
  * counterpart: this is a packaging of the same computation.
  *   Same arguments and result as moe_trellis_gemv, minus ws / ws_bytes.  The workspace
  *   is a 4 MiB array compiled into the library (a __device__ array every GPU that loads
- *   the library holds until exit), so the GEMV workspace, 12 * T * k * F + 4 * T * D
- *   bytes plus 8 bytes per row (T <= 36 at k = 8, D = 4096, F = 1024), must fit in it;
- *   larger calls return TQ_ERR_WORKSPACE without doing anything.
+ *   the library holds until exit), so the GEMV workspace -- 8 * S * T * k * F (gate/up
+ *   results, S = 1..8 column splits for small batches) + 8 * T * k * F + 8 * T * D bytes
+ *   (fixed-point h' and x', two words each) plus 16 bytes per row, each part rounded up
+ *   to 256 bytes; T <= 25 at k = 8, D = 4096, F = 1024 -- must fit in it; larger calls
+ *   return TQ_ERR_WORKSPACE without doing anything.
  *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   Arguments are checked first, with the same statuses as moe_trellis_gemv; then a call
  *   whose workspace would not fit returns TQ_ERR_WORKSPACE.
@@ -369,11 +394,21 @@ int moe_trellis_gemv_noalloc(const tq_moe_layer *layer, const uint16_t *x_rot,
 
 /*
  * moe_trellis_gemm -- same result as moe_trellis_gemv for prefill-sized batches: the
- * bit streams are decoded to fp16 operands of tcgen05 tensor-core MMAs (accumulating
- * in tensor memory), each weight decoded once per block of up to 256 routes of its
+ * bit streams are decoded to tensor-core operands of tcgen05 MMAs (accumulating in
+ * tensor memory), each weight decoded once per block of up to 256 routes of its
  * expert.  Same arguments as moe_trellis_gemv; the workspace must hold
  * moe_trellis_workspace_size() bytes; D must be a multiple of 256 (TQ_ERR_UNSUPPORTED
  * otherwise).
+ *   T16 layers: fp16 operands (codes exact as fp16 subnormals t * 2^-24, activations
+ *   fp16), kind::f16 MMAs.  The rotated h' rows are stored as fp16 h' / 2^e with the
+ *   row's largest magnitude in [2^14, 2^15), so no finite h overflows.
+ *   Pair-trellis layers (codebook TQ_CODEBOOK_PAIR_E4M3, the exlr8 card's FP8 decode):
+ *   E4M3 weights and E4M3 activations, kind::f8f6f4 MMAs at twice the fp16 rate.  Each
+ *   route row of x' and of h' is scaled by the power of two 2^-e that puts its largest
+ *   magnitude in (224, 448] and rounded to E4M3 (nearest even), so the activations carry
+ *   E4M3's 2^-4 relative rounding; y = s * 2^-5 * 2^e * sum_j w_j * v8_j.
+ * moe_trellis_gemv and moe_trellis_gemv_noalloc run T16 layers only
+ * (TQ_ERR_UNSUPPORTED for a pair-trellis layer).
  */
 int moe_trellis_gemm(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
                      const int32_t *perm, const int32_t *active_ids, const int32_t *n_active,

@@ -31,7 +31,7 @@ primitives used as steps.
 """
 import numpy as np
 
-from . import t16
+from . import pair_trellis, t16
 
 KAPPA = 2.0 ** -12
 HADAMARD_N = 128
@@ -191,11 +191,17 @@ class ExpertWeights:
             rows, cols = (F, D) if proj in ("gate", "up") else (D, F)
             bits = getattr(g, proj)[idx]
             scales = getattr(g, "s_" + proj)[idx]
-            self._cache[key] = dequantize(t16.decode_matrix(bits, g.K, rows, cols), scales)
+            if getattr(self.layer, "codebook", "t16") == "pair_e4m3":
+                # the exlr8 card's pair trellis decoded to E4M3, W = s * 2^-5 * w
+                self._cache[key] = pair_trellis.dequantize(pair_trellis.decode_matrix(bits, g.K, rows, cols), scales)
+            else:
+                self._cache[key] = dequantize(t16.decode_matrix(bits, g.K, rows, cols), scales)
         return self._cache[key]
 
     def down_rows(self, e: int, row_ids) -> np.ndarray:
         """Selected rows of the down projection (fp64), without decoding the rest."""
+        if getattr(self.layer, "codebook", "t16") == "pair_e4m3":
+            return self.matrix(e, "down")[np.asarray(row_ids)]
         g, idx = self._where[int(e)]
         D, F = self.layer.D, self.layer.F
         codes = t16.decode_rows(g.down[idx], g.K, D, F, row_ids)

@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     from trellis_quantized_moe_gemv_b200 import api
-    assert api.abi_version() == 2
+    assert api.abi_version() == 3
     for code in range(7):
         assert lib.tq_status_string(code)
     assert b"ALIGNMENT" in lib.tq_status_string(3)
@@ -65,6 +65,10 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.trellis_decode(None, 2, 16, 16, FAKE, None) == 1
     assert lib.trellis_decode(MISALIGNED, 2, 16, 16, FAKE, None) == 3
     assert lib.trellis_decode(FAKE, 2, 0, 16, FAKE, None) == 0          # empty: no-op
+    assert lib.trellis_decode_e4m3(FAKE, 5, 16, 16, FAKE, None) == 1
+    assert lib.trellis_decode_e4m3(FAKE, 2, 16, 24, FAKE, None) == 1
+    assert lib.trellis_decode_e4m3(MISALIGNED, 2, 16, 16, FAKE, None) == 3
+    assert lib.trellis_decode_e4m3(FAKE, 2, 0, 16, FAKE, None) == 0
     assert lib.hadamard128(FAKE, 0, 4, 100, FAKE, None) == 1            # cols % 128
     assert lib.hadamard128(FAKE, 7, 4, 128, FAKE, None) == 1            # dtype
     assert lib.hadamard128(MISALIGNED, 0, 4, 128, FAKE, None) == 3
@@ -130,6 +134,14 @@ def test_moe_workspace_and_layer_validation(lib):
     assert lib.moe_trellis_workspace_size(ctypes.byref(bad), 16, 8) == 0
     bad = _layer_struct(D=200)
     assert lib.moe_trellis_workspace_size(ctypes.byref(bad), 16, 8) == 0
+    bad = _layer_struct()
+    bad.codebook = 7                                      # unknown codebook
+    assert lib.moe_trellis_workspace_size(ctypes.byref(bad), 16, 8) == 0
+    fp8 = _layer_struct()
+    fp8.codebook = 1                                      # pair trellis: GEMM only
+    assert lib.moe_trellis_workspace_size(ctypes.byref(fp8), 16, 8) == need
+    assert lib.moe_trellis_gemv(ctypes.byref(fp8), *[FAKE] * 5, 16, 8, FAKE, FAKE, need, None) == 2
+    assert lib.moe_trellis_gemv_noalloc(ctypes.byref(fp8), *[FAKE] * 5, 1, 8, FAKE, None) == 2
     args = [FAKE] * 5
     # workspace too small
     assert lib.moe_trellis_gemv(ctypes.byref(st), *args, 16, 8, FAKE, FAKE, gemv_need - 1, None) == 4

@@ -93,3 +93,25 @@ def route_experts(offsets):
     off = np.asarray(offsets)
     counts = np.diff(off)
     return np.repeat(np.arange(counts.size), counts)
+
+
+def gemm_views_e4m3(ws, T, k, D, F, two_sided):
+    """moe_trellis_gemm workspace of a pair-trellis (E4M3) layer: the same regions as
+    gemm_views, with the route-ordered x' rows as E4M3 bytes xr8 [R][D] and their
+    power-of-two scales x_scale [R] (in the row-sum slot), and h' as E4M3 bytes hr8 [R][F]
+    with hr_scale [R]."""
+    R = T * k
+    v = {}
+    off = 0
+    v["xr8"] = ws[0:R * D].view(torch.float8_e4m3fn).reshape(R, D)
+    off = _a256(R * D * 2)
+    v["x_scale"], off = _take(ws, off, R * 4, torch.float32, (R,))
+    if two_sided:
+        v["gu"], off = _take(ws, off, R * 2 * F * 4, torch.float32, (R, 2, F))
+    else:
+        v["h"], off = _take(ws, off, R * F * 4, torch.float32, (R, F))
+    v["hr8"] = ws[off:off + R * F].view(torch.float8_e4m3fn).reshape(R, F)
+    off += _a256(R * F * 2)
+    off += _a256(R * 4)                      # h' row sums (unused by the E4M3 path)
+    v["hr_scale"], off = _take(ws, off, R * 4, torch.float32, (R,))
+    return v

@@ -39,7 +39,10 @@ class TqMoeLayer(ctypes.Structure):
                 ("n_groups", ctypes.c_int), ("groups", TqWidthGroup * 3),
                 ("expert_slot", ctypes.c_void_p),
                 ("sign_x", ctypes.c_void_p), ("sign_gu", ctypes.c_void_p),
-                ("sign_h", ctypes.c_void_p), ("sign_y", ctypes.c_void_p)]
+                ("sign_h", ctypes.c_void_p), ("sign_y", ctypes.c_void_p),
+                ("codebook", ctypes.c_int)]
+
+CODEBOOKS = {"t16": 0, "pair_e4m3": 1}
 
 
 _lib = None
@@ -58,6 +61,7 @@ SIGNATURES = {
     "tq_profile_disable": ([], _I),
     "tq_profile_collect": ([_VP, _VP, _I], _I),
     "trellis_decode": ([_VP, _I, _I, _I, _VP, _VP], _I),
+    "trellis_decode_e4m3": ([_VP, _I, _I, _I, _VP, _VP], _I),
     "trellis_encode_workspace_size": ([_I, _I, _I], _SZ),
     "trellis_encode": ([_VP, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP], _I),
     "hadamard128": ([_VP, _I, _I64, _I64, _VP, _VP], _I),
@@ -192,6 +196,17 @@ def trellis_decode(bits: torch.Tensor, K: int, rows: int, cols: int,
         out = torch.empty((rows, cols), dtype=torch.float16, device=bits.device)
     _require(out, torch.float16, "out")
     _check(_fn("trellis_decode")(_p(bits), K, rows, cols, _p(out), _stream(stream)), "trellis_decode")
+    return out
+
+
+def trellis_decode_e4m3(bits: torch.Tensor, K: int, rows: int, cols: int,
+                        out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Pair-trellis bit streams -> E4M3 codes [rows, cols] (torch.float8_e4m3fn)."""
+    _require(bits, torch.int32, "bits")
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.float8_e4m3fn, device=bits.device)
+    _require(out, torch.float8_e4m3fn, "out")
+    _check(_fn("trellis_decode_e4m3")(_p(bits), K, rows, cols, _p(out), _stream(stream)), "trellis_decode_e4m3")
     return out
 
 
@@ -377,13 +392,16 @@ class DeviceLayer:
     `expert_slot[e] = (group << 16) | index` locates expert e.
     """
 
-    def __init__(self, E: int, D: int, F: int, groups: List[dict], device="cuda", signs: Optional[dict] = None):
+    def __init__(self, E: int, D: int, F: int, groups: List[dict], device="cuda", signs: Optional[dict] = None,
+                 codebook: str = "t16"):
         self.E, self.D, self.F = E, D, F
+        self.codebook = codebook
         self.device = torch.device(device)
         self.groups = []
         slot = np.full(E, -1, dtype=np.int32)
         st = TqMoeLayer()
         st.E, st.D, st.F, st.n_groups = E, D, F, len(groups)
+        st.codebook = CODEBOOKS[codebook]
         if not 1 <= len(groups) <= 3:
             raise ValueError("1..3 width groups")
         for gi, g in enumerate(groups):
@@ -423,7 +441,8 @@ class DeviceLayer:
     def from_synthetic(layer, device="cuda") -> "DeviceLayer":
         groups = [dict(K=g.K, ids=g.ids, gate=g.gate, up=g.up, down=g.down,
                        s_gate=g.s_gate, s_up=g.s_up, s_down=g.s_down) for g in layer.groups]
-        return DeviceLayer(layer.E, layer.D, layer.F, groups, device, getattr(layer, "signs", None))
+        return DeviceLayer(layer.E, layer.D, layer.F, groups, device, getattr(layer, "signs", None),
+                           getattr(layer, "codebook", "t16"))
 
     def compressed_bytes(self, experts) -> int:
         """Bit-stream + scale bytes of the given experts (all three projections)."""
@@ -512,8 +531,8 @@ def moe_layer(layer: DeviceLayer, x: torch.Tensor, logits: torch.Tensor, k: int,
         hadamard128_signed(x, layer.signs["x"], bufs.x_rot, stream)
     else:
         hadamard128(x, bufs.x_rot, stream)
-    use_gemm = path == "gemm" or (path == "auto" and T >= GEMM_MIN_TOKENS
-                                  and hasattr(lib(), "moe_trellis_gemm"))
+    use_gemm = (path == "gemm" or layer.codebook != "t16"      # the GEMV decodes T16 only
+                or (path == "auto" and T >= GEMM_MIN_TOKENS))
     fn = moe_trellis_gemm if use_gemm else moe_trellis_gemv
     fn(layer, bufs.x_rot, bufs.routing, T, k, bufs.y_perm, bufs.ws, stream)
     if layer.signs is not None:

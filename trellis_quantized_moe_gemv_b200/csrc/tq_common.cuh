@@ -215,4 +215,68 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, 
 
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 
+// ---------------------------------------------------------------------------- pair trellis
+// The exlr8 card's pmcgx codebook ("Stores"): two weights share a 20-bit state (pair q of
+// a tile reads stream bits 2Kq .. 2Kq + 19, tail-biting), each weight is the binary16 sum
+// of the two halves of the state's product with its multiplier (mod 2^32), bit 14 of
+// each half cleared, rounded to E4M3 (nearest even).  Pair q holds tile positions 2q and
+// 2q + 1, i.e. rows 2(q mod 8) and 2(q mod 8) + 1 of column q div 8.
+constexpr uint32_t kPairMultA = 0xCBAC1FEDu;
+constexpr uint32_t kPairMultB = 0xBCA14C51u;
+constexpr uint32_t kPairHalfMask = 0xBFFFBFFFu;   // bit 14 of both halves
+constexpr float kKappa8 = 1.0f / 32.0f;           // W = s * 2^-5 * w
+
+__device__ __forceinline__ uint32_t hadd2_rn(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// E4M3 bytes of two binary16 values (x: low half -> low byte), nearest even, saturating.
+__device__ __forceinline__ uint32_t e4m3x2_from_f16x2(uint32_t x) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(d) : "r"(x));
+    return d;
+}
+
+// 20-bit state of the pair whose window starts at compile-time bit offset O of v.
+template <int O, int NS>
+__device__ __forceinline__ uint32_t pair_state(const uint32_t (&v)[NS]) {
+    constexpr int wi = O >> 5, sh = O & 31;
+    const uint32_t x = sh == 0 ? v[wi] : funnel_r(v[wi], v[wi + 1], sh);
+    return x & 0xFFFFFu;
+}
+
+// E4M3 bytes of one weight for two pairs (columns c0, c1 of the same row): P0, P1 are the
+// two pairs' products with the weight's multiplier; the result's low byte is P0's weight.
+__device__ __forceinline__ uint32_t pair_weights_e4m3x2(uint32_t P0, uint32_t P1) {
+    const uint32_t lo = prmt(P0, P1, 0x5410u) & kPairHalfMask;   // {lo16(P0), lo16(P1)}
+    const uint32_t hi = prmt(P0, P1, 0x7632u) & kPairHalfMask;   // {hi16(P0), hi16(P1)}
+    return e4m3x2_from_f16x2(hadd2_rn(lo, hi));
+}
+
+// One lane cell of a tile: 16 rows x 4 consecutive columns (quarter t4: columns 4t4 ..
+// 4t4 + 3, i.e. pairs 32 t4 .. 32 t4 + 31).  v holds the 2K words of the quarter's
+// stream bits and the next word (tail-biting).  Writes the E4M3 bytes of row r, columns
+// 4t4 .. 4t4 + 3 (byte c = column 4t4 + c) to rows[r].
+template <int K, int I>
+__device__ __forceinline__ void pair_cell_rows(const uint32_t (&v)[2 * K + 1], uint32_t (&rows)[16]) {
+    if constexpr (I < 8) {
+        uint32_t pa[4], pb[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            // pair 8c + I of the quarter starts at bit 2K (8c + I) of the lane's words
+            const uint32_t st = c == 0 ? pair_state<2 * K * I>(v)
+                              : c == 1 ? pair_state<2 * K * (8 + I)>(v)
+                              : c == 2 ? pair_state<2 * K * (16 + I)>(v)
+                                       : pair_state<2 * K * (24 + I)>(v);
+            pa[c] = st * kPairMultA;
+            pb[c] = st * kPairMultB;
+        }
+        rows[2 * I] = prmt(pair_weights_e4m3x2(pa[0], pa[1]), pair_weights_e4m3x2(pa[2], pa[3]), 0x5410u);
+        rows[2 * I + 1] = prmt(pair_weights_e4m3x2(pb[0], pb[1]), pair_weights_e4m3x2(pb[2], pb[3]), 0x5410u);
+        pair_cell_rows<K, I + 1>(v, rows);
+    }
+}
+
 }  // namespace tq

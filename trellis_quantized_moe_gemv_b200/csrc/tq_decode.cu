@@ -60,7 +60,50 @@ __global__ void __launch_bounds__(256) trellis_decode_kernel(const uint32_t *__r
     }
 }
 
+// Standalone decode of a pair-trellis (E4M3) matrix: thread (tile, quarter t4) decodes the
+// 32 pairs of columns 4t4 .. 4t4 + 3 of its tile (pair_cell_rows) and stores each row's 4
+// bytes.  out is E4M3 bytes [rows][cols], row-major.
+template <int K>
+__global__ void __launch_bounds__(256) trellis_decode_e4m3_kernel(const uint32_t *__restrict__ bits, int rows,
+                                                                  int cols, uint8_t *__restrict__ out) {
+    const int tiles_per_row = cols / 16;
+    const long long n_cells = (long long)(rows / 16) * tiles_per_row * 4;
+    const long long cell = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (cell >= n_cells) return;
+    const int t4 = (int)(cell & 3);
+    const long long tile = cell >> 2;
+    const int strip = (int)(tile / tiles_per_row), tj = (int)(tile % tiles_per_row);
+    const uint32_t *w = bits + (size_t)tile * (8 * K);
+    uint32_t v[2 * K + 1];
+#pragma unroll
+    for (int i = 0; i < 2 * K; ++i) v[i] = __ldg(w + 2 * K * t4 + i);
+    v[2 * K] = __ldg(w + 2 * K * ((t4 + 1) & 3));   // next quarter's first word (tail-biting)
+    uint32_t r[16];
+    pair_cell_rows<K, 0>(v, r);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        *reinterpret_cast<uint32_t *>(out + (size_t)(strip * 16 + i) * cols + tj * 16 + 4 * t4) = r[i];
+}
+
 }  // namespace tq
+
+TQ_API int trellis_decode_e4m3(const uint32_t *bits, int K, int rows, int cols, uint8_t *out, tq_stream stream) {
+    if (K < 2 || K > 4 || rows < 0 || cols < 0 || rows % 16 || cols % 16) return TQ_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0) return TQ_OK;
+    if (!bits || !out) return TQ_ERR_INVALID_ARG;
+    if (!tq::aligned16(bits) || !tq::aligned16(out)) return TQ_ERR_ALIGNMENT;
+    const long long cells = (long long)(rows / 16) * (cols / 16) * 4;
+    if ((cells + 255) / 256 > 0x7fffffffll) return TQ_ERR_UNSUPPORTED;
+    const unsigned grid = (unsigned)((cells + 255) / 256);
+    cudaStream_t s = (cudaStream_t)stream;
+    tq::LaunchScope ls(s, tq::kStageDecode);
+    switch (K) {
+        case 2: tq::trellis_decode_e4m3_kernel<2><<<grid, 256, 0, s>>>(bits, rows, cols, out); break;
+        case 3: tq::trellis_decode_e4m3_kernel<3><<<grid, 256, 0, s>>>(bits, rows, cols, out); break;
+        default: tq::trellis_decode_e4m3_kernel<4><<<grid, 256, 0, s>>>(bits, rows, cols, out); break;
+    }
+    return tq::launch_status();
+}
 
 TQ_API int trellis_decode(const uint32_t *bits, int K, int rows, int cols, uint16_t *out,
                           tq_stream stream) {

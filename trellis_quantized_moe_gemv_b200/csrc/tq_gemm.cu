@@ -39,26 +39,41 @@ namespace tq {
 constexpr int kGBM = 128;          // weight rows per MMA tile (one accumulator)
 constexpr int kGTiles = 2;         // weight tiles per CTA: both share every activation slab
 constexpr int kGBN = 256;          // max routes per CTA
-constexpr int kGBK = 64;           // K columns per K-block
+constexpr int kGRowBytes = 128;    // bytes of one operand row per K-block (128-byte swizzle)
 constexpr int kGGroups = 2;        // K-block slots: K-block kb is decoded into A slot kb % 2
 constexpr int kGDecodeGroups = 2 * kGGroups;   // 4-warp groups: (K-block parity, weight tile)
-constexpr int kGBitsStages = 6;    // bit-stream ring (multiple of kGGroups)
+constexpr int kGBitsBytes = 48 * 1024;   // bit-stream ring: 6 stages (T16) or 3 (pair trellis)
 constexpr int kGBStages = 3;       // activation (B) ring
 constexpr int kGKbRing = 4;        // K-block barrier ring: > the A and B reuse distances
 constexpr int kGDecodeWarps = 4 * kGDecodeGroups;
 constexpr int kGFirstDecodeWarp = 3;   // warp 0: bit-stream producer, 1: MMA, 2: B producer
 constexpr int kGThreads = (kGFirstDecodeWarp + kGDecodeWarps) * 32;
 constexpr int kGStrips = 8 * kGTiles;  // 16-row strips per CTA
-constexpr int kGBitsSlot = 512;    // per strip per K-block: 4 tiles x up to 128 B
 constexpr int kGBoxes = 4;         // TMA boxes of 32, 64, 128, 256 rows
 constexpr uint32_t kGTmemCols = 512;   // two 256-column fp32 accumulators
+constexpr int kGMaxBitsStages = 6;
+
+// Per-codebook shape of a K-block.  T16 weights become fp16 operands (64 columns per
+// 128-byte row, kind::f16 MMAs of K = 16); pair-trellis weights become E4M3 operands (128
+// columns per row, kind::f8f6f4 MMAs of K = 32).  Either way a K-block is 4 MMAs per
+// weight tile and the operand rows are 128 bytes, so the shared-memory layout, the
+// swizzle and the descriptors are the same.
+template <bool FP8>
+struct GemmShape {
+    static constexpr int kTiles = FP8 ? 8 : 4;               // 16-column tiles per K-block
+    static constexpr int kCols = 16 * kTiles;                // K columns per K-block
+    static constexpr int kSlot = kTiles * 128;               // bit-stream bytes per strip (K <= 4)
+    static constexpr int kStage = kGStrips * kSlot;
+    static constexpr int kBitsStages = kGBitsBytes / kStage; // 6 or 3
+    static_assert(kBitsStages >= 2 && kBitsStages <= kGMaxBitsStages, "bit-stream ring");
+};
 
 struct __align__(1024) GemmSmem {
-    __half a[kGGroups][kGTiles][kGBM * kGBK];  // 2 x 16 KB per decode group, 1024-aligned
-    __half b[kGBStages][kGBN * kGBK];          // 32 KB per stage
-    unsigned char bits[kGBitsStages][kGStrips * kGBitsSlot];
-    uint64_t bits_full[kGBitsStages];          // producer -> decoders (count 1 + bytes)
-    uint64_t bits_empty[kGBitsStages];         // decoders -> producer (count 8)
+    unsigned char a[kGGroups][kGTiles][kGBM * kGRowBytes];  // 2 x 16 KB per decode group, 1024-aligned
+    unsigned char b[kGBStages][kGBN * kGRowBytes];          // 32 KB per stage
+    unsigned char bits[kGBitsBytes];                        // bit-stream stages (GemmShape)
+    uint64_t bits_full[kGMaxBitsStages];       // producer -> decoders (count 1 + bytes)
+    uint64_t bits_empty[kGMaxBitsStages];      // decoders -> producer (count 8)
     // One barrier pair per K-block (ring of kGKbRing): kb_ready completes when the 8
     // decode warps of the K-block have arrived and its activation slab has landed (the
     // MMA thread waits once per K-block); kb_done is the MMA commit, waited by the
@@ -144,6 +159,17 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// E4M3 x E4M3 -> fp32 (kind::f8f6f4, K = 32); the instruction descriptor's A and B format
+// fields are 0 (E4M3) in the same bit positions as kind::f16's fp16.
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -242,6 +268,53 @@ __device__ __forceinline__ void decode_cell(uint32_t bits_stage_s, uint32_t a_ti
     decode_rows<K, 0>(v, addr);
 }
 
+// Pair-trellis (E4M3) cell: 16 rows x 4 columns (quarter t4 of column tile j of strip
+// slot sig) decoded to E4M3 bytes and stored, 4 bytes per row, into the K-major
+// 128-byte-swizzled A buffer: row m = 16 sig + r, K byte 16 j + 4 t4 (16-byte chunk j,
+// swizzled by m mod 8).  Stage rows are 8 column tiles of one strip.
+template <int K>
+__device__ __forceinline__ void decode_cell_e4m3(uint32_t bits_stage_s, uint32_t a_tile_s, int sig, int row, int j,
+                                                 int t4) {
+    constexpr int TB = 32 * K;
+    const uint32_t tile = bits_stage_s + row * (8 * TB) + j * TB;
+    uint32_t v[2 * K + 1];
+    if constexpr (K == 2) {
+        uint4 a = lds128(tile + 16 * t4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else if constexpr (K == 3) {
+        const uint32_t q = tile + 24 * t4;
+        uint2 a = lds64(q), b = lds64(q + 8), c = lds64(q + 16);
+        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y; v[4] = c.x; v[5] = c.y;
+    } else {
+        const uint32_t q = tile + 32 * t4;
+        uint4 a = lds128(q), b = lds128(q + 16);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+    v[2 * K] = lds32(tile + 8 * K * ((t4 + 1) & 3));
+    uint32_t rows[16];
+    pair_cell_rows<K, 0>(v, rows);
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        const uint32_t addr = a_tile_s + (16 * sig + r) * 128 + ((j ^ (r & 7)) << 4) + 4 * t4;
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(rows[r]) : "memory");
+    }
+}
+
+// Decode weight tile t of one K-block (8 strips x 8 column tiles) of the pair trellis: the
+// 4-warp group's 128 threads take 2 cells each (same quarter t4, column tiles j, j + 4).
+template <int K, bool GATEUP>
+__device__ __forceinline__ void decode_tile_e4m3(uint32_t bits_stage_s, uint32_t a_tile_s, int t, int wl, int lane) {
+    const int t4 = lane & 3;
+    const int base = wl * 8 + (lane >> 2);   // 0..31: (strip slot, column tile mod 4)
+    const int sig = base >> 2;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int j = (base & 3) + 4 * h;
+        const int row = GATEUP ? (sig & 1) * 8 + 4 * t + (sig >> 1) : 8 * t + sig;
+        decode_cell_e4m3<K>(bits_stage_s, a_tile_s, sig, row, j, t4);
+    }
+}
+
 // Decode weight tile t of one K-block (8 strips x 4 column tiles) with a 4-warp group:
 // thread (wl, lane) takes one (strip slot, column tile, quarter) cell.  Rows of the
 // bit-stream stage: gate/up: [8 gate strips][8 up strips] of the tile pair (tile t,
@@ -267,9 +340,10 @@ struct GemmArgs {
     int raw_gu;                  // gate/up of the two-sided transform: store g and u, not h
 };
 
-template <bool GATEUP>
+template <bool GATEUP, bool FP8>
 __global__ void __launch_bounds__(kGThreads, 1)
     moe_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs args) {
+    using SH = GemmShape<FP8>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // The stage buffers need 1024-byte alignment (128-byte swizzle atoms).  Offset the
     // __shared__ array itself (no round trip through an integer) so that the compiler
@@ -293,10 +367,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     int box = 0;
     while ((32 << box) < n) ++box;          // box rows 32 << box >= n
     const int nmma = max(16, (n + 15) & ~15);
-    const int num_kb = args.kdim / kGBK;
+    const int num_kb = args.kdim / SH::kCols;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kGBitsStages; ++i) {
+        for (int i = 0; i < SH::kBitsStages; ++i) {
             mbar_init(&sm.bits_full[i], 1);
             mbar_init(&sm.bits_empty[i], 8);
         }
@@ -325,29 +399,30 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ bit-stream producer
         const int K = ex.K;
-        const int row_bytes = 4 * 32 * K;                     // 4 column tiles of one strip
+        const int row_bytes = SH::kTiles * 32 * K;            // the K-block's column tiles of one strip
         const CUtensorMap *m1 = &maps.bits_first[ex.group], *m2 = &maps.bits_second[ex.group];
         const int strip0 = GATEUP ? mt * 8 : mt * 16;         // first strip of the CTA
         int issued = 0;
         for (int kb = 0; kb < num_kb; ++kb) {
-            const int i = kb % kGBitsStages;
-            if (kb >= kGBitsStages && !wait(&sm.bits_empty[i], ((kb / kGBitsStages) - 1) & 1)) break;
+            const int i = kb % SH::kBitsStages;
+            if (kb >= SH::kBitsStages && !wait(&sm.bits_empty[i], ((kb / SH::kBitsStages) - 1) & 1)) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&sm.bits_full[i], (uint32_t)kGStrips * row_bytes);
-                const int x = kb * 4 * 8 * K;                 // word offset of the K-block
+                const int x = kb * SH::kTiles * 8 * K;        // word offset of the K-block
+                unsigned char *stage = sm.bits + i * SH::kStage;
                 if (GATEUP) {
-                    tma_load_3d(sm.bits[i], m1, x, strip0, ex.index, &sm.bits_full[i]);
-                    tma_load_3d(sm.bits[i] + 8 * row_bytes, m2, x, strip0, ex.index, &sm.bits_full[i]);
+                    tma_load_3d(stage, m1, x, strip0, ex.index, &sm.bits_full[i]);
+                    tma_load_3d(stage + 8 * row_bytes, m2, x, strip0, ex.index, &sm.bits_full[i]);
                 } else {
-                    tma_load_3d(sm.bits[i], m1, x, strip0, ex.index, &sm.bits_full[i]);
+                    tma_load_3d(stage, m1, x, strip0, ex.index, &sm.bits_full[i]);
                 }
             }
             __syncwarp();
             ++issued;
         }
         // drain: every issued copy has landed before the CTA can exit
-        for (int kb = max(0, issued - kGBitsStages); kb < issued; ++kb)
-            mbar_wait_sleep(&sm.bits_full[kb % kGBitsStages], (kb / kGBitsStages) & 1);
+        for (int kb = max(0, issued - SH::kBitsStages); kb < issued; ++kb)
+            mbar_wait_sleep(&sm.bits_full[kb % SH::kBitsStages], (kb / SH::kBitsStages) & 1);
     } else if (warp == 2) {
         // ------------------------------------------------------------ activation producer
         int issued = 0;
@@ -358,7 +433,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             uint64_t *ready = &sm.kb_ready[kb % kGKbRing];
             if (lane == 0) {
                 mbar_arrive_expect_tx(ready, (32u << box) * 128u);
-                tma_load_2d(sm.b[i], &maps.b[box], kb * kGBK, r0 + n0, ready);
+                tma_load_2d(sm.b[i], &maps.b[box], kb * SH::kCols, r0 + n0, ready);
             }
             __syncwarp();
             ++issued;
@@ -390,9 +465,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
                 for (int t = 0; t < kGTiles; ++t)
 #pragma unroll
-                    for (int k = 0; k < kGBK / 16; ++k)
-                        umma_f16(tmem_d + t * kGBN, a_desc0 + (uint64_t)((g * kGTiles + t) * a_step + 2 * k),
-                                 b_desc0 + (uint64_t)(i * b_step + 2 * k), idesc, (kb | k) != 0);
+                    for (int k = 0; k < 4; ++k) {   // 32-byte K steps: K = 16 fp16 or 32 E4M3
+                        const uint64_t ad = a_desc0 + (uint64_t)((g * kGTiles + t) * a_step + 2 * k);
+                        const uint64_t bd = b_desc0 + (uint64_t)(i * b_step + 2 * k);
+                        if constexpr (FP8) umma_e4m3(tmem_d + t * kGBN, ad, bd, idesc, (kb | k) != 0);
+                        else umma_f16(tmem_d + t * kGBN, ad, bd, idesc, (kb | k) != 0);
+                    }
                 umma_commit(&sm.kb_done[kb % kGKbRing]);
             }
         }
@@ -408,14 +486,20 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const int slot = dg >> 1, tile = dg & 1;
         const uint32_t a_s = smem_u32(sm.a[slot][tile]);
         for (int kb = slot; kb < num_kb; kb += kGGroups) {
-            const int i = kb % kGBitsStages;
-            if (!wait(&sm.bits_full[i], (kb / kGBitsStages) & 1)) break;
+            const int i = kb % SH::kBitsStages;
+            if (!wait(&sm.bits_full[i], (kb / SH::kBitsStages) & 1)) break;
             const int pk = kb - kGGroups;     // the K-block that last used this A slot
             if (pk >= 0 && !wait(&sm.kb_done[pk % kGKbRing], (pk / kGKbRing) & 1)) break;
-            const uint32_t bits_s = smem_u32(sm.bits[i]);
-            if (ex.K == 2) decode_tile<2, GATEUP>(bits_s, a_s, tile, wl, lane);
-            else if (ex.K == 3) decode_tile<3, GATEUP>(bits_s, a_s, tile, wl, lane);
-            else decode_tile<4, GATEUP>(bits_s, a_s, tile, wl, lane);
+            const uint32_t bits_s = smem_u32(sm.bits + i * SH::kStage);
+            if constexpr (FP8) {
+                if (ex.K == 2) decode_tile_e4m3<2, GATEUP>(bits_s, a_s, tile, wl, lane);
+                else if (ex.K == 3) decode_tile_e4m3<3, GATEUP>(bits_s, a_s, tile, wl, lane);
+                else decode_tile_e4m3<4, GATEUP>(bits_s, a_s, tile, wl, lane);
+            } else {
+                if (ex.K == 2) decode_tile<2, GATEUP>(bits_s, a_s, tile, wl, lane);
+                else if (ex.K == 3) decode_tile<3, GATEUP>(bits_s, a_s, tile, wl, lane);
+                else decode_tile<4, GATEUP>(bits_s, a_s, tile, wl, lane);
+            }
             fence_proxy_async();      // make the generic-proxy writes visible to the MMA
             __syncwarp();
             if (lane == 0) {
@@ -440,19 +524,20 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 const int col = cb + i;
                 float2 v = make_float2(0.f, 1.f);
                 if (col < n) {
-                    v.x = args.rowsum[r0 + n0 + col];
+                    if (args.rowsum) v.x = args.rowsum[r0 + n0 + col];
                     if (args.rowscale) v.y = args.rowscale[r0 + n0 + col];
                 }
                 rsw[i] = v;
             }
             const int f = (mtile * 4 + q) * 16 + (lane & 15);
             const int hi = lane >> 4;
-            float sk0, sk1 = 0.f;            // the lane's row scales times 2^-12
+            const float kappa = FP8 ? kKappa8 : kKappa;
+            float sk0, sk1 = 0.f;            // the lane's row scales times the codebook's normaliser
             if (GATEUP) {
-                sk0 = __half2float(ex.s_gate[f]) * kKappa;
-                sk1 = __half2float(ex.s_up[f]) * kKappa;
+                sk0 = __half2float(ex.s_gate[f]) * kappa;
+                sk1 = __half2float(ex.s_up[f]) * kappa;
             } else {
-                sk0 = __half2float(ex.s_down[mtile * kGBM + row]) * kKappa;
+                sk0 = __half2float(ex.s_down[mtile * kGBM + row]) * kappa;
             }
             __syncwarp();
             if (wait(&sm.acc_full, 0)) {
@@ -474,9 +559,17 @@ __global__ void __launch_bounds__(kGThreads, 1)
                             const int col = c0 + c + hi;
                             if (col < n) {
                                 const int route = r0 + n0 + col;
-                                const float sx = rsc[c + hi].x;
-                                const float g = sk0 * fmaf(16777216.0f, graw, -255.0f * sx);
-                                const float u = sk1 * fmaf(16777216.0f, uraw, -255.0f * sx);
+                                float g, u;
+                                if constexpr (FP8) {
+                                    // E4M3 codes are signed values; the route row's scale
+                                    const float xs = rsc[c + hi].y;
+                                    g = (sk0 * xs) * graw;
+                                    u = (sk1 * xs) * uraw;
+                                } else {
+                                    const float sx = rsc[c + hi].x;
+                                    g = sk0 * fmaf(16777216.0f, graw, -255.0f * sx);
+                                    u = sk1 * fmaf(16777216.0f, uraw, -255.0f * sx);
+                                }
                                 if (args.raw_gu) {
                                     args.out[(size_t)route * 2 * L.F + f] = g;
                                     args.out[((size_t)route * 2 + 1) * L.F + f] = u;
@@ -490,9 +583,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
                             const int col = c0 + c;
-                            if (col < n)
-                                args.out[(size_t)(r0 + n0 + col) * L.D + d] =
-                                    (sk0 * rsc[c].y) * fmaf(16777216.0f, __uint_as_float(v[c]), -255.0f * rsc[c].x);
+                            if (col < n) {
+                                float yv;
+                                if constexpr (FP8) yv = (sk0 * rsc[c].y) * __uint_as_float(v[c]);
+                                else yv = (sk0 * rsc[c].y) * fmaf(16777216.0f, __uint_as_float(v[c]), -255.0f * rsc[c].x);
+                                args.out[(size_t)(r0 + n0 + col) * L.D + d] = yv;
+                            }
                         }
                     }
                 }
@@ -622,6 +718,109 @@ __global__ void __launch_bounds__(256) swiglu_rows_kernel(const float *__restric
     if (lane == 0) rowsum[j] = sum;
 }
 
+// E4M3 bytes of four floats (v[0] in the lowest byte), nearest even, saturating.
+__device__ __forceinline__ uint32_t e4m3x4_from_f32(const float (&v)[4]) {
+    uint16_t lo, hi;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(v[1]), "f"(v[0]));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(v[3]), "f"(v[2]));
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+// Power of two 2^e that puts a row's largest magnitude m in (224, 448] (E4M3's largest
+// value is 448); 1 for a zero row.
+__device__ __forceinline__ int e4m3_row_exponent(float m) {
+    if (!(m > 0.f)) return 0;
+    int e = ilogbf(m) - 8;                       // m / 2^e in [256, 512)
+    if (ldexpf(m, -e) > 448.f) ++e;              // -> (224, 256)
+    return max(e, -100);
+}
+
+// Route-ordered E4M3 activation rows for the pair-trellis GEMM, one warp per destination
+// row j (source row perm[j] / k, or j when perm is null; ROTATE applies the 128-wide
+// rotation): the row is scaled by 2^-e (e4m3_row_exponent of its largest magnitude),
+// rounded to E4M3 and stored as bytes [j][cols]; rowscale[j] = 2^e.  The row is read twice.
+// An out-of-range source raises device flag bit 0 and stores zeros.
+template <typename T, bool ROTATE>
+__global__ void __launch_bounds__(256) route_rows_e4m3_kernel(const T *__restrict__ x, int dst_rows, int cols,
+                                                              const int32_t *__restrict__ perm, int k, int src_rows,
+                                                              uint8_t *__restrict__ dst, float *__restrict__ rowscale) {
+    const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (j >= dst_rows) return;
+    const int src = perm ? perm[j] / k : j;
+    const bool valid = src >= 0 && src < src_rows && (!perm || perm[j] >= 0);
+    if (!valid && lane == 0) raise_flag(1);
+    auto load = [&](int c, float (&v)[4]) {
+        v[0] = v[1] = v[2] = v[3] = 0.f;
+        if (valid) {
+            float4 f = load4<T>(x + (size_t)src * cols + c + 4 * lane);
+            v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+            if (ROTATE) fwht128_warp(v, lane);
+        }
+    };
+    float m = 0.f;
+    for (int c = 0; c < cols; c += 128) {
+        float v[4];
+        load(c, v);
+        m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fmaxf(fabsf(v[2]), fabsf(v[3])), m));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int e = e4m3_row_exponent(m);
+    const float inv = ldexpf(1.f, -e);
+    if (lane == 0) rowscale[j] = ldexpf(1.f, e);
+    for (int c = 0; c < cols; c += 128) {
+        float v[4];
+        load(c, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] *= inv;
+        *reinterpret_cast<uint32_t *>(dst + (size_t)j * cols + c + 4 * lane) = e4m3x4_from_f32(v);
+    }
+}
+
+// The two-sided transform between the pair-trellis GEMMs: as swiglu_rows_kernel, with
+// h' stored as E4M3 bytes of h' / 2^e (e4m3_row_exponent) and rowscale[j] = 2^e.
+__global__ void __launch_bounds__(256) swiglu_rows_e4m3_kernel(const float *__restrict__ gu, int rows, int F,
+                                                               const int8_t *__restrict__ sign_gu,
+                                                               const int8_t *__restrict__ sign_h,
+                                                               uint8_t *__restrict__ dst, float *__restrict__ rowscale) {
+    const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (j >= rows) return;
+    auto row_chunk = [&](int c, float (&h)[4]) {
+        const float4 g4 = load4<float>(gu + (size_t)j * 2 * F + c + 4 * lane);
+        const float4 u4 = load4<float>(gu + ((size_t)j * 2 + 1) * F + c + 4 * lane);
+        float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w};
+        fwht128_warp(g, lane);
+        fwht128_warp(u, lane);
+        const char4 so = *reinterpret_cast<const char4 *>(sign_gu + c + 4 * lane);
+        const char4 si = *reinterpret_cast<const char4 *>(sign_h + c + 4 * lane);
+        const float o[4] = {(float)so.x, (float)so.y, (float)so.z, (float)so.w};
+        const float in[4] = {(float)si.x, (float)si.y, (float)si.z, (float)si.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = silu_f32(g[i] * o[i]) * (u[i] * o[i]) * in[i];
+        fwht128_warp(h, lane);
+    };
+    float m = 0.f;
+    for (int c = 0; c < F; c += 128) {
+        float h[4];
+        row_chunk(c, h);
+        m = fmaxf(fmaxf(fabsf(h[0]), fabsf(h[1])), fmaxf(fmaxf(fabsf(h[2]), fabsf(h[3])), m));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int e = e4m3_row_exponent(m);
+    const float inv = ldexpf(1.f, -e);
+    if (lane == 0) rowscale[j] = ldexpf(1.f, e);
+    for (int c = 0; c < F; c += 128) {
+        float h[4];
+        row_chunk(c, h);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] *= inv;
+        *reinterpret_cast<uint32_t *>(dst + (size_t)j * F + c + 4 * lane) = e4m3x4_from_f32(h);
+    }
+}
+
 // Tiles of <= 256 routes per active expert: out[0] = count, then (expert, first route).
 __global__ void __launch_bounds__(1024) gemm_tile_list_kernel(const int32_t *__restrict__ offsets,
                                                               const int32_t *__restrict__ active_ids,
@@ -684,17 +883,20 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// Route-ordered fp16 activations [rows][cols] -> 4 maps with boxes of 64 columns x
-// {32, 64, 128, 256} rows and the 128-byte swizzle.
-static int make_maps(const __half *base, int rows, int cols, GemmMaps &maps) {
+// Route-ordered activations [rows][cols] (fp16, or E4M3 bytes) -> 4 maps with boxes of
+// one 128-byte row segment (64 fp16 or 128 E4M3 columns) x {32, 64, 128, 256} rows and
+// the 128-byte swizzle.
+static int make_maps(const void *base, int rows, int cols, bool e4m3, GemmMaps &maps) {
     auto enc = tensor_map_encoder();
     if (!enc) return record_error("cuTensorMapEncodeTiled entry point not found");
+    const size_t esize = e4m3 ? 1 : sizeof(__half);
     for (int b = 0; b < kGBoxes; ++b) {
         cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-        cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(__half)};
-        cuuint32_t box[2] = {(cuuint32_t)kGBK, (cuuint32_t)(32 << b)};
+        cuuint64_t strides[1] = {(cuuint64_t)cols * esize};
+        cuuint32_t box[2] = {(cuuint32_t)(kGRowBytes / esize), (cuuint32_t)(32 << b)};
         cuuint32_t estr[2] = {1, 1};
-        CUresult r = enc(&maps.b[b], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void *)base, dims, strides, box, estr,
+        CUresult r = enc(&maps.b[b], e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                         (void *)base, dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return record_error("cuTensorMapEncodeTiled failed");
@@ -703,8 +905,8 @@ static int make_maps(const __half *base, int rows, int cols, GemmMaps &maps) {
 }
 
 // Bit streams of every width group for one projection as a 3D uint32 tensor
-// [n_experts][n_strips][words_per_strip], box {4 tiles, box_strips, 1}.
-static int make_bits_maps(const tq_moe_layer *L, bool gateup, GemmMaps &maps) {
+// [n_experts][n_strips][words_per_strip], box {tiles_per_kb tiles, box_strips, 1}.
+static int make_bits_maps(const tq_moe_layer *L, bool gateup, int tiles_per_kb, GemmMaps &maps) {
     auto enc = tensor_map_encoder();
     if (!enc) return record_error("cuTensorMapEncodeTiled entry point not found");
     for (int g = 0; g < 3; ++g) {
@@ -719,7 +921,7 @@ static int make_bits_maps(const tq_moe_layer *L, bool gateup, GemmMaps &maps) {
             const cuuint64_t words = (cuuint64_t)tiles * 8 * G.K;
             cuuint64_t dims[3] = {words, (cuuint64_t)n_strips, (cuuint64_t)G.n_experts};
             cuuint64_t strides[2] = {words * 4, words * 4 * (cuuint64_t)n_strips};
-            cuuint32_t box[3] = {(cuuint32_t)(4 * 8 * G.K), (cuuint32_t)(gateup ? 8 : 16), 1};
+            cuuint32_t box[3] = {(cuuint32_t)(tiles_per_kb * 8 * G.K), (cuuint32_t)(gateup ? 8 : 16), 1};
             cuuint32_t estr[3] = {1, 1, 1};
             CUresult r = enc(dst, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, (void *)base, dims, strides, box, estr,
                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -746,29 +948,40 @@ size_t gemm_workspace_bytes(const tq_moe_layer *L, int T, int k) {
            align256_g((1 + 2 * (size_t)gemm_max_tiles(T, k, L->E)) * sizeof(int32_t));
 }
 
+template <bool FP8>
+static int set_gemm_smem() {
+    const int bytes = (int)(sizeof(GemmSmem) + 1024);
+    if (cudaFuncSetAttribute(moe_gemm_kernel<true, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(moe_gemm_kernel<false, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+            cudaSuccess)
+        return record_cuda_error("cudaFuncSetAttribute(moe_gemm_kernel)");
+    return TQ_OK;
+}
+
+// The routed experts through the tensor-core GEMM.  Workspace: route-ordered activation
+// rows (fp16 for T16; E4M3 bytes for the pair trellis) and one float per route (T16: the
+// row sum; pair trellis: the row's power-of-two scale), h (or g and u when two-sided),
+// the rotated h' rows (fp16 h' / 2^e, or E4M3), their row sums and scales, the tile list.
 int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offsets, const int32_t *perm,
                  const int32_t *active_ids, const int32_t *n_active, int T, int k, float *y_perm, void *ws,
                  cudaStream_t s) {
     static bool configured = false;
     if (!configured) {
-        const int bytes = (int)(sizeof(GemmSmem) + 1024);
-        if (cudaFuncSetAttribute(moe_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(moe_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-                cudaSuccess)
-            return record_cuda_error("cudaFuncSetAttribute(moe_gemm_kernel)");
+        if (set_gemm_smem<false>() || set_gemm_smem<true>()) return TQ_ERR_CUDA;
         configured = true;
     }
+    const bool fp8 = L->codebook == TQ_CODEBOOK_PAIR_E4M3;
     const int R = T * k;
     char *w = reinterpret_cast<char *>(ws);
-    __half *xp = reinterpret_cast<__half *>(w);
+    void *xp = w;
     w += align256_g((size_t)R * L->D * sizeof(__half));
-    float *sxp = reinterpret_cast<float *>(w);
+    float *sxp = reinterpret_cast<float *>(w);   // T16: row sums of x'; pair trellis: row scales
     w += align256_g((size_t)R * sizeof(float));
     const int two = L->sign_gu != nullptr;     // two-sided transform
     float *h = reinterpret_cast<float *>(w);   // h, or g and u when two-sided
     w += align256_g((size_t)R * (two ? 2 : 1) * L->F * sizeof(float));
-    __half *hr = reinterpret_cast<__half *>(w);
+    void *hr = w;
     w += align256_g((size_t)R * L->F * sizeof(__half));
     float *shr = reinterpret_cast<float *>(w);
     w += align256_g((size_t)R * sizeof(float));
@@ -778,16 +991,18 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     const int max_tiles = gemm_max_tiles(T, k, L->E);
 
     GemmMaps maps_x, maps_h;
-    int st = make_maps(xp, R, L->D, maps_x);
+    int st = make_maps(xp, R, L->D, fp8, maps_x);
     if (st) return st;
-    st = make_maps(hr, R, L->F, maps_h);
+    st = make_maps(hr, R, L->F, fp8, maps_h);
     if (st) return st;
-    st = make_bits_maps(L, true, maps_x);
+    const int tiles_per_kb = fp8 ? GemmShape<true>::kTiles : GemmShape<false>::kTiles;
+    st = make_bits_maps(L, true, tiles_per_kb, maps_x);
     if (st) return st;
-    st = make_bits_maps(L, false, maps_h);
+    st = make_bits_maps(L, false, tiles_per_kb, maps_h);
     if (st) return st;
 
     const size_t smem = sizeof(GemmSmem) + 1024;
+    const unsigned row_blocks = (unsigned)(((size_t)R * 32 + 255) / 256);
     {
         LaunchScope ls(s, kStageGemmPrep);
         gemm_tile_list_kernel<<<1, 1024, 0, s>>>(offsets, active_ids, n_active, max_tiles, tiles);
@@ -795,34 +1010,59 @@ int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
     st = launch_status();
     if (st) return st;
     {
-        // x_rot is already rotated: copy its rows to their route rows (+ row sums)
+        // x_rot is already rotated: copy its rows to their route rows (+ row sums, or as
+        // scaled E4M3)
         LaunchScope ls(s, kStageGemmPrep);
-        route_rows_kernel<__half, false><<<(R * 32 + 255) / 256, 256, 0, s>>>(x_rot, R, L->D, perm, k, T, xp, sxp,
-                                                                             nullptr);
+        if (fp8)
+            route_rows_e4m3_kernel<__half, false><<<row_blocks, 256, 0, s>>>(x_rot, R, L->D, perm, k, T,
+                                                                            reinterpret_cast<uint8_t *>(xp), sxp);
+        else
+            route_rows_kernel<__half, false><<<row_blocks, 256, 0, s>>>(x_rot, R, L->D, perm, k, T,
+                                                                       reinterpret_cast<__half *>(xp), sxp, nullptr);
     }
     st = launch_status();
     if (st) return st;
     {
-        GemmArgs a{*L, offsets, tiles, sxp, nullptr, h, L->D, two};
+        const dim3 grid(L->F / (64 * kGTiles), max_tiles);
         LaunchScope ls(s, kStageGemmGateUp);
-        moe_gemm_kernel<true><<<dim3(L->F / (64 * kGTiles), max_tiles), kGThreads, smem, s>>>(maps_x, a);
+        if (fp8) {
+            GemmArgs a{*L, offsets, tiles, nullptr, sxp, h, L->D, two};
+            moe_gemm_kernel<true, true><<<grid, kGThreads, smem, s>>>(maps_x, a);
+        } else {
+            GemmArgs a{*L, offsets, tiles, sxp, nullptr, h, L->D, two};
+            moe_gemm_kernel<true, false><<<grid, kGThreads, smem, s>>>(maps_x, a);
+        }
     }
     st = launch_status();
     if (st) return st;
     {
         LaunchScope ls(s, kStageRotateH);
-        if (two)
-            swiglu_rows_kernel<<<(R * 32 + 255) / 256, 256, 0, s>>>(h, R, L->F, L->sign_gu, L->sign_h, hr, shr, scr);
-        else
-            route_rows_kernel<float, true><<<(R * 32 + 255) / 256, 256, 0, s>>>(h, R, L->F, nullptr, 1, R, hr, shr,
-                                                                                scr);
+        if (fp8) {
+            uint8_t *h8 = reinterpret_cast<uint8_t *>(hr);
+            if (two)
+                swiglu_rows_e4m3_kernel<<<row_blocks, 256, 0, s>>>(h, R, L->F, L->sign_gu, L->sign_h, h8, scr);
+            else
+                route_rows_e4m3_kernel<float, true><<<row_blocks, 256, 0, s>>>(h, R, L->F, nullptr, 1, R, h8, scr);
+        } else {
+            __half *h16 = reinterpret_cast<__half *>(hr);
+            if (two)
+                swiglu_rows_kernel<<<row_blocks, 256, 0, s>>>(h, R, L->F, L->sign_gu, L->sign_h, h16, shr, scr);
+            else
+                route_rows_kernel<float, true><<<row_blocks, 256, 0, s>>>(h, R, L->F, nullptr, 1, R, h16, shr, scr);
+        }
     }
     st = launch_status();
     if (st) return st;
     {
-        GemmArgs a{*L, offsets, tiles, shr, scr, y_perm, L->F, 0};
+        const dim3 grid(L->D / (kGBM * kGTiles), max_tiles);
         LaunchScope ls(s, kStageGemmDown);
-        moe_gemm_kernel<false><<<dim3(L->D / (kGBM * kGTiles), max_tiles), kGThreads, smem, s>>>(maps_h, a);
+        if (fp8) {
+            GemmArgs a{*L, offsets, tiles, nullptr, scr, y_perm, L->F, 0};
+            moe_gemm_kernel<false, true><<<grid, kGThreads, smem, s>>>(maps_h, a);
+        } else {
+            GemmArgs a{*L, offsets, tiles, shr, scr, y_perm, L->F, 0};
+            moe_gemm_kernel<false, false><<<grid, kGThreads, smem, s>>>(maps_h, a);
+        }
     }
     return launch_status();
 }

@@ -839,6 +839,7 @@ int validate_layer(const tq_moe_layer *L) {
         return TQ_ERR_INVALID_ARG;
     if (L->D > kMaxCols || L->F > kMaxCols) return TQ_ERR_UNSUPPORTED;
     if (L->n_groups < 1 || L->n_groups > 3 || !L->expert_slot) return TQ_ERR_INVALID_ARG;
+    if (L->codebook != TQ_CODEBOOK_T16 && L->codebook != TQ_CODEBOOK_PAIR_E4M3) return TQ_ERR_INVALID_ARG;
     const int n_signs = !!L->sign_x + !!L->sign_gu + !!L->sign_h + !!L->sign_y;
     if (n_signs != 0 && n_signs != 4) return TQ_ERR_INVALID_ARG;   // all four or none
     for (const int8_t *sg : {L->sign_x, L->sign_gu, L->sign_h, L->sign_y})
@@ -999,6 +1000,7 @@ TQ_API int moe_trellis_gemv(const tq_moe_layer *layer, const uint16_t *x_rot, co
                             int k, float *y_perm, void *ws, size_t ws_bytes, tq_stream stream) {
     int st = moe_validate_call(layer, x_rot, offsets, perm, active_ids, n_active, T, k, y_perm, ws, ws_bytes);
     if (st || T == 0) return st;
+    if (layer->codebook != TQ_CODEBOOK_T16) return TQ_ERR_UNSUPPORTED;   // the GEMV decodes T16 only
     const __half *x = reinterpret_cast<const __half *>(x_rot);
     cudaStream_t s = (cudaStream_t)stream;
     return run_moe_gemv(layer, x, offsets, perm, active_ids, n_active, T, k, y_perm, ws, s);

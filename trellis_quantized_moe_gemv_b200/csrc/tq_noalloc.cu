@@ -59,6 +59,7 @@ TQ_API int moe_trellis_gemv_noalloc(const tq_moe_layer *layer, const uint16_t *x
     // the same argument statuses as moe_trellis_gemv, then the size of the call
     int st = moe_validate_args(layer, x_rot, offsets, perm, active_ids, n_active, T, k, y_perm);
     if (st || T == 0) return st;
+    if (layer->codebook != TQ_CODEBOOK_T16) return TQ_ERR_UNSUPPORTED;   // as moe_trellis_gemv
     if (tq::workspace_bytes(layer, T, k) > tq::kNoAllocScratchBytes) return TQ_ERR_WORKSPACE;
     void *scratch = nullptr;
     st = tq::noalloc_scratch(&scratch);

@@ -120,6 +120,8 @@ class SyntheticLayer:
     # Layer sign vectors of the two-sided transform (int8, +1/-1), shared by every
     # expert: x [D], gu [F], h [F], y [D]; None for the input-side-only layer.
     signs: Optional[dict] = None
+    # codebook of the bit streams: "t16" or "pair_e4m3" (same stored layout, K bits per weight)
+    codebook: str = "t16"
 
 
 def width_map(rng: np.random.Generator, E: int, split: dict) -> np.ndarray:
@@ -136,15 +138,17 @@ def width_map(rng: np.random.Generator, E: int, split: dict) -> np.ndarray:
 
 
 def make_layer(seed: int, E: int = E_EXPERTS, D: int = D_HIDDEN, F: int = F_INTER,
-               split: dict = None, uniform_K: int = None, name: str = "") -> SyntheticLayer:
+               split: dict = None, uniform_K: int = None, name: str = "",
+               codebook: str = "t16") -> SyntheticLayer:
     """A synthetic trellis-coded MoE layer with uniform random bit streams and U[0.5,1.5]
-    fp16 scales.  Either `split` (experts per width) or `uniform_K` is given."""
+    fp16 scales.  Either `split` (experts per width) or `uniform_K` is given; `codebook`
+    names how the streams are read ("t16" or "pair_e4m3")."""
     rng = np.random.default_rng(seed)
     if uniform_K is not None:
         expert_bits = np.full(E, uniform_K, dtype=np.int32)
     else:
         expert_bits = width_map(rng, E, split)
-    layer = SyntheticLayer(E=E, D=D, F=F, expert_bits=expert_bits, name=name, seed=seed)
+    layer = SyntheticLayer(E=E, D=D, F=F, expert_bits=expert_bits, name=name, seed=seed, codebook=codebook)
     for K in (2, 3, 4):
         ids = np.nonzero(expert_bits == K)[0].astype(np.int32)
         if ids.size == 0:
@@ -223,8 +227,19 @@ def with_signs(layer: SyntheticLayer, seed: int) -> SyntheticLayer:
 
 
 def small_layer(seed: int, E: int = 12, D: int = 256, F: int = 128, split: dict = None,
-                uniform_K: int = None):
+                uniform_K: int = None, codebook: str = "t16"):
     """A small layer for fast parity tests (dimensions multiples of 128)."""
     if split is None and uniform_K is None:
         split = {2: E - 3, 3: 2, 4: 1}
-    return make_layer(seed, E, D, F, split=split, uniform_K=uniform_K, name="small")
+    return make_layer(seed, E, D, F, split=split, uniform_K=uniform_K, name="small", codebook=codebook)
+
+
+def moe_prefill_t8192_fp8(seed: int = 1006, T: int = 8192, E: int = E_EXPERTS,
+                          D: int = D_HIDDEN, F: int = F_INTER):
+    """The prefill layer shape with pair-trellis (E4M3) streams, every expert K=3, 8192
+    tokens with Zipf(1.1)-skewed top-8 routing."""
+    layer = make_layer(seed, E, D, F, uniform_K=3, name="moe_prefill_t8192_fp8", codebook="pair_e4m3")
+    rng = np.random.default_rng(seed + 7)
+    x = random_activations(rng, (T, D), "bf16")
+    logits = zipf_gumbel_logits(rng, T, E)
+    return dict(layer=layer, x=x, logits=logits, k=TOP_K)
