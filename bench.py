@@ -202,11 +202,12 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workload
 
-def build_decode_workload(api, inputs, torch, device, rank, n_copies, two_sided=False):
+def build_decode_workload(api, inputs, torch, device, rank, n_copies, two_sided=False, T=16):
     """Layer copy 0 from the seeded numpy generators (the copy the parity tests check);
     copies 1..3 with the same widths, their bit streams and scales drawn on the device
-    from a seeded torch generator; every copy has its own tokens and logits."""
-    w0 = inputs.moe_decode_t16(seed=1003 + 100 * rank)
+    from a seeded torch generator; every copy has its own tokens and logits (T tokens:
+    16, or another count for profiling runs)."""
+    w0 = inputs.moe_decode_t16(seed=1003 + 100 * rank, T=T)
     host_layer = w0["layer"]
     layers, xs, logits = [], [], []
     if two_sided:
@@ -234,27 +235,30 @@ def build_decode_workload(api, inputs, torch, device, rank, n_copies, two_sided=
         layers.append(api.DeviceLayer(host_layer.E, host_layer.D, host_layer.F, groups, device, signs))
     for c in range(n_copies):
         rng = np.random.default_rng(9000 + 100 * rank + c)
-        x = w0["x"] if c == 0 else inputs.random_activations(rng, (16, host_layer.D), "bf16")
-        lg = w0["logits"] if c == 0 else inputs.normal_logits(rng, 16, host_layer.E)
+        x = w0["x"] if c == 0 else inputs.random_activations(rng, (T, host_layer.D), "bf16")
+        lg = w0["logits"] if c == 0 else inputs.normal_logits(rng, T, host_layer.E)
         xs.append((x, lg))
     return w0, layers, xs
 
 
-def gateup_algorithmic_bytes(layer, counts):
-    """Algorithmic bytes of one gate/up GEMV launch: the touched experts' gate and up bit
-    streams (K/8 B per weight) and scales, their tokens' rotated activations read once
-    per expert, and h written (fp32)."""
+def gemv_algorithmic_bytes(layer, counts):
+    """Algorithmic bytes of one fused GEMV launch (gate/up, SwiGLU and down of every
+    active expert): per expert with n routes, its gate, up and down bit streams (K/8 B per
+    weight) and scales, its routes' rotated activations read (2 B per value), g and u
+    written and read back (fp32), h' written and read (2 B per value) and y written
+    (fp32)."""
     K_of = {}
     for g in layer.groups:
         for e in g["ids"].tolist():
             K_of[e] = g["K"]
     total = 0
+    D, F = layer.D, layer.F
     for e, n in enumerate(counts):
         n = int(n)
         if n == 0:
             continue
-        total += 2 * layer.F * layer.D * K_of[e] // 8 + 2 * layer.F * 2
-        total += n * layer.D * 2 + n * layer.F * 4
+        total += 3 * F * D * K_of[e] // 8 + (2 * F + D) * 2
+        total += n * (D * 2 + 2 * F * 4 * 2 + F * 2 * 2 + D * 4)
     return total
 
 
@@ -279,8 +283,9 @@ def gateup_flops(layer, T, k):
 
 
 WORKLOADS = {
-    "moe_decode_t16": dict(T=16, path="gemv", stage="gemv_gateup",
-                           kernel="moe_gemv_items_kernel<1, 1> (gate/up GEMV, int8 tensor cores, 4 routes per pass)",
+    "moe_decode_t16": dict(T=16, path="gemv", stage="moe_gemv",
+                           kernel="moe_gemv_fused_kernel<1> (gate/up, SwiGLU and down GEMVs in one persistent launch, "
+                                  "int8 tensor cores, 4 routes per pass)",
                            widths="368/15/1 experts at K=2/3/4", routing="top-8 of N(0,1) logits"),
     "moe_prefill_t8192": dict(T=8192, path="gemm", stage="gemm_gateup",
                               kernel="moe_gemm_kernel<1> (gate/up tcgen05 GEMM + SiLU)",
@@ -313,10 +318,10 @@ def run_ours(args, rank, world, local_rank):
     wl = WORKLOADS[args.workload]
     T, k = (args.tokens or wl["T"]), 8
     if args.workload == "moe_decode_t16":
-        if args.tokens or args.experts:
-            raise SystemExit("--tokens/--experts apply to the prefill workload")
+        if args.experts:
+            raise SystemExit("--experts applies to the prefill workload")
         NL = args.layers
-        w0, layers, xs = build_decode_workload(api, inputs, torch, device, rank, NL, args.two_sided)
+        w0, layers, xs = build_decode_workload(api, inputs, torch, device, rank, NL, args.two_sided, T=T)
     else:
         NL = 1
         w0, layers, xs = build_prefill_workload(api, inputs, device, rank, T=T, E=args.experts or 384,
@@ -341,7 +346,9 @@ def run_ours(args, rank, world, local_rank):
     # the dominant kernel only, a second set of graphs, replayed after the timed region,
     # those of every stage.
     api.profile_enable(64 * NL)
-    api.profile_stages([wl["stage"]])
+    # the GEMV's stages: the fused launch, or (fewer than 32 routes) gate/up, h', down
+    timed_stages = ["moe_gemv", "rotate_h", "gemv_down"] if wl["path"] == "gemv" else [wl["stage"]]
+    api.profile_stages(timed_stages)
     api.profile_collect()
     launches0 = api.launch_count()
 
@@ -420,24 +427,28 @@ def run_ours(args, rank, world, local_rank):
     # HBM-bound) or FLOPs (prefill GEMM, tensor-bound) over its average duration; the
     # stage totals cover the last replay of each layer copy's graph (eager: every step)
     counts = [b.routing.counts.cpu().numpy() for b in bufs]
-    g_ms, g_n = stages[wl["stage"]]
+    split_gemv = wl["path"] == "gemv" and stages.get("gemv_down", (0.0, 0))[1] > 0
+    g_n = stages[wl["stage"]][1]
+    g_ms = sum(stages[n_][0] for n_ in timed_stages if n_ in stages) if split_gemv else stages[wl["stage"]][0]
     g_avg_ms = g_ms / max(g_n, 1)
+    kernel_label = ("moe_gemv_items_kernel x 2 + quantize_rows_kernel (the split form below 32 routes)"
+                    if split_gemv else wl["kernel"])
     stage_avg = {k_: v[0] / v[1] for k_, v in stage_breakdown.items() if v[1]}
     peaks, peak_src = load_peaks()
     if wl["path"] == "gemv":
-        per_copy_bytes = [gateup_algorithmic_bytes(L, c) for L, c in zip(layers, counts)]
+        per_copy_bytes = [gemv_algorithmic_bytes(L, c) for L, c in zip(layers, counts)]
         if args.eager:
             unit_work = sum(per_copy_bytes[i % NL] for i in range(args.steps)) / max(args.steps, 1)
         else:
             unit_work = sum(per_copy_bytes) / NL
         achieved = unit_work / (g_avg_ms * 1e-3) / 1e9
         peak = float(peaks["hbm_gbs"])
-        prof = profile_traffic("moe_gemv_gateup_decode_t16")
+        prof = profile_traffic("moe_gemv_fused_decode_t16")
         traffic = None
         if prof is not None:
             units = sum(int((c > 0).sum()) for c in counts) / NL
             traffic = float(prof["dram_bytes_per_unit"]) * units
-        roofline = {"kernel": wl["kernel"], "bound": "hbm", "achieved": achieved, "peak": peak,
+        roofline = {"kernel": kernel_label, "bound": "hbm", "achieved": achieved, "peak": peak,
                     "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_src + " (copy bandwidth)",
                     "bytes_per_launch": unit_work, "avg_launch_ms": g_avg_ms, "traffic": traffic}
     else:
@@ -742,32 +753,32 @@ def run_batch1(args, local_rank):
             torch.cuda.synchronize()
             api.profile_enable(64 * steps)
             api.profile_collect()
-            gu_bytes = dn_bytes = 0
+            gv_bytes = 0
             for i in range(steps):
                 flush.zero_()
                 api.moe_layer(L, data[i % 16][0], data[i % 16][1], k, bufs=bufs, path="gemv")
                 counts = bufs.routing.counts.cpu().numpy()
-                n_exp = int((counts > 0).sum())
-                gu_bytes += n_exp * (2 * F * D * K // 8 + 2 * F * 2) + T * D * 2 + T * k * 2 * F * 4
-                dn_bytes += n_exp * (D * F * K // 8 + D * 2) + T * k * F * 2 + T * k * D * 4
+                gv_bytes += gemv_algorithmic_bytes(L, counts)
             torch.cuda.synchronize()
             st = api.profile_collect()
             api.profile_disable()
             if api.device_status():
                 raise RuntimeError("device anomaly flags during the batch-1 measurement")
-            gu_ms = st["gemv_gateup"][0] / max(st["gemv_gateup"][1], 1)
-            dn_ms = st["gemv_down"][0] / max(st["gemv_down"][1], 1)
+            # the routed-expert GEMV: one fused launch, or (small batches) gate/up items, the
+            # h' quantisation and down items
+            split = st.get("gemv_down", (0.0, 0))[1] > 0
+            gv_stages = ("moe_gemv", "rotate_h", "gemv_down") if split else ("moe_gemv",)
+            gv_ms = sum(st[n][0] for n in gv_stages if n in st) / steps
             step_ms = sum(v[0] for v in st.values()) / steps
             hbm = float(peaks["hbm_gbs"])
-            gu_gbs = gu_bytes / steps / (gu_ms * 1e-3) / 1e9
-            dn_gbs = dn_bytes / steps / (dn_ms * 1e-3) / 1e9
+            gv_gbs = gv_bytes / steps / (gv_ms * 1e-3) / 1e9
             print(json.dumps({
                 "metric": "decode GEMV HBM GB/s on compressed bytes", "workload": "moe_gemv_single_width_K%d_t%d" % (K, T),
                 "K": K, "tokens": T, "top_k": k, "steps": steps, "l2": "512 MB written before every step",
-                "gateup": {"avg_launch_ms": gu_ms, "bytes_per_launch": gu_bytes / steps, "achieved_gbs": gu_gbs,
-                           "frac": gu_gbs / hbm},
-                "down": {"avg_launch_ms": dn_ms, "bytes_per_launch": dn_bytes / steps, "achieved_gbs": dn_gbs,
-                         "frac": dn_gbs / hbm},
+                "gemv": {"kernel": ("moe_gemv_items_kernel (gate/up) + quantize_rows_kernel (h') + moe_gemv_items_kernel "
+                                    "(down)" if split else "moe_gemv_fused_kernel (gate/up, SwiGLU, down)"),
+                         "avg_launch_ms": gv_ms,
+                         "bytes_per_launch": gv_bytes / steps, "achieved_gbs": gv_gbs, "frac": gv_gbs / hbm},
                 "layer_device_ms": step_ms, "layer_tok_s": T / (step_ms * 1e-3),
                 "peak": hbm, "peak_source": src + " (copy bandwidth)"}), flush=True)
             del bufs, data

@@ -102,8 +102,10 @@ int tq_device_status(int32_t *flags_out, int clear);
  * counterpart on the pages).  Every kernel launch increments a host counter.  While
  * profiling is enabled, each launch is bracketed by two CUDA events recorded on its
  * stream and tagged with its stage:
- *   0 route_topk, 1 route_permute, 2 hadamard128 of the input, 3 GEMV gate/up+SiLU,
- *   4 rotation of h, 5 GEMV down, 6 route_unpermute, 7 trellis_decode, 8 trellis_gemv,
+ *   0 route_topk, 1 route_permute, 2 hadamard128 of the input, 3 MoE GEMV (the fused
+ *   launch: gate/up, SwiGLU with the rotation of h, and down; or, for the smallest
+ *   batches, the gate/up launch), 4 rotation (and, GEMV, quantisation) of h, 5 MoE GEMV
+ *   down launch of the smallest batches, 6 route_unpermute, 7 trellis_decode, 8 trellis_gemv,
  *   9 GEMM gate/up+SiLU, 10 GEMM down, 11 GEMM preparation (tile list, route-ordered
  *   activation rows), 12 GEMV activation quantisation (x' rows to 16-bit fixed point),
  *   13 trellis_encode, 14 route_gather_rows.
@@ -190,9 +192,11 @@ int hadamard128_signed(const void *x, int x_dtype, int64_t rows, int64_t cols, c
  *            bytes, 16-byte aligned (TQ_ERR_WORKSPACE otherwise).
  *   rows % 16 == 0, cols % 128 == 0, cols <= 16384, K in {2, 3, 4}.
  * Numerics: each row of x_rot enters the tensor-core contraction as 16-bit fixed point
- * with one power-of-two scale per row (|x_q| <= 32639, rounded to nearest), codes
- * exactly; sums are exact in int32 and the scales are applied in double.  Elements
- * smaller than 1/32 of their row's largest are rounded to that row's step.
+ * x_q = rint(x / 2^e) with one power-of-two scale per row (|x_q| <= 32639), codes exactly;
+ * sums are exact in int32 and the scales are applied in double.  A row whose rounding
+ * step is coarse for its mass (2^(e-1) * cols > 2^-12 * sum |x|) also carries its residual
+ * as a second 16-bit word at 2^(e-15), i.e. it is 32-bit fixed point.  Error per element:
+ * at most 2^(e-1) (one word) or 2^(e-16) (two words).
  */
 size_t trellis_gemv_workspace_size(int rows, int cols, int batch);
 int trellis_gemv(const uint32_t *bits, const uint16_t *scales, int K, int rows, int cols,
@@ -334,10 +338,13 @@ typedef struct {
 
 /*
  * Workspace bytes moe_trellis_gemv and moe_trellis_gemm need for T tokens and k routes
- * (the larger of the two).  GEMV: the gate and up results of every route ([T*k][2][F]
- * fp32), the rotated SwiGLU activations h' and the rotated
- * tokens x' as 16-bit fixed point (two half-words per value plus 8 bytes per row).  GEMM: route-ordered fp16 activation rows, row sums,
- * h and h' and the tile list.  Returns 0 on invalid arguments.
+ * (the larger of the two).  GEMV: the gate and up results of every route ([T*k][S][2][F]
+ * fp32, S column splits), the rotated SwiGLU activations h' and the rotated tokens x' as
+ * fixed point (four half-word planes per value, 16 bytes per row) and the counters of its
+ * work queue.  GEMM: route-ordered activation rows and their sums or scales, h, h' with
+ * its sums and scales, and the tile list.  The split count S depends on the device's SM
+ * count, so query the size on the device that runs the call.  Returns 0 on invalid
+ * arguments.
  */
 size_t moe_trellis_workspace_size(const tq_moe_layer *layer, int T, int k);
 
@@ -352,10 +359,16 @@ size_t moe_trellis_workspace_size(const tq_moe_layer *layer, int T, int k);
  *   offsets, perm, active_ids, n_active : from route_permute (device).
  *   y_perm   : [T*k][D] fp32, expert-grouped route order.
  *   ws       : device workspace of at least moe_trellis_workspace_size() bytes.
- *   Mixed widths run in one launch per stage; routes of an expert are processed
- *   together, each weight decoded once per 4 of its routes.  x' and h' enter the
- *   tensor-core contraction as 16-bit fixed point with one power-of-two scale per row
- *   (as in trellis_gemv); h' is rotated from fp32 h without an fp16 rounding.
+ *   From 32 routes (T*k): two launches, the fixed-point quantisation of x', then one
+ *   persistent kernel that takes gate/up items and then down items from a work queue; the
+ *   CTA finishing an expert's last gate/up item computes that expert's h' (SwiGLU,
+ *   rotation, quantisation) and its down items wait for it.  Below 32 routes: four
+ *   launches (x' quantisation, gate/up, h', down) with the same arithmetic.  Mixed
+ *   widths run in the same launches; routes of an
+ *   expert are processed together, each weight decoded once per 4 (or 8) of its routes.
+ *   x' and h' enter the tensor-core contraction as fixed point with one power-of-two
+ *   scale per row (as in trellis_gemv: 16 bits, 32 for a row whose rounding step is
+ *   coarse for its mass); h' is rotated from fp32 h without an fp16 rounding.
  *   D, F <= 16384.
  */
 int moe_trellis_gemv(const tq_moe_layer *layer, const uint16_t *x_rot, const int32_t *offsets,
@@ -373,9 +386,10 @@ int moe_trellis_gemv(const tq_moe_layer *layer, const uint16_t *x_rot, const int
  *   is a 4 MiB array compiled into the library (a __device__ array every GPU that loads
  *   the library holds until exit), so the GEMV workspace -- 8 * S * T * k * F (gate/up
  *   results, S = 1..8 column splits for small batches) + 8 * T * k * F + 8 * T * D bytes
- *   (fixed-point h' and x', two words each) plus 16 bytes per row, each part rounded up
- *   to 256 bytes; T <= 25 at k = 8, D = 4096, F = 1024 -- must fit in it; larger calls
- *   return TQ_ERR_WORKSPACE without doing anything.
+ *   (fixed-point h' and x', two words each) plus 16 bytes per row and 4 * (1 + 2E) bytes
+ *   of work-queue counters, each part rounded up to 256 bytes; T <= 25 at k = 8, E = 384,
+ *   D = 4096, F = 1024 -- must fit in it; larger calls return TQ_ERR_WORKSPACE without
+ *   doing anything.
  *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   Arguments are checked first, with the same statuses as moe_trellis_gemv; then a call
  *   whose workspace would not fit returns TQ_ERR_WORKSPACE.

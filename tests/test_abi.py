@@ -126,6 +126,7 @@ def test_moe_workspace_and_layer_validation(lib):
     # column splits: min(8, ceil(3 * SMs / 32), D / 128)), h' and x' as fixed point (four
     # half-word planes per value: main and residual word) and 16 bytes of metadata per row
     gemv_need = 128 * 2 * 2 * 128 * 4 + 128 * 4 * 128 * 2 + 128 * 16 + 16 * 4 * 256 * 2 + 256
+    gemv_need += 256     # the fused kernel's work queue and per-expert counters: (1 + 2E) ints
     # the GEMM path also holds route-ordered activations (fp16), their row sums, h, h',
     # its row sums and power-of-two row scales, and the tile list
     gemm_need = 128 * 256 * 2 + 512 + 128 * 128 * 4 + 128 * 128 * 2 + 512 + 512 + 256

@@ -150,7 +150,7 @@ def device_status(clear: bool = False) -> int:
     return out.value
 
 
-STAGES = ("route_topk", "route_permute", "rotate_x", "gemv_gateup", "rotate_h", "gemv_down",
+STAGES = ("route_topk", "route_permute", "rotate_x", "moe_gemv", "rotate_h", "gemv_down",
           "route_unpermute", "trellis_decode", "trellis_gemv", "gemm_gateup", "gemm_down", "gemm_prep",
           "gemv_quant", "trellis_encode", "route_gather")
 

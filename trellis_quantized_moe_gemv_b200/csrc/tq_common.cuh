@@ -33,7 +33,7 @@ inline bool aligned8(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 7
 // ---------------------------------------------------------------------------- profiling
 // Stage tags of the library's kernel launches (tq_profile_* in the C ABI).
 enum Stage {
-    kStageTopk = 0, kStagePermute = 1, kStageRotateX = 2, kStageGemvGateUp = 3,
+    kStageTopk = 0, kStagePermute = 1, kStageRotateX = 2, kStageMoeGemv = 3,
     kStageRotateH = 4, kStageGemvDown = 5, kStageUnpermute = 6, kStageDecode = 7,
     kStageGemv = 8, kStageGemmGateUp = 9, kStageGemmDown = 10, kStageGemmPrep = 11,
     kStageGemvQuant = 12, kStageEncode = 13, kStageGather = 14, kNumStages = 15

@@ -163,14 +163,26 @@ __device__ __forceinline__ void ring_issue(const WarpRing &ring, int st, int c, 
 // Activation half-words of the lane's 4 columns of tile j (null row: zeros): each
 // 16-bit value holds one signed byte twice, so a 32-bit word [x_c x_c x_c+1 x_c+1]
 // is the B operand of column c+1 (bytes 2, 3) and, shifted left by 16, of column c.
+// FRESH: the rows were written earlier in this same launch (published by a release and
+// picked up by a gpu-scope acquire before the read), so they take plain coherent loads,
+// which may hit L1, instead of the read-only path.
+__device__ __forceinline__ uint2 ld_weak_v2(const uint2 *p) {
+    uint2 v;
+    asm volatile("ld.global.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
+template <bool FRESH = false>
 __device__ __forceinline__ uint2 x_halves(const uint16_t *xw, int j, int t4) {
-    return xw ? __ldg(reinterpret_cast<const uint2 *>(xw + 16 * j + 4 * t4)) : make_uint2(0u, 0u);
+    if (!xw) return make_uint2(0u, 0u);
+    const uint2 *p = reinterpret_cast<const uint2 *>(xw + 16 * j + 4 * t4);
+    return FRESH ? ld_weak_v2(p) : __ldg(p);
 }
 
 // Stream tiles [j0, je) of the 8 strips against the lane's activation rows xw[b] (the
 // lane's limb of route 4b + g/2 of the pass, or null); activations are loaded one tile
 // ahead.  Returns false, after draining its copies, if a bounded wait gave up.
-template <int K, int NB>
+template <int K, int NB, bool FRESH = false>
 __device__ __forceinline__ bool stream_range(const WarpRing &ring, uint32_t &parity, int j0, int je,
                                              const uint32_t *strip_lane, const uint16_t *const (&xw)[NB],
                                              AccI<NB> &acc) {
@@ -181,7 +193,7 @@ __device__ __forceinline__ bool stream_range(const WarpRing &ring, uint32_t &par
     for (int c = 0; c < min(kStages, n_chunks); ++c) ring_issue<K>(ring, c, c, j0, je, strip_lane);
     uint2 xn[NB];
 #pragma unroll
-    for (int b = 0; b < NB; ++b) xn[b] = j0 < je ? x_halves(xw[b], j0, t4) : make_uint2(0u, 0u);
+    for (int b = 0; b < NB; ++b) xn[b] = j0 < je ? x_halves<FRESH>(xw[b], j0, t4) : make_uint2(0u, 0u);
     for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kStages;
         const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&ring.bar[st], (parity >> st) & 1u));
@@ -222,7 +234,7 @@ __device__ __forceinline__ bool stream_range(const WarpRing &ring, uint32_t &par
             const int jn = jb + t + 1;
             if (jn < je) {
 #pragma unroll
-                for (int b = 0; b < NB; ++b) xn[b] = x_halves(xw[b], jn, t4);
+                for (int b = 0; b < NB; ++b) xn[b] = x_halves<FRESH>(xw[b], jn, t4);
             }
             tile_rows<K, NB, 0>(v, x, acc);
         }
@@ -232,13 +244,13 @@ __device__ __forceinline__ bool stream_range(const WarpRing &ring, uint32_t &par
     return true;
 }
 
-template <int NB>
+template <int NB, bool FRESH = false>
 __device__ __forceinline__ bool stream_any(int K, const WarpRing &ring, uint32_t &parity, int j0, int je,
                                            const uint32_t *strip_lane, const uint16_t *const (&xw)[NB],
                                            AccI<NB> &acc) {
-    if (K == 2) return stream_range<2, NB>(ring, parity, j0, je, strip_lane, xw, acc);
-    if (K == 3) return stream_range<3, NB>(ring, parity, j0, je, strip_lane, xw, acc);
-    return stream_range<4, NB>(ring, parity, j0, je, strip_lane, xw, acc);
+    if (K == 2) return stream_range<2, NB, FRESH>(ring, parity, j0, je, strip_lane, xw, acc);
+    if (K == 3) return stream_range<3, NB, FRESH>(ring, parity, j0, je, strip_lane, xw, acc);
+    return stream_range<4, NB, FRESH>(ring, parity, j0, je, strip_lane, xw, acc);
 }
 
 // Shared-memory partials of the CTA's warps; aliases the stage buffers (never the
@@ -303,8 +315,9 @@ __device__ __forceinline__ void split_range(int n, int part, int parts, int &b, 
 // xq[row][0][col] = xh * 0x0101, xq[row][1][col] = xl * 0x0101.  When
 // 2^(e-1) * cols > 2^-12 * sum |v| the row also gets its residual word
 // r_q = rint((v - x_q 2^e) / 2^(e-15)) (|r_q| <= 2^14; v - x_q 2^e is exact in fp32) in
-// planes 2 and 3.  meta[row] = (e, sum x_q, residual flag, sum r_q).  The row is read
-// again in the second pass instead of being kept in registers, so any row length works.
+// planes 2 and 3.  meta[row] = (e, sum x_q, residual flag, sum r_q).  A warp keeps its
+// first KEPT chunks in registers between the two passes; further chunks (rows longer
+// than KEPT * 128 * WARPS) are read again in the second pass.
 
 // Plain rows x[row][cols].
 template <typename T>
@@ -318,46 +331,88 @@ struct RowSrc {
 };
 
 // SwiGLU of the gate/up GEMV's column-split partial sums: h = silu(sum_s g_s) * sum_s u_s
-// from gu[row][s][0][cols] (gate) and gu[row][s][1][cols] (up).
+// from gu[row][s][0][cols] (gate) and gu[row][s][1][cols] (up), summed in split order.
 // sign_gu (optional): the output side of the two-sided transform, applied to g and u
 // before the SwiGLU: g = sign_gu * rotate(g), u likewise.
+__device__ __forceinline__ void swiglu_finish(float4 g, float4 u, const int8_t *sign_gu, int c, int lane,
+                                              float (&v)[4]) {
+    float gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w};
+    if (sign_gu) {
+        fwht128_warp(gv, lane);
+        fwht128_warp(uv, lane);
+        const char4 sg = *reinterpret_cast<const char4 *>(sign_gu + c * 128 + 4 * lane);
+        const float s4[4] = {(float)sg.x, (float)sg.y, (float)sg.z, (float)sg.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            gv[i] *= s4[i];
+            uv[i] *= s4[i];
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = silu_f32(gv[i]) * uv[i];
+}
+
+// The partials read from global memory through L2 (the h' quantisation launch).
 struct SwigluSrc {
     const float *gu;
     int cols, splits;
     const int8_t *sign_gu;
     __device__ __forceinline__ void load(int row, int c, int lane, float (&v)[4]) const {
         const float *p = gu + (size_t)row * splits * 2 * cols + (size_t)c * 128 + 4 * lane;
-        float4 g = *reinterpret_cast<const float4 *>(p), u = *reinterpret_cast<const float4 *>(p + cols);
+        float4 g = __ldcg(reinterpret_cast<const float4 *>(p)), u = __ldcg(reinterpret_cast<const float4 *>(p + cols));
         for (int sp = 1; sp < splits; ++sp) {
-            const float4 g2 = *reinterpret_cast<const float4 *>(p + (size_t)sp * 2 * cols);
-            const float4 u2 = *reinterpret_cast<const float4 *>(p + (size_t)sp * 2 * cols + cols);
+            const float4 g2 = __ldcg(reinterpret_cast<const float4 *>(p + (size_t)sp * 2 * cols));
+            const float4 u2 = __ldcg(reinterpret_cast<const float4 *>(p + (size_t)sp * 2 * cols + cols));
             g.x += g2.x; g.y += g2.y; g.z += g2.z; g.w += g2.w;
             u.x += u2.x; u.y += u2.y; u.z += u2.z; u.w += u2.w;
         }
-        float gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w};
-        if (sign_gu) {
-            fwht128_warp(gv, lane);
-            fwht128_warp(uv, lane);
-            const char4 sg = *reinterpret_cast<const char4 *>(sign_gu + c * 128 + 4 * lane);
-            const float s4[4] = {(float)sg.x, (float)sg.y, (float)sg.z, (float)sg.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                gv[i] *= s4[i];
-                uv[i] *= s4[i];
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = silu_f32(gv[i]) * uv[i];
+        swiglu_finish(g, u, sign_gu, c, lane, v);
     }
 };
 
-template <typename Src, bool ROTATE>
-__global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int cols, const int8_t *__restrict__ signs,
-                                                            uint16_t *__restrict__ xq, RowQ *__restrict__ meta) {
-    chain_entry();
-    __shared__ float s_max[8], s_l1[8];
-    __shared__ int s_sum[8], s_rsum[8];
-    const int row = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// The same inside the fused kernel.  staged: gu is one route's [s][2][cols] already in
+// shared memory (stage_row_async; the row argument is ignored); otherwise the partials
+// are read from global memory through L2 (they were written by other CTAs of the same
+// launch).
+struct SwigluFusedSrc {
+    const float *gu;
+    int cols, splits;
+    const int8_t *sign_gu;
+    bool staged;
+    __device__ __forceinline__ float4 ld(const float *p) const {
+        return staged ? *reinterpret_cast<const float4 *>(p) : __ldcg(reinterpret_cast<const float4 *>(p));
+    }
+    __device__ __forceinline__ void load(int row, int c, int lane, float (&v)[4]) const {
+        const float *p = gu + (staged ? 0 : (size_t)row * splits * 2 * cols) + (size_t)c * 128 + 4 * lane;
+        float4 g = ld(p), u = ld(p + cols);
+        for (int sp = 1; sp < splits; ++sp) {
+            const float4 g2 = ld(p + (size_t)sp * 2 * cols), u2 = ld(p + (size_t)sp * 2 * cols + cols);
+            g.x += g2.x; g.y += g2.y; g.z += g2.z; g.w += g2.w;
+            u.x += u2.x; u.y += u2.y; u.z += u2.z; u.w += u2.w;
+        }
+        swiglu_finish(g, u, sign_gu, c, lane, v);
+    }
+};
+
+// One route's split partials (bytes, a multiple of 16) copied from global memory into
+// shared memory with 16-byte cp.async copies through L2, all in flight at once; returns
+// after the CTA's copies have landed.
+__device__ __forceinline__ void stage_row_async(unsigned char *dst, const float *src, int bytes) {
+    const uint32_t d = smem_u32(dst);
+    const char *g = reinterpret_cast<const char *>(src);
+    for (int o = threadIdx.x * 16; o < bytes; o += kItemThreads * 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d + o), "l"(g + o) : "memory");
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+}
+
+// One row quantised by the whole CTA (WARPS warps); the s_* arrays hold WARPS entries.
+// KEPT: 128-value chunks per warp kept in registers between the two passes.
+template <int WARPS, typename Src, bool ROTATE, int KEPT>
+__device__ __forceinline__ void quantize_row(const Src &src, int row, int cols, const int8_t *__restrict__ signs,
+                                             uint16_t *__restrict__ xq, RowQ *__restrict__ meta, float *s_max,
+                                             float *s_l1, int *s_sum, int *s_rsum) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int chunks = cols / 128;
     auto load = [&](int c, float (&v)[4]) {
         src.load(row, c, lane, v);
@@ -369,8 +424,23 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int c
             fwht128_warp(v, lane);
         }
     };
+    // pass 1: max |v| and sum |v|, chunks in increasing order (the first KEPT of
+    // the warp's chunks stay in registers)
     float m = 0.f, l1 = 0.f;
-    for (int c = warp; c < chunks; c += 8) {
+    float kept[KEPT > 0 ? KEPT : 1][4];
+#pragma unroll
+    for (int j = 0; j < KEPT; ++j) {
+        const int c = warp + j * WARPS;
+        if (c < chunks) {
+            load(c, kept[j]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                m = fmaxf(m, fabsf(kept[j][i]));
+                l1 += fabsf(kept[j][i]);
+            }
+        }
+    }
+    for (int c = warp + KEPT * WARPS; c < chunks; c += WARPS) {
         float v[4];
         load(c, v);
 #pragma unroll
@@ -392,7 +462,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int c
     m = s_max[0];
     l1 = s_l1[0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) {
+    for (int w = 1; w < WARPS; ++w) {
         m = fmaxf(m, s_max[w]);
         l1 += s_l1[w];
     }
@@ -405,9 +475,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int c
     const bool res = m > 0.f && ldexpf((float)cols, e - 1) > ldexpf(l1, -kResBudgetLog2);
     uint16_t *qh = xq + (size_t)row * 4 * cols, *ql = qh + cols, *rh = ql + cols, *rl = rh + cols;
     int sum = 0, rsum = 0;
-    for (int c = warp; c < chunks; c += 8) {
-        float v[4];
-        load(c, v);
+    auto quantize_chunk = [&](int c, const float (&v)[4]) {
         uint32_t wh[4], wl[4], vh[4], vl[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -436,6 +504,17 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int c
             *reinterpret_cast<uint2 *>(rh + off) = make_uint2(vh[0] | (vh[1] << 16), vh[2] | (vh[3] << 16));
             *reinterpret_cast<uint2 *>(rl + off) = make_uint2(vl[0] | (vl[1] << 16), vl[2] | (vl[3] << 16));
         }
+    };
+    // pass 2: quantise and store
+#pragma unroll
+    for (int j = 0; j < KEPT; ++j) {
+        const int c = warp + j * WARPS;
+        if (c < chunks) quantize_chunk(c, kept[j]);
+    }
+    for (int c = warp + KEPT * WARPS; c < chunks; c += WARPS) {
+        float v[4];
+        load(c, v);
+        quantize_chunk(c, v);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -449,21 +528,38 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Src src, int c
     __syncthreads();
     if (threadIdx.x == 0) {
         int total = 0, rtotal = 0;
-        for (int w = 0; w < 8; ++w) {
+        for (int w = 0; w < WARPS; ++w) {
             total += s_sum[w];
             rtotal += s_rsum[w];
         }
         meta[row] = RowQ{e, total, res ? 1 : 0, rtotal};
     }
+    __syncthreads();   // the s_* arrays are reused by the next row
 }
 
-template <bool ROTATE, typename Src>
+// One CTA of WARPS warps per row.  zero (optional): the first CTA also clears zero[0,
+// n_zero) (the fused GEMV's queue and expert counters, used by the kernel that follows).
+template <typename Src, bool ROTATE, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32) quantize_rows_kernel(const Src src, int cols,
+                                                                   const int8_t *__restrict__ signs,
+                                                                   uint16_t *__restrict__ xq, RowQ *__restrict__ meta,
+                                                                   int *__restrict__ zero, int n_zero) {
+    chain_entry();
+    __shared__ float s_max[WARPS], s_l1[WARPS];
+    __shared__ int s_sum[WARPS], s_rsum[WARPS];
+    if (zero && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
+    quantize_row<WARPS, Src, ROTATE, 32 / WARPS>(src, blockIdx.x, cols, signs, xq, meta, s_max, s_l1, s_sum, s_rsum);
+}
+
+template <bool ROTATE, typename Src, int WARPS = 8>
 int launch_quantize_rows(const Src &src, long long rows, int cols, uint16_t *xq, RowQ *meta, cudaStream_t s,
-                         int stage, const int8_t *signs = nullptr) {
+                         int stage, const int8_t *signs = nullptr, int *zero = nullptr, int n_zero = 0) {
     if (rows <= 0) return TQ_OK;
     if (rows > 0x7fffffffll) return TQ_ERR_UNSUPPORTED;
     LaunchScope ls(s, stage);
-    launch_chained(quantize_rows_kernel<Src, ROTATE>, (unsigned)rows, 256, 0, s, src, cols, signs, xq, meta);
+    launch_chained(quantize_rows_kernel<Src, ROTATE, WARPS>, (unsigned)rows, WARPS * 32, 0, s, src, cols, signs, xq,
+                   meta, zero, n_zero);
     return launch_status();
 }
 
@@ -514,6 +610,8 @@ __device__ __forceinline__ bool expert_ref(const tq_moe_layer &L, int e, ExpertR
 // !GATEUP: item = (active expert, 128 output rows); activations = quantised h'
 //          (indexed by route); out = y [routes][D] fp32.
 constexpr int kNb2MinRoutes = 5;
+// routes from which the three GEMV stages run as one fused launch (below: the split form)
+constexpr int kFusedMinRoutes = 32;
 constexpr int kMaxGateUpSplits = 8;
 
 // Column splits of the gate/up items: enough CTAs for ~3 per SM at the batch's largest
@@ -538,34 +636,38 @@ struct PassSlots {
     int next;
 };
 
-template <bool GATEUP, int NB>
-__global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
-    moe_gemv_items_kernel(const tq_moe_layer L, const uint16_t *__restrict__ xq, const RowQ *__restrict__ xmeta,
-                          const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm,
-                          const int32_t *__restrict__ active_ids, const int32_t *__restrict__ n_active_p,
-                          int k, int n_routes, int gu_splits, float *__restrict__ out) {
-    chain_entry();
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    ItemSmem &sm_items = *reinterpret_cast<ItemSmem *>(smem_raw);
-    ItemRed<NB> &red = *reinterpret_cast<ItemRed<NB> *>(smem_raw);
-    __shared__ PassSlots<NB> ps;
+// Metadata of an activation row (FRESH: written earlier in this launch, plain coherent load).
+template <bool FRESH>
+__device__ __forceinline__ RowQ load_rowq(const RowQ *p) {
+    if constexpr (FRESH) {
+        int4 v;
+        asm volatile("ld.global.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+        return RowQ{v.x, v.y, v.z, v.w};
+    } else {
+        return *p;
+    }
+}
+
+// One work item (see above) on the CTA's warp rings.  Returns false if a bounded wait
+// gave up (the CTA must stop; every warp drained its copies first).  An expert id the
+// layer does not hold raises device flag bit 0 and the item is skipped.  FRESH: activation
+// rows and their metadata were written earlier in this launch (x_halves).
+template <bool GATEUP, int NB, bool FRESH>
+__device__ __forceinline__ bool gemv_item(const tq_moe_layer &L, int item, int splits, const uint16_t *__restrict__ xq,
+                                          const RowQ *__restrict__ xmeta, const int32_t *__restrict__ offsets,
+                                          const int32_t *__restrict__ perm, const int32_t *__restrict__ active_ids,
+                                          int k, int n_routes, float *__restrict__ out, const WarpRing &ring,
+                                          uint32_t &parity, ItemRed<NB> &red, PassSlots<NB> &ps) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2;
-    const int splits = GATEUP ? gu_splits : 1;
     constexpr int NS = 4 * NB;
     const int per_expert = (GATEUP ? L.F / 64 : L.D / 128) * splits;
-    const int item = blockIdx.x;
-    if (item >= *n_active_p * per_expert) return;
     const int a = item / per_expert, sub = (item % per_expert) / splits, sp = item % splits;
     const int e = active_ids[a];
     ExpertRef ex;
     if (!expert_ref(L, e, ex)) {
         if (threadIdx.x == 0) raise_flag(1);
-        return;
+        return true;
     }
-    const WarpRing ring{sm_items.buf[warp], sm_items.bar[warp]};
-    ring_init(ring);
-    uint32_t parity = 0;
-
     const int cols = GATEUP ? L.D : L.F;
     const int r0 = offsets[e], ne = offsets[e + 1] - r0;
     const int tiles = cols / 16;
@@ -593,7 +695,7 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
                 } else {
                     row = r0 + tt;
                 }
-                need = (row >= 0 && xmeta[row].res) ? 2 : 1;
+                need = (row >= 0 && load_rowq<FRESH>(xmeta + row).res) ? 2 : 1;
             }
             ps.cand[threadIdx.x] = row;
             ps.need[threadIdx.x] = need;
@@ -627,9 +729,9 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
         }
         AccI<NB> acc;
         zero(acc);
-        bool ok = stream_any<NB>(ex.K, ring, parity, jb, je, strip_lane, xw, acc);
+        bool ok = stream_any<NB, FRESH>(ex.K, ring, parity, jb, je, strip_lane, xw, acc);
         ok = __syncthreads_and(ok);
-        if (!ok) return;   // every warp drained its copies; the item is left unwritten
+        if (!ok) return false;   // every warp drained its copies; the item is left unwritten
         store_partials(acc, red);   // the rings are idle now
         __syncthreads();
         if (GATEUP) {
@@ -640,7 +742,7 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
                 const int f = (sub * 4 + st) * 16 + row;
                 float gv = 0.f, uv = 0.f;    // a route with an invalid index: h = 0
                 if (xrow >= 0) {
-                    RowQ m = xmeta[xrow];
+                    RowQ m = load_rowq<FRESH>(xmeta + xrow);
                     if (sp) m.sum = m.rsum = 0;   // the -255 sum x term is added once, by split 0
                     const int2 g = red_sum(red, st, row, rt), u = red_sum(red, st + 4, row, rt);
                     int2 g2 = make_int2(0, 0), u2 = make_int2(0, 0);
@@ -660,7 +762,7 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
                 const int rt = i % NS, row = (i / NS) & 15, st = i / (16 * NS);
                 const int xrow = ps.row[rt];
                 if (xrow < 0 || ps.word[rt] != 0) continue;
-                const RowQ m = xmeta[xrow];
+                const RowQ m = load_rowq<FRESH>(xmeta + xrow);
                 const int2 y = red_sum(red, st, row, rt);
                 const int2 y2 = m.res ? red_sum(red, st, row, rt + 1) : make_int2(0, 0);
                 const int d = (sub * 8 + st) * 16 + row;
@@ -669,6 +771,143 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
         }
         tb = ps.next;
         __syncthreads();   // the rings and the pass slots are reused by the next pass
+    }
+    return true;
+}
+
+// Waits (thread 0) until *flag is non-zero, polling through L2 with a sleep between
+// polls; gives up after kFlagWaitNs (device flag bit 1).  Returns whether it was set.
+constexpr uint64_t kFlagWaitNs = 2000000000ull;
+// Polls with relaxed loads (an acquire load would invalidate the SM's L1 at every poll,
+// under the feet of the other CTAs there); the fence after the load that saw the flag
+// makes it an acquire of the producer's release.
+__device__ __forceinline__ bool wait_flag(const int *flag) {
+    uint64_t t0 = 0;
+    for (uint32_t n = 0;; ++n) {
+        int v;
+        asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v) {
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            return true;
+        }
+        if (n == 0) t0 = global_timer_ns();
+        else if ((n & 15) == 0 && global_timer_ns() - t0 > kFlagWaitNs) break;
+        __nanosleep(200);
+    }
+    raise_flag(2);
+    return false;
+}
+
+__device__ __forceinline__ void set_flag(int *flag) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
+}
+
+// The split form for the smallest batches: one CTA per work item (blockIdx.x; CTAs past
+// the active experts' items exit at once), gate/up and down as two launches with the h'
+// quantisation between them.  Below kFusedMinRoutes routes a decode step's critical path
+// is a chain of dependent global-memory round trips, which kernel boundaries with
+// programmatic dependent launch shorten more than the fused kernel's flags do.
+template <bool GATEUP, int NB>
+__global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
+    moe_gemv_items_kernel(const tq_moe_layer L, const uint16_t *__restrict__ xq, const RowQ *__restrict__ xmeta,
+                          const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm,
+                          const int32_t *__restrict__ active_ids, const int32_t *__restrict__ n_active_p, int k,
+                          int n_routes, int gu_splits, float *__restrict__ out) {
+    chain_entry();
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    ItemSmem &sm_items = *reinterpret_cast<ItemSmem *>(smem_raw);
+    ItemRed<NB> &red = *reinterpret_cast<ItemRed<NB> *>(smem_raw);
+    __shared__ PassSlots<NB> ps;
+    const int warp = threadIdx.x >> 5;
+    const int splits = GATEUP ? gu_splits : 1;
+    const int per_expert = (GATEUP ? L.F / 64 : L.D / 128) * splits;
+    if ((int)blockIdx.x >= *n_active_p * per_expert) return;
+    const WarpRing ring{sm_items.buf[warp], sm_items.bar[warp]};
+    ring_init(ring);
+    uint32_t parity = 0;
+    gemv_item<GATEUP, NB, false>(L, blockIdx.x, splits, xq, xmeta, offsets, perm, active_ids, k, n_routes, out, ring,
+                                 parity, red, ps);
+}
+
+// The routed experts' GEMVs of one decode step in one persistent launch.  Every CTA takes
+// work items from a queue (sync[0]): first every gate/up item (expert by expert), then
+// every down item.  The CTA that completes the last gate/up item of an expert (counter
+// sync[1 + a]) applies the SwiGLU, the rotation and the fixed-point quantisation to that
+// expert's routes (h') and raises the expert's ready flag sync[1 + E + a]; a down item
+// waits for its expert's flag.  A CTA only waits for work that a running CTA has already
+// taken (down items come after every gate/up item in the queue), so the waits end; each is
+// bounded all the same.  The arithmetic is that of the separate kernels, so the results
+// are the same bit for bit.  sync[] is cleared by the x' quantisation kernel before.
+template <int NB>
+__global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
+    moe_gemv_fused_kernel(const tq_moe_layer L, const uint16_t *__restrict__ xq, const RowQ *__restrict__ xmeta,
+                          float *__restrict__ gu, uint16_t *__restrict__ hq, RowQ *__restrict__ hmeta,
+                          const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm,
+                          const int32_t *__restrict__ active_ids, const int32_t *__restrict__ n_active_p, int k,
+                          int n_routes, int gu_splits, int *__restrict__ sync, float *__restrict__ y_perm) {
+    chain_entry();
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    ItemSmem &sm_items = *reinterpret_cast<ItemSmem *>(smem_raw);
+    ItemRed<NB> &red = *reinterpret_cast<ItemRed<NB> *>(smem_raw);
+    __shared__ PassSlots<NB> ps;
+    __shared__ int s_item, s_flag;
+    __shared__ float s_max[kItemWarps], s_l1[kItemWarps];
+    __shared__ int s_sum[kItemWarps], s_rsum[kItemWarps];
+    const int warp = threadIdx.x >> 5;
+    const int n_active = *n_active_p;
+    const int gu_per = (L.F / 64) * gu_splits, dn_per = L.D / 128;
+    const int n_gu = n_active * gu_per, n_all = n_gu + n_active * dn_per;
+    const WarpRing ring{sm_items.buf[warp], sm_items.bar[warp]};
+    ring_init(ring);
+    uint32_t parity = 0;
+    for (;;) {
+        if (threadIdx.x == 0) s_item = atomicAdd(&sync[0], 1);
+        __syncthreads();
+        const int item = s_item;
+        if (item >= n_all) break;
+        if (item < n_gu) {
+            if (!gemv_item<true, NB, false>(L, item, gu_splits, xq, xmeta, offsets, perm, active_ids, k, n_routes, gu,
+                                            ring, parity, red, ps))
+                break;
+            // publish this item's g and u; the last of the expert's items turns them into h'
+            const int a = item / gu_per;
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) s_flag = atomicAdd(&sync[1 + a], 1) == gu_per - 1;
+            __syncthreads();
+            if (s_flag) {
+                __threadfence();
+                const int e = active_ids[a];
+                if (e >= 0 && e < L.E) {
+                    const int r0 = offsets[e], r1 = offsets[e + 1];
+                    // a route's partials (splits x 2 x F fp32) are staged in the idle ring
+                    // buffers when they fit, so that their L2 reads overlap (both passes
+                    // of the quantisation then read shared memory)
+                    const int row_bytes = gu_splits * 2 * L.F * (int)sizeof(float);
+                    const bool staged = row_bytes <= (int)sizeof(sm_items.buf);
+                    unsigned char *st = &sm_items.buf[0][0][0];
+                    for (int r = r0; r < r1; ++r) {
+                        if (staged) stage_row_async(st, gu + (size_t)r * gu_splits * 2 * L.F, row_bytes);
+                        const SwigluFusedSrc src{staged ? reinterpret_cast<const float *>(st) : gu, L.F, gu_splits,
+                                                 L.sign_gu, staged};
+                        quantize_row<kItemWarps, SwigluFusedSrc, true, 0>(src, r, L.F, L.sign_h, hq, hmeta, s_max,
+                                                                          s_l1, s_sum, s_rsum);
+                    }
+                }
+                __threadfence();
+                __syncthreads();
+                if (threadIdx.x == 0) set_flag(&sync[1 + L.E + a]);
+            }
+        } else {
+            const int d = item - n_gu, a = d / dn_per;
+            if (threadIdx.x == 0) s_flag = wait_flag(&sync[1 + L.E + a]);
+            __syncthreads();
+            if (s_flag &&
+                !gemv_item<false, NB, true>(L, d, 1, hq, hmeta, offsets, perm, active_ids, k, n_routes, y_perm, ring,
+                                            parity, red, ps))
+                break;
+        }
+        __syncthreads();   // s_item and s_flag are rewritten by the next item
     }
 }
 
@@ -863,12 +1102,16 @@ struct MoeGemvWs {
     RowQ *hmeta;
     uint16_t *xq;
     RowQ *xmeta;
+    int *sync;      // fused kernel: work queue, per-expert gate/up counters and h' flags
 };
+
+inline size_t sync_ints(const tq_moe_layer *L) { return 1 + 2 * (size_t)L->E; }
 
 size_t workspace_bytes(const tq_moe_layer *L, int T, int k) {
     const size_t routes = (size_t)T * k;
     return align256(routes * gate_up_splits(L, T, k) * 2 * L->F * 4) + align256(routes * 4 * L->F * 2) +
-           align256(routes * sizeof(RowQ)) + align256((size_t)T * 4 * L->D * 2) + align256((size_t)T * sizeof(RowQ));
+           align256(routes * sizeof(RowQ)) + align256((size_t)T * 4 * L->D * 2) + align256((size_t)T * sizeof(RowQ)) +
+           align256(sync_ints(L) * sizeof(int));
 }
 
 MoeGemvWs moe_gemv_ws(const tq_moe_layer *L, int T, int k, void *ws) {
@@ -884,6 +1127,8 @@ MoeGemvWs moe_gemv_ws(const tq_moe_layer *L, int T, int k, void *ws) {
     w.xq = reinterpret_cast<uint16_t *>(p);
     p += align256((size_t)T * 4 * L->D * 2);
     w.xmeta = reinterpret_cast<RowQ *>(p);
+    p += align256((size_t)T * sizeof(RowQ));
+    w.sync = reinterpret_cast<int *>(p);
     return w;
 }
 
@@ -892,44 +1137,70 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
                  void *ws, cudaStream_t s) {
     const size_t smem = sizeof(ItemSmem);
     static bool configured = false;
+    static int resident[3] = {0, 0, 0};   // CTAs per SM of the fused kernel, NB = 1, 2
     if (!configured) {
-        if (set_smem(moe_gemv_items_kernel<true, 1>, smem) || set_smem(moe_gemv_items_kernel<false, 1>, smem) ||
+        if (set_smem(moe_gemv_fused_kernel<1>, smem) || set_smem(moe_gemv_fused_kernel<2>, smem) ||
+            set_smem(moe_gemv_items_kernel<true, 1>, smem) || set_smem(moe_gemv_items_kernel<false, 1>, smem) ||
             set_smem(moe_gemv_items_kernel<true, 2>, smem) || set_smem(moe_gemv_items_kernel<false, 2>, smem))
             return TQ_ERR_CUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[1], moe_gemv_fused_kernel<1>, kItemThreads,
+                                                          smem) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[2], moe_gemv_fused_kernel<2>, kItemThreads,
+                                                          smem) != cudaSuccess)
+            return record_cuda_error("cudaOccupancyMaxActiveBlocksPerMultiprocessor");
         configured = true;
     }
     const int routes = T * k;
     const MoeGemvWs w = moe_gemv_ws(L, T, k, ws);
-    const int max_active = min(L->E, routes);
+    const long long max_active = min(L->E, routes);
     const int splits = gate_up_splits(L, T, k);
-    const int gu_items = max_active * (L->F / 64) * splits;
-    const int dn_items = max_active * (L->D / 128);
-    int st = launch_quantize_rows<false>(RowSrc<__half>{x_rot, L->D}, T, L->D, w.xq, w.xmeta, s, kStageGemvQuant);
-    if (st) return st;
+    const long long max_items = max_active * ((long long)(L->F / 64) * splits + L->D / 128);
     // 8 routes per pass once a batch averages kNb2MinRoutes or more routes per expert
     // (each decoded weight then feeds twice the MMAs instead of being decoded twice)
     const bool nb2 = routes >= kNb2MinRoutes * min(L->E, routes);
-    {
-        LaunchScope ls(s, kStageGemvGateUp);
+    const int nb = nb2 ? 2 : 1;
+    if (routes < kFusedMinRoutes) {
+        // split form: x' quantisation, gate/up items, h' quantisation, down items
+        const unsigned gu_items = (unsigned)(max_active * (L->F / 64) * splits);
+        const unsigned dn_items = (unsigned)(max_active * (L->D / 128));
+        int st = launch_quantize_rows<false>(RowSrc<__half>{x_rot, L->D}, T, L->D, w.xq, w.xmeta, s, kStageGemvQuant);
+        if (st) return st;
+        {
+            LaunchScope ls(s, kStageMoeGemv);
+            if (nb2)
+                launch_chained(moe_gemv_items_kernel<true, 2>, gu_items, kItemThreads, smem, s, *L, w.xq, w.xmeta,
+                               offsets, perm, active_ids, n_active, k, routes, splits, w.gu);
+            else
+                launch_chained(moe_gemv_items_kernel<true, 1>, gu_items, kItemThreads, smem, s, *L, w.xq, w.xmeta,
+                               offsets, perm, active_ids, n_active, k, routes, splits, w.gu);
+        }
+        st = launch_status();
+        if (st) return st;
+        st = launch_quantize_rows<true>(SwigluSrc{w.gu, L->F, splits, L->sign_gu}, routes, L->F, w.hq, w.hmeta, s,
+                                        kStageRotateH, L->sign_h);
+        if (st) return st;
+        LaunchScope ls(s, kStageGemvDown);
         if (nb2)
-            launch_chained(moe_gemv_items_kernel<true, 2>, gu_items, kItemThreads, smem, s, *L, w.xq, w.xmeta, offsets,
-                           perm, active_ids, n_active, k, routes, splits, w.gu);
+            launch_chained(moe_gemv_items_kernel<false, 2>, dn_items, kItemThreads, smem, s, *L, w.hq, w.hmeta, offsets,
+                           perm, active_ids, n_active, k, routes, 1, y_perm);
         else
-            launch_chained(moe_gemv_items_kernel<true, 1>, gu_items, kItemThreads, smem, s, *L, w.xq, w.xmeta, offsets,
-                           perm, active_ids, n_active, k, routes, splits, w.gu);
+            launch_chained(moe_gemv_items_kernel<false, 1>, dn_items, kItemThreads, smem, s, *L, w.hq, w.hmeta, offsets,
+                           perm, active_ids, n_active, k, routes, 1, y_perm);
+        return launch_status();
     }
-    st = launch_status();
+    // x' rows to fixed point; the same launch clears the fused kernel's queue and counters
+    int st = launch_quantize_rows<false>(RowSrc<__half>{x_rot, L->D}, T, L->D, w.xq, w.xmeta, s, kStageGemvQuant,
+                                         nullptr, w.sync, (int)sync_ints(L));
     if (st) return st;
-    st = launch_quantize_rows<true>(SwigluSrc{w.gu, L->F, splits, L->sign_gu}, routes, L->F, w.hq, w.hmeta, s,
-                                    kStageRotateH, L->sign_h);
-    if (st) return st;
-    LaunchScope ls(s, kStageGemvDown);
+    const long long slots = (long long)max(1, resident[nb]) * num_sms();
+    const unsigned grid = (unsigned)max(1ll, min(slots, max_items));
+    LaunchScope ls(s, kStageMoeGemv);
     if (nb2)
-        launch_chained(moe_gemv_items_kernel<false, 2>, dn_items, kItemThreads, smem, s, *L, w.hq, w.hmeta, offsets,
-                       perm, active_ids, n_active, k, routes, 1, y_perm);
+        launch_chained(moe_gemv_fused_kernel<2>, grid, kItemThreads, smem, s, *L, w.xq, w.xmeta, w.gu, w.hq, w.hmeta,
+                       offsets, perm, active_ids, n_active, k, routes, splits, w.sync, y_perm);
     else
-        launch_chained(moe_gemv_items_kernel<false, 1>, dn_items, kItemThreads, smem, s, *L, w.hq, w.hmeta, offsets,
-                       perm, active_ids, n_active, k, routes, 1, y_perm);
+        launch_chained(moe_gemv_fused_kernel<1>, grid, kItemThreads, smem, s, *L, w.xq, w.xmeta, w.gu, w.hq, w.hmeta,
+                       offsets, perm, active_ids, n_active, k, routes, splits, w.sync, y_perm);
     return launch_status();
 }
 
