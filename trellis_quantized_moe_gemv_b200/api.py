@@ -516,7 +516,7 @@ class MoeBuffers:
                               device=dev)
 
 
-GEMM_MIN_TOKENS = 360   # measured crossover of the two paths on the 384-expert decode layer
+GEMM_MIN_TOKENS = 340   # measured crossover of the two paths on the 384-expert decode layer
 
 
 def moe_layer(layer: DeviceLayer, x: torch.Tensor, logits: torch.Tensor, k: int,

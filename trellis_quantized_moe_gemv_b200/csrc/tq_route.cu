@@ -107,8 +107,10 @@ __device__ __forceinline__ void permute_cta(const int32_t *topk_ids, int n_route
     __shared__ int32_t warp_sum[kPermWarps], warp_sum_a[kPermWarps];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+    // per-warp count rows in use: warps past the routes of a chunk never write theirs
+    const int wrows = min(kPermWarps, (n_routes + 31) / 32);
     for (int e = tid; e < E; e += kPermThreads) cursor[e] = 0;
-    for (int x = tid; x < kPermWarps * E; x += kPermThreads) wcnt[x] = 0;
+    for (int x = tid; x < wrows * E; x += kPermThreads) wcnt[x] = 0;
     __syncthreads();
     bool bad = false;
     for (int i = tid; i < n_routes; i += kPermThreads) {
@@ -171,6 +173,7 @@ __device__ __forceinline__ void permute_cta(const int32_t *topk_ids, int n_route
 
     const unsigned lt_mask = (1u << lane) - 1u;
     for (int chunk = 0; chunk < n_routes; chunk += kPermThreads) {
+        const int wmax = min(kPermWarps, (min(n_routes - chunk, kPermThreads) + 31) / 32);
         const int i = chunk + tid;
         const int e = i < n_routes ? topk_ids[i] : -1;
         const bool valid = e >= 0 && e < E;
@@ -181,7 +184,7 @@ __device__ __forceinline__ void permute_cta(const int32_t *topk_ids, int n_route
         __syncthreads();
         for (int ee = tid; ee < E; ee += kPermThreads) {
             int run = 0;
-            for (int w = 0; w < kPermWarps; ++w) {
+            for (int w = 0; w < wmax; ++w) {
                 const int v = wcnt[w * E + ee];
                 wcnt[w * E + ee] = run;
                 run += v;
@@ -198,7 +201,7 @@ __device__ __forceinline__ void permute_cta(const int32_t *topk_ids, int n_route
         }
         __syncthreads();
         for (int ee = tid; ee < E; ee += kPermThreads) cursor[ee] += total[ee];
-        for (int x = tid; x < kPermWarps * E; x += kPermThreads) wcnt[x] = 0;
+        for (int x = tid; x < wmax * E; x += kPermThreads) wcnt[x] = 0;
         __syncthreads();
     }
 }
