@@ -610,8 +610,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
 // applies the 128-wide rotation on the way.  rowsum[j] = fp32 sum of the stored fp16
 // values.  With rowscale (the rotated h rows of the down projection) the row is stored
 // as v / 2^e, 2^e = rowscale[j] chosen so that its largest magnitude lies in
-// [2^14, 2^15) (2^e = 1 for a zero row, 2^e >= 2^-112); the row is read twice.  An out-of-range source
-// raises device flag bit 0 and stores zeros.
+// [2^14, 2^15) (2^e = 1 for a zero row, 2^e >= 2^-112); a row of at most KEPT * 128
+// values stays in registers between the max and the store pass, a longer one is read
+// twice.  An out-of-range source raises device flag bit 0 and stores zeros.
+constexpr int kRowsKept = 8;   // 128-value chunks per lane kept in registers (rows of <= 1024)
+
 template <typename T, bool ROTATE>
 __global__ void __launch_bounds__(256) route_rows_kernel(const T *__restrict__ x, int dst_rows, int cols,
                                                          const int32_t *__restrict__ perm, int k, int src_rows,
@@ -631,13 +634,25 @@ __global__ void __launch_bounds__(256) route_rows_kernel(const T *__restrict__ x
             if (ROTATE) fwht128_warp(v, lane);
         }
     };
+    const bool keep = rowscale && cols <= kRowsKept * 128;
+    float kept[kRowsKept][4];
     float inv_scale = 1.f;
     if (rowscale) {
         float m = 0.f;
-        for (int c = 0; c < cols; c += 128) {
-            float v[4];
-            load(c, v);
-            m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fmaxf(fabsf(v[2]), fabsf(v[3])), m));
+        if (keep) {
+#pragma unroll
+            for (int q = 0; q < kRowsKept; ++q)
+                if (q * 128 < cols) {
+                    load(q * 128, kept[q]);
+                    m = fmaxf(fmaxf(fabsf(kept[q][0]), fabsf(kept[q][1])),
+                              fmaxf(fmaxf(fabsf(kept[q][2]), fabsf(kept[q][3])), m));
+                }
+        } else {
+            for (int c = 0; c < cols; c += 128) {
+                float v[4];
+                load(c, v);
+                m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fmaxf(fabsf(v[2]), fabsf(v[3])), m));
+            }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -646,9 +661,7 @@ __global__ void __launch_bounds__(256) route_rows_kernel(const T *__restrict__ x
         if (lane == 0) rowscale[j] = ldexpf(1.f, e);
     }
     float sum = 0.f;
-    for (int c = 0; c < cols; c += 128) {
-        float v[4];
-        load(c, v);
+    auto store = [&](int c, const float (&v)[4]) {
         __half2 lo = __floats2half2_rn(v[0] * inv_scale, v[1] * inv_scale);
         __half2 hi = __floats2half2_rn(v[2] * inv_scale, v[3] * inv_scale);
         const float2 lf = __half22float2(lo), hf = __half22float2(hi);
@@ -657,6 +670,17 @@ __global__ void __launch_bounds__(256) route_rows_kernel(const T *__restrict__ x
         u.x = *reinterpret_cast<uint32_t *>(&lo);
         u.y = *reinterpret_cast<uint32_t *>(&hi);
         *reinterpret_cast<uint2 *>(dst + (size_t)j * cols + c + 4 * lane) = u;
+    };
+    if (keep) {
+#pragma unroll
+        for (int q = 0; q < kRowsKept; ++q)
+            if (q * 128 < cols) store(q * 128, kept[q]);
+    } else {
+        for (int c = 0; c < cols; c += 128) {
+            float v[4];
+            load(c, v);
+            store(c, v);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
@@ -758,23 +782,44 @@ __global__ void __launch_bounds__(256) route_rows_e4m3_kernel(const T *__restric
             if (ROTATE) fwht128_warp(v, lane);
         }
     };
+    // rows of at most kRowsKept * 128 values stay in registers between the two passes
+    const bool keep = cols <= kRowsKept * 128;
+    float kept[kRowsKept][4];
     float m = 0.f;
-    for (int c = 0; c < cols; c += 128) {
-        float v[4];
-        load(c, v);
-        m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fmaxf(fabsf(v[2]), fabsf(v[3])), m));
+    if (keep) {
+#pragma unroll
+        for (int q = 0; q < kRowsKept; ++q)
+            if (q * 128 < cols) {
+                load(q * 128, kept[q]);
+                m = fmaxf(fmaxf(fabsf(kept[q][0]), fabsf(kept[q][1])), fmaxf(fmaxf(fabsf(kept[q][2]), fabsf(kept[q][3])), m));
+            }
+    } else {
+        for (int c = 0; c < cols; c += 128) {
+            float v[4];
+            load(c, v);
+            m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fmaxf(fabsf(v[2]), fabsf(v[3])), m));
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const int e = e4m3_row_exponent(m);
     const float inv = ldexpf(1.f, -e);
     if (lane == 0) rowscale[j] = ldexpf(1.f, e);
-    for (int c = 0; c < cols; c += 128) {
-        float v[4];
-        load(c, v);
+    auto store = [&](int c, float (&v)[4]) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) v[i] *= inv;
         *reinterpret_cast<uint32_t *>(dst + (size_t)j * cols + c + 4 * lane) = e4m3x4_from_f32(v);
+    };
+    if (keep) {
+#pragma unroll
+        for (int q = 0; q < kRowsKept; ++q)
+            if (q * 128 < cols) store(q * 128, kept[q]);
+    } else {
+        for (int c = 0; c < cols; c += 128) {
+            float v[4];
+            load(c, v);
+            store(c, v);
+        }
     }
 }
 
