@@ -394,6 +394,16 @@ struct SwigluFusedSrc {
     }
 };
 
+// Rows whose values are final (already rotated): h[c * 128 + 4 * lane ...] through a
+// generic pointer (shared or global memory); the row argument is ignored.
+struct FinalRowSrc {
+    const float *h;
+    __device__ __forceinline__ void load(int, int c, int lane, float (&v)[4]) const {
+        const float4 f = *reinterpret_cast<const float4 *>(h + (size_t)c * 128 + 4 * lane);
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    }
+};
+
 // One route's split partials (bytes, a multiple of 16) copied from global memory into
 // shared memory with 16-byte cp.async copies through L2, all in flight at once; returns
 // after the CTA's copies have landed.
@@ -881,17 +891,36 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
                 if (e >= 0 && e < L.E) {
                     const int r0 = offsets[e], r1 = offsets[e + 1];
                     // a route's partials (splits x 2 x F fp32) are staged in the idle ring
-                    // buffers when they fit, so that their L2 reads overlap (both passes
-                    // of the quantisation then read shared memory)
+                    // buffers when they fit, so that their L2 reads overlap.  One pass
+                    // computes the final h' values (SwiGLU, signs, rotation) chunk by chunk
+                    // into a row buffer -- shared memory after the staged partials when it
+                    // fits, else over the route's own split-0 gate partials, whose chunk
+                    // has just been read -- and the quantisation reads that buffer twice.
                     const int row_bytes = gu_splits * 2 * L.F * (int)sizeof(float);
+                    const int h_bytes = L.F * (int)sizeof(float);
                     const bool staged = row_bytes <= (int)sizeof(sm_items.buf);
+                    const bool h_smem = staged && row_bytes + h_bytes <= (int)sizeof(sm_items.buf);
                     unsigned char *st = &sm_items.buf[0][0][0];
+                    const int lane = threadIdx.x & 31;
                     for (int r = r0; r < r1; ++r) {
-                        if (staged) stage_row_async(st, gu + (size_t)r * gu_splits * 2 * L.F, row_bytes);
+                        float *grow = gu + (size_t)r * gu_splits * 2 * L.F;
+                        if (staged) stage_row_async(st, grow, row_bytes);
                         const SwigluFusedSrc src{staged ? reinterpret_cast<const float *>(st) : gu, L.F, gu_splits,
                                                  L.sign_gu, staged};
-                        quantize_row<kItemWarps, SwigluFusedSrc, true, 0>(src, r, L.F, L.sign_h, hq, hmeta, s_max,
-                                                                          s_l1, s_sum, s_rsum);
+                        float *hrow = h_smem ? reinterpret_cast<float *>(st + row_bytes) : grow;
+                        for (int c = warp; c < L.F / 128; c += kItemWarps) {
+                            float v[4];
+                            src.load(r, c, lane, v);
+                            if (L.sign_h) {   // input side of the two-sided transform: rotate(signs * h)
+                                const char4 sg = *reinterpret_cast<const char4 *>(L.sign_h + c * 128 + 4 * lane);
+                                v[0] *= sg.x; v[1] *= sg.y; v[2] *= sg.z; v[3] *= sg.w;
+                            }
+                            fwht128_warp(v, lane);
+                            *reinterpret_cast<float4 *>(hrow + (size_t)c * 128 + 4 * lane) = make_float4(v[0], v[1], v[2], v[3]);
+                        }
+                        __syncthreads();
+                        quantize_row<kItemWarps, FinalRowSrc, false, 0>(FinalRowSrc{hrow}, r, L.F, nullptr, hq, hmeta,
+                                                                        s_max, s_l1, s_sum, s_rsum);
                     }
                 }
                 __threadfence();
