@@ -846,8 +846,9 @@ __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
 // expert's routes (h') and raises the expert's ready flag sync[1 + E + a]; a down item
 // waits for its expert's flag.  A CTA only waits for work that a running CTA has already
 // taken (down items come after every gate/up item in the queue), so the waits end; each is
-// bounded all the same.  The arithmetic is that of the separate kernels, so the results
-// are the same bit for bit.  sync[] is cleared by the x' quantisation kernel before.
+// bounded all the same.  The items and the quantisation steps are those of the split form
+// (moe_gemv_items_kernel, quantize_rows_kernel); only the h' row reductions run over this
+// CTA's 4 warps instead of 8.  sync[] is cleared by the x' quantisation kernel before.
 template <int NB>
 __global__ void __launch_bounds__(kItemThreads, NB == 1 ? 5 : 4)
     moe_gemv_fused_kernel(const tq_moe_layer L, const uint16_t *__restrict__ xq, const RowQ *__restrict__ xmeta,
