@@ -43,6 +43,10 @@
  *   - No C++ exception crosses this ABI.  Every entry point is usable inside CUDA-graph
  *     capture: none reads device data on the host or synchronises.
  *   - Sizes of zero (T = 0, rows = 0) are valid no-ops returning TQ_OK.
+ *   - Kernels run on the current device.  The first call of an entry point on a device
+ *     sets its kernels' launch attributes (shared-memory limits) and reads the SM count
+ *     for that device; later calls there reuse them.  Calls from several host threads
+ *     are safe once each device in use has had one call of each entry point.
  */
 #ifndef TRELLIS_MOE_H
 #define TRELLIS_MOE_H

@@ -85,15 +85,37 @@ inline int launch_status() {
     return record_error(cudaGetErrorString(e));
 }
 
-inline int num_sms() {
-    static int cached = 0;
-    if (cached == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&cached, cudaDevAttrMultiProcessorCount, dev);
-        if (cached <= 0) cached = 148;
+// Per-device caches: a process that drives several GPUs configures and sizes each one
+// (kernel attributes apply to the current device); a device id past kMaxDevices is
+// simply never cached.
+constexpr int kMaxDevices = 64;
+inline int current_device() {
+    int d = 0;
+    cudaGetDevice(&d);
+    return d;
+}
+struct PerDeviceFlag {
+    bool done[kMaxDevices] = {};
+    bool get() const {
+        const int d = current_device();
+        return d >= 0 && d < kMaxDevices && done[d];
     }
-    return cached;
+    void set() {
+        const int d = current_device();
+        if (d >= 0 && d < kMaxDevices) done[d] = true;
+    }
+};
+
+inline int num_sms() {
+    static int cached[kMaxDevices] = {};
+    const int dev = current_device();
+    int n = dev >= 0 && dev < kMaxDevices ? cached[dev] : 0;
+    if (n == 0) {
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+        if (dev >= 0 && dev < kMaxDevices) cached[dev] = n;
+    }
+    return n;
 }
 
 // ---------------------------------------------------------------------------- PTX wrappers

@@ -226,12 +226,12 @@ inline size_t enc_ws_bytes(int K, long long tiles) {
 template <int K>
 int run_encode(const float *target, int rows, int cols, uint32_t *bits, uint32_t *tile_cost, uint8_t *ws,
                cudaStream_t s) {
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceFlag configured;
+    if (!configured.get()) {
         if (cudaFuncSetAttribute(trellis_encode_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)enc_smem<K>()) != cudaSuccess)
             return record_cuda_error("cudaFuncSetAttribute");
-        configured = true;
+        configured.set();
     }
     const long long tiles = (long long)(rows / 16) * (cols / 16);
     LaunchScope ls(s, kStageEncode);

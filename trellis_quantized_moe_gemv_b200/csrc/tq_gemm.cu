@@ -1011,10 +1011,10 @@ static int set_gemm_smem() {
 int run_moe_gemm(const tq_moe_layer *L, const __half *x_rot, const int32_t *offsets, const int32_t *perm,
                  const int32_t *active_ids, const int32_t *n_active, int T, int k, float *y_perm, void *ws,
                  cudaStream_t s) {
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceFlag configured;
+    if (!configured.get()) {
         if (set_gemm_smem<false>() || set_gemm_smem<true>()) return TQ_ERR_CUDA;
-        configured = true;
+        configured.set();
     }
     const bool fp8 = L->codebook == TQ_CODEBOOK_PAIR_E4M3;
     const int R = T * k;

@@ -1073,10 +1073,10 @@ template <int NB>
 int run_gemv(const uint32_t *bits, const __half *scales, int K, int rows, int cols, const __half *x, int batch,
              float *y, const GemvWs &w, cudaStream_t s) {
     const size_t smem = sizeof(ItemSmem);
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceFlag configured;
+    if (!configured.get()) {
         if (set_smem(trellis_gemv_kernel<NB>, smem)) return TQ_ERR_CUDA;
-        configured = true;
+        configured.set();
     }
     int st = launch_quantize_rows<false>(RowSrc<__half>{x, cols}, batch, cols, w.xq, w.meta, s, kStageGemvQuant);
     if (st) return st;
@@ -1166,9 +1166,12 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
                  const int32_t *active_ids, const int32_t *n_active, int T, int k, float *y_perm,
                  void *ws, cudaStream_t s) {
     const size_t smem = sizeof(ItemSmem);
-    static bool configured = false;
-    static int resident[3] = {0, 0, 0};   // CTAs per SM of the fused kernel, NB = 1, 2
-    if (!configured) {
+    static PerDeviceFlag configured;
+    static int resident_dev[kMaxDevices][3];   // CTAs per SM of the fused kernel, NB = 1, 2
+    int resident_local[3] = {0, 0, 0};
+    const int dev = current_device();
+    int *resident = dev >= 0 && dev < kMaxDevices ? resident_dev[dev] : resident_local;
+    if (!configured.get()) {
         if (set_smem(moe_gemv_fused_kernel<1>, smem) || set_smem(moe_gemv_fused_kernel<2>, smem) ||
             set_smem(moe_gemv_items_kernel<true, 1>, smem) || set_smem(moe_gemv_items_kernel<false, 1>, smem) ||
             set_smem(moe_gemv_items_kernel<true, 2>, smem) || set_smem(moe_gemv_items_kernel<false, 2>, smem))
@@ -1178,7 +1181,7 @@ int run_moe_gemv(const tq_moe_layer *L, const __half *x_rot, const int32_t *offs
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[2], moe_gemv_fused_kernel<2>, kItemThreads,
                                                           smem) != cudaSuccess)
             return record_cuda_error("cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-        configured = true;
+        configured.set();
     }
     const int routes = T * k;
     const MoeGemvWs w = moe_gemv_ws(L, T, k, ws);

@@ -386,12 +386,12 @@ __global__ void __launch_bounds__(256) permute_inverse_kernel(const int32_t *__r
 static int route_permute_multi(const int32_t *topk_ids, int R, int E, int32_t *counts, int32_t *offsets,
                                int32_t *perm, int32_t *inv, int32_t *active_ids, int32_t *n_active,
                                cudaStream_t s) {
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceFlag configured;
+    if (!configured.get()) {
         if (cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(sizeof(int32_t) * (2 + kPermWarps) * kPermMaxE)) != cudaSuccess)
             return TQ_ERR_CUDA;
-        configured = true;
+        configured.set();
     }
     const int n_blocks = (R + kPermBlockRoutes - 1) / kPermBlockRoutes;
     {
@@ -465,12 +465,12 @@ TQ_API int route_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *
     if ((long long)T * k >= kPermMultiMin)
         return route_permute_multi(topk_ids, T * k, E, counts, offsets, perm, inv, active_ids, n_active, s);
     const size_t smem = permute_smem_bytes(E);
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceFlag configured;
+    if (!configured.get()) {
         if (cudaFuncSetAttribute(route_permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)permute_smem_bytes(kPermMaxE)) != cudaSuccess)
             return TQ_ERR_CUDA;
-        configured = true;
+        configured.set();
     }
     LaunchScope ls(s, kStagePermute);
     launch_chained(route_permute_kernel, 1, kPermThreads, smem, s, topk_ids, T * k, E, counts, offsets, perm, inv,
@@ -493,8 +493,8 @@ TQ_API int route_topk_permute(const float *logits, int T, int E, int k, int32_t 
     }
     cudaStream_t s = (cudaStream_t)stream;
     const size_t smem = permute_smem_bytes(E) + sizeof(int32_t) * (size_t)T * k;
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceFlag configured;
+    if (!configured.get()) {
         const int most = (int)(permute_smem_bytes(kPermMaxE) + sizeof(int32_t) * kFusedRouteMax);
         if (cudaFuncSetAttribute(route_topk_permute_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) !=
                 cudaSuccess ||
@@ -503,7 +503,7 @@ TQ_API int route_topk_permute(const float *logits, int T, int E, int k, int32_t 
             cudaFuncSetAttribute(route_topk_permute_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) !=
                 cudaSuccess)
             return TQ_ERR_CUDA;
-        configured = true;
+        configured.set();
     }
     const int per = (E + 31) / 32;
     LaunchScope ls(s, kStageTopk);
